@@ -1,0 +1,51 @@
+// Host-side declarations shared by the library's translation units: the
+// thread-local error message and the kernel launchers that the C ABI
+// (api.cu) dispatches to.  Launchers assume validated arguments.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/gwb.h"
+
+namespace gwb {
+
+// Records a message for gwb_last_error() and returns `st`.
+gwb_status fail(gwb_status st, const char *fmt, ...);
+
+// Maps the launch error (if any) of the last kernel to a gwb_status.
+gwb_status check_launch(const char *what);
+
+// ------------------------------------------------------------ elementwise kernels
+void launch_qpack_affine(const float *w, int64_t N, int64_t K, int bits, int gs, uint32_t *wq,
+                         uint16_t *scales, uint16_t *biases, cudaStream_t st);
+void launch_dequant_affine(const uint32_t *wq, const uint16_t *scales, const uint16_t *biases, int64_t N,
+                           int64_t K, int bits, int gs, uint16_t *w_out, cudaStream_t st);
+void launch_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
+                         const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *w_out, cudaStream_t st);
+void launch_quant_per_token_i8(const uint16_t *x, int64_t M, int64_t K, int8_t *qx, float *sx,
+                               cudaStream_t st);
+void launch_qpack_sym_i4(const float *w, int64_t N, int64_t K, uint32_t *wq, float *sw, cudaStream_t st);
+
+// ------------------------------------------------------------ GEMV regime (M <= 8)
+// Returns false when the (bits, gs) combination has no GEMV kernel (the caller
+// then uses the tensor-core path).
+bool gemv_affine_supported(int bits, int gs);
+gwb_status launch_gemv_affine(const uint16_t *x, int M, const uint32_t *wq, const uint16_t *scales,
+                              const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
+                              cudaStream_t st);
+gwb_status launch_gemv_gptq(const uint16_t *x, int M, const int32_t *qweight, const uint16_t *scales,
+                            const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
+                            uint16_t *y, cudaStream_t st);
+
+// ------------------------------------------------------------ tensor-core GEMM regime
+gwb_status launch_tc_affine(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
+                            const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
+                            cudaStream_t st);
+gwb_status launch_tc_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
+                          const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
+                          uint16_t *y, cudaStream_t st);
+gwb_status launch_tc_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
+                          int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
+gwb_status read_and_clear_device_error(cudaStream_t st, unsigned int *flag);
+
+}  // namespace gwb

@@ -1,0 +1,522 @@
+// Tensor-core (tcgen05) GEMM regime of the fused dequant + matmul, for
+//   * the MLX affine layout (bf16 activations, kind::f16 with bf16 operands),
+//   * the GPTQ layout (fp16 activations, kind::f16 with fp16 operands),
+//   * W4A8 (int8 activations x symmetric int4 weights, kind::i8, s32).
+//
+// The problem is computed transposed ("swap AB"): the tensor core's M side is
+// 128 output features (rows of W), its N side is BT tokens.  One CTA owns a
+// 128 x BT output tile and the whole K loop:
+//
+//   warp 0      TMA producer: per K step, the activation tile (BT x BK, 128-byte
+//               swizzled, zero-filled past M/K) and the packed weight tile
+//               (raw words) into a ring of STAGES shared-memory stages.
+//   warp 1      TMEM allocation and the single MMA-issuing thread: waits for the
+//               dequantized A tile and the activation tile of a stage, issues
+//               BK/16 (BK/32 for int8) tcgen05.mma into the TMEM accumulator and
+//               commits the stage back to the producer.
+//   warps 2-9   dequantizers: unpack the stage's raw words in registers, apply
+//               the group scale / bias (or zero), and store the 128 x BK A tile
+//               in the same 128-byte-swizzled K-major layout TMA produces, then
+//               signal the MMA thread; after the K loop they drain TMEM with
+//               tcgen05.ld and write the output tile.
+//
+// Every mbarrier wait is bounded (see ptx.cuh); on a timeout the CTA stops
+// issuing work, drains what it issued, frees its TMEM and exits.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gwb {
+namespace {
+
+constexpr int kTcThreads = 320;
+constexpr int kDqThreads = 256;
+constexpr int kTileN = 128;  // output features per CTA (tensor-core M)
+constexpr int kMaxSmem = 232448;
+
+enum class Fmt { Affine, Gptq, I8 };
+
+struct TcArgs {
+  int M, N, K, gs;
+  const uint16_t *scales;   // affine: bf16 [N, K/gs];   gptq: fp16 [K/gs, N]
+  const uint16_t *biases;   // affine: bf16 [N, K/gs]
+  const int32_t *qzeros;    // gptq: [K/gs, N/8]
+  const int32_t *g_idx;     // gptq: [K] or null
+  const float *sx, *sw;     // i8: per-token / per-channel scales
+  uint16_t *y;              // bf16 (affine, i8) or fp16 (gptq) [M, N]
+  int32_t *acc;             // i8: optional int32 [M, N]
+};
+
+template <Fmt F, int BITS>
+struct Traits;
+template <int BITS>
+struct Traits<Fmt::Affine, BITS> {
+  static constexpr int BK = 64;                       // bf16: 64 elements = 128 bytes per row
+  static constexpr int RAW_BYTES = kTileN * BK * BITS / 8;
+  static constexpr int NMMA = BK / 16;
+};
+template <>
+struct Traits<Fmt::Gptq, 4> {
+  static constexpr int BK = 64;
+  static constexpr int RAW_BYTES = (BK / 8) * kTileN * 4;
+  static constexpr int NMMA = BK / 16;
+};
+template <>
+struct Traits<Fmt::I8, 4> {
+  static constexpr int BK = 128;                      // int8: 128 elements = 128 bytes per row
+  static constexpr int RAW_BYTES = kTileN * BK / 2;
+  static constexpr int NMMA = BK / 32;
+};
+
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
+  return (a & mask) | magic;  // one LOP3
+}
+__device__ __forceinline__ float bf16_val(uint16_t h) { return __uint_as_float(static_cast<uint32_t>(h) << 16); }
+
+__device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t *>(&v); }
+__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t u) { return *reinterpret_cast<__nv_bfloat162 *>(&u); }
+__device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t *>(&v); }
+__device__ __forceinline__ __half2 as_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+// Byte offset of 16-byte chunk `c` of row `r` in a 128-byte-swizzled K-major tile.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// ---------------------------------------------------------------- dequantizers
+// Affine, 4-bit: one word = 8 consecutive k = one 16-byte chunk of bf16.
+// Pair p (k = 2p, 2p+1) sits in byte p of the word; PRMT moves the low nibble
+// of byte p of w and of w>>4 into the two halves, and OR-ing 0x4300 makes the
+// exact bf16 value 128 + code.
+__device__ __forceinline__ uint4 dq_affine4(uint32_t w, __nv_bfloat162 s2, __nv_bfloat162 b2) {
+  const uint32_t t = w >> 4;
+  const __nv_bfloat162 m128 = __floats2bfloat162_rn(128.0f, 128.0f);
+  uint32_t o[4];
+#pragma unroll
+  for (int p = 0; p < 4; p++) {
+    const uint32_t pr = lop_and_or(__byte_perm(w, t, p | ((4 + p) << 8)), 0x000F000Fu, 0x43004300u);
+    o[p] = bf162_bits(__hfma2(__hsub2(as_bf162(pr), m128), s2, b2));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Affine, 2-bit: one word = 16 consecutive k = two chunks.  Pair p (k = 2p,
+// 2p+1) is nibble p; its two codes land at bits 0-1 (value 128 + q) and bits
+// 2-3 of the high half (value 128 + 4q), so the high half uses scale s/4.
+__device__ __forceinline__ void dq_affine2(uint32_t w, __nv_bfloat162 s2q, __nv_bfloat162 b2, uint4 &c0, uint4 &c1) {
+  const uint32_t t = w >> 4;
+  const __nv_bfloat162 m128 = __floats2bfloat162_rn(128.0f, 128.0f);
+  uint32_t o[8];
+#pragma unroll
+  for (int p = 0; p < 8; p++) {
+    const uint32_t idx = (p & 1) ? (4 + (p >> 1)) : (p >> 1);
+    const uint32_t pr = lop_and_or(__byte_perm(w, t, idx | (idx << 8)), 0x000C0003u, 0x43004300u);
+    o[p] = bf162_bits(__hfma2(__hsub2(as_bf162(pr), m128), s2q, b2));
+  }
+  c0 = make_uint4(o[0], o[1], o[2], o[3]);
+  c1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// Affine, 8-bit: codes above 127 do not fit the bf16 mantissa trick, so each
+// byte becomes the fp32 2^23 + code (exact), then fmaf(code, s, b) in fp32 and
+// a paired round to bf16.  Two words = one chunk.
+__device__ __forceinline__ uint4 dq_affine8(uint32_t w0, uint32_t w1, float s, float b) {
+  uint32_t o[4];
+#pragma unroll
+  for (int h = 0; h < 2; h++) {
+    const uint32_t w = h ? w1 : w0;
+#pragma unroll
+    for (int p = 0; p < 2; p++) {
+      const float lo = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | (2 * p))) - 8388608.0f;
+      const float hi = __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540 | (2 * p + 1))) - 8388608.0f;
+      o[2 * h + p] = bf162_bits(__floats2bfloat162_rn(fmaf(lo, s, b), fmaf(hi, s, b)));
+    }
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// GPTQ: one qweight word = 8 consecutive k of one out-feature = one chunk of
+// fp16.  (1024 + q) - (1024 + zero) is exact, and the product with the fp16
+// scale is the single rounding gptq_dequant also performs.
+__device__ __forceinline__ uint4 dq_gptq(uint32_t w, const uint32_t (&z2)[4], const uint32_t (&s2)[4]) {
+  const uint32_t t = w >> 4;
+  uint32_t o[4];
+#pragma unroll
+  for (int p = 0; p < 4; p++) {
+    const uint32_t pr = lop_and_or(__byte_perm(w, t, p | ((4 + p) << 8)), 0x000F000Fu, 0x64006400u);
+    o[p] = h2_bits(__hmul2(__hsub2(as_h2(pr), as_h2(z2[p])), as_h2(s2[p])));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Symmetric int4 -> int8: each nibble is placed in the high half of its byte,
+// i.e. the byte holds 16 * code as a signed int8; the accumulator is divided
+// by 16 (exactly) in the epilogue.  Two words = one 16-byte chunk.
+__device__ __forceinline__ uint2 dq_i4(uint32_t w) {
+  const uint32_t lo = (w << 4) & 0xF0F0F0F0u;  // codes 0,2,4,6
+  const uint32_t hi = w & 0xF0F0F0F0u;         // codes 1,3,5,7
+  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+}
+
+// ---------------------------------------------------------------- the kernel
+template <Fmt F, int BITS, int BT, int STAGES>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    k_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const TcArgs args) {
+  using T = Traits<F, BITS>;
+  constexpr int BK = T::BK;
+  constexpr int B_BYTES = BT * 128;
+  constexpr int A_BYTES = kTileN * 128;
+  constexpr int STAGE = B_BYTES + A_BYTES + T::RAW_BYTES;
+  constexpr uint32_t NCOLS = BT < 32 ? 32 : BT;
+  constexpr uint32_t IDESC = (F == Fmt::I8) ? make_idesc(2, 1, kTileN, BT)
+                             : (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN, BT)
+                                                : make_idesc(1, 1, kTileN, BT);
+
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *base = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(base + STAGES * STAGE);
+  uint64_t *afull = full + STAGES;
+  uint64_t *empty = afull + STAGES;
+  uint64_t *accf = empty + STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accf + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kTileN, m0 = blockIdx.y * BT;
+  const int nk = (args.K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&afull[s], kDqThreads / 32);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, NCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nk; i++) {
+        const int s = i % STAGES, r = i / STAGES;
+        if (!mbar_wait(&empty[s], (r & 1) ^ 1)) { *abort_flag = 1; break; }
+        unsigned char *st = base + s * STAGE;
+        mbar_arrive_expect_tx(&full[s], B_BYTES + T::RAW_BYTES);
+        tma_load_2d(st, &tm_x, i * BK, m0, &full[s]);
+        if constexpr (F == Fmt::Gptq) tma_load_2d(st + B_BYTES + A_BYTES, &tm_w, n0, i * (BK / 8), &full[s]);
+        else tma_load_2d(st + B_BYTES + A_BYTES, &tm_w, i * (BK * BITS / 32), n0, &full[s]);
+        issued = i + 1;
+      }
+      // Drain: every issued copy has landed before the CTA can exit.
+      for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; i++)
+        mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int done = 0;
+      for (int i = 0; i < nk; i++) {
+        const int s = i % STAGES, ph = (i / STAGES) & 1;
+        if (*abort_flag) break;
+        if (!mbar_wait(&afull[s], ph) || !mbar_wait(&full[s], ph)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        unsigned char *st = base + s * STAGE;
+        const uint32_t a0 = smem_u32(st + B_BYTES), b0 = smem_u32(st);
+#pragma unroll
+        for (int kk = 0; kk < T::NMMA; kk++) {
+          const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
+          if constexpr (F == Fmt::I8) umma_i8(tmem, ad, bd, IDESC, (i | kk) != 0);
+          else umma_f16(tmem, ad, bd, IDESC, (i | kk) != 0);
+        }
+        umma_commit(&empty[s]);
+        done = i + 1;
+      }
+      umma_commit(accf);
+      // Wait for the commits' arrivals so no asynchronous arrive targets this
+      // CTA's shared memory after it exits.
+      for (int i = done - STAGES < 0 ? 0 : done - STAGES; i < done; i++)
+        mbar_wait(&empty[i % STAGES], (i / STAGES) & 1);
+    }
+  } else {
+    // ------------------------------------------------------------ dequantizers
+    const int d = threadIdx.x - 64;
+    const int r = d & (kTileN - 1), h = d >> 7;   // tile row, half of the K step
+    const int n = n0 + r;
+    const int nc = n < args.N ? n : args.N - 1;    // clamped row for scale loads
+    for (int i = 0; i < nk; i++) {
+      const int s = i % STAGES, ph = (i / STAGES) & 1;
+      // Scale data for this thread's half step (loaded before the wait so the
+      // latency overlaps it).
+      const int kh = i * BK + h * (BK / 2);        // first k of this half step
+      float sf = 0.f, bfv = 0.f;
+      uint32_t z2[4], s2[4];
+      if constexpr (F == Fmt::Affine) {
+        const int G = args.K / args.gs;
+        int g = kh / args.gs;
+        g = g < G ? g : G - 1;
+        sf = bf16_val(__ldg(args.scales + (int64_t)nc * G + g));
+        bfv = bf16_val(__ldg(args.biases + (int64_t)nc * G + g));
+      } else if constexpr (F == Fmt::Gptq) {
+        if (args.g_idx == nullptr) {
+          const int G = args.K / args.gs;
+          int g = kh / args.gs;
+          g = g < G ? g : G - 1;
+          const uint32_t sv = __ldg(args.scales + (int64_t)g * args.N + nc);
+          const uint32_t zw = (uint32_t)__ldg(args.qzeros + (int64_t)g * (args.N / 8) + nc / 8);
+          const uint32_t zv = 0x6400u | (((zw >> ((nc % 8) * 4)) & 0xFu) + 1u);
+#pragma unroll
+          for (int p = 0; p < 4; p++) { s2[p] = sv | (sv << 16); z2[p] = zv | (zv << 16); }
+        }
+      }
+      if (*abort_flag) break;
+      if (!mbar_wait(&full[s], ph)) { *abort_flag = 1; break; }
+      unsigned char *st = base + s * STAGE;
+      unsigned char *A = st + B_BYTES;
+      const unsigned char *R = st + B_BYTES + A_BYTES;
+      if constexpr (F == Fmt::Affine && BITS == 4) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(R + (r * 8 + h * 4) * 4);
+        const __nv_bfloat162 s2b = __floats2bfloat162_rn(sf, sf), b2b = __floats2bfloat162_rn(bfv, bfv);
+        const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+          *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + j)) = dq_affine4(wv[j], s2b, b2b);
+      } else if constexpr (F == Fmt::Affine && BITS == 2) {
+        const uint2 raw = *reinterpret_cast<const uint2 *>(R + (r * 4 + h * 2) * 4);
+        const __nv_bfloat162 s2q = __floats2bfloat162_rn(sf, sf * 0.25f), b2b = __floats2bfloat162_rn(bfv, bfv);
+        uint4 c0, c1;
+        dq_affine2(raw.x, s2q, b2b, c0, c1);
+        *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 0)) = c0;
+        *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 1)) = c1;
+        dq_affine2(raw.y, s2q, b2b, c0, c1);
+        *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 2)) = c0;
+        *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 3)) = c1;
+      } else if constexpr (F == Fmt::Affine && BITS == 8) {
+        const uint4 *rp = reinterpret_cast<const uint4 *>(R + (r * 16 + h * 8) * 4);
+        const uint4 ra = rp[0], rb = rp[1];
+        *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 0)) = dq_affine8(ra.x, ra.y, sf, bfv);
+        *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 1)) = dq_affine8(ra.z, ra.w, sf, bfv);
+        *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 2)) = dq_affine8(rb.x, rb.y, sf, bfv);
+        *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 3)) = dq_affine8(rb.z, rb.w, sf, bfv);
+      } else if constexpr (F == Fmt::Gptq) {
+        const uint32_t *Rw = reinterpret_cast<const uint32_t *>(R);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const int kq = 4 * h + j;                  // k-octet within the step = chunk index
+          const uint32_t w = Rw[kq * kTileN + r];
+          if (args.g_idx != nullptr) {
+#pragma unroll
+            for (int p = 0; p < 4; p++) {
+              uint32_t sv[2], zv[2];
+#pragma unroll
+              for (int e = 0; e < 2; e++) {
+                const int k = i * BK + kq * 8 + 2 * p + e;
+                const int g = k < args.K ? __ldg(args.g_idx + k) : 0;
+                sv[e] = __ldg(args.scales + (int64_t)g * args.N + nc);
+                const uint32_t zw = (uint32_t)__ldg(args.qzeros + (int64_t)g * (args.N / 8) + nc / 8);
+                zv[e] = 0x6400u | (((zw >> ((nc % 8) * 4)) & 0xFu) + 1u);
+              }
+              s2[p] = sv[0] | (sv[1] << 16);
+              z2[p] = zv[0] | (zv[1] << 16);
+            }
+          }
+          *reinterpret_cast<uint4 *>(A + sw128_off(r, kq)) = dq_gptq(w, z2, s2);
+        }
+      } else {  // I8
+        const uint4 *rp = reinterpret_cast<const uint4 *>(R + (r * 16 + h * 8) * 4);
+        const uint4 ra = rp[0], rb = rp[1];
+        const uint32_t wv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const uint2 lo = dq_i4(wv[2 * j]), hi = dq_i4(wv[2 * j + 1]);
+          *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + j)) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[s]);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (!*abort_flag && mbar_wait(accf, 0)) {
+      tc_fence_after();
+      const int q = warp & 3, eh = (warp - 2) >> 2;
+      const int row = n0 + 32 * q + lane;
+      for (int ch = eh; ch < BT / 16; ch += 2) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ch * 16), v);
+        tmem_ld_wait();
+        if (row < args.N) {
+          float swn = 0.f;
+          if constexpr (F == Fmt::I8) swn = args.sw[row];
+#pragma unroll
+          for (int j = 0; j < 16; j++) {
+            const int m = m0 + ch * 16 + j;
+            if (m < args.M) {
+              const int64_t o = (int64_t)m * args.N + row;
+              if constexpr (F == Fmt::I8) {
+                const int a = static_cast<int>(v[j]) >> 4;   // the tensor core summed 16 * code
+                if (args.acc) args.acc[o] = a;
+                if (args.y)
+                  args.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn((float)a * (args.sx[m] * swn)));
+              } else if constexpr (F == Fmt::Gptq) {
+                args.y[o] = __half_as_ushort(__float2half_rn(__uint_as_float(v[j])));
+              } else {
+                args.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+              }
+            }
+          }
+        }
+      }
+    } else {
+      *abort_flag = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, NCOLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+gwb_status make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return fail(GWB_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GWB_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return GWB_OK;
+}
+
+template <Fmt F, int BITS, int BT>
+constexpr int stages_for() {
+  constexpr int stage = BT * 128 + kTileN * 128 + Traits<F, BITS>::RAW_BYTES;
+  constexpr int s = (kMaxSmem - 2048) / stage;
+  return s > 6 ? 6 : s;
+}
+
+template <Fmt F, int BITS, int BT>
+gwb_status run_tc(const CUtensorMap &tx, const CUtensorMap &tw, const TcArgs &a, cudaStream_t st) {
+  constexpr int STAGES = stages_for<F, BITS, BT>();
+  static_assert(STAGES >= 2, "shared memory too small");
+  constexpr int stage = BT * 128 + kTileN * 128 + Traits<F, BITS>::RAW_BYTES;
+  const size_t smem = (size_t)STAGES * stage + 1024 + 256;
+  auto kern = k_tc<F, BITS, BT, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  dim3 grid((a.N + kTileN - 1) / kTileN, (a.M + BT - 1) / BT);
+  kern<<<grid, kTcThreads, smem, st>>>(tx, tw, a);
+  return check_launch("tensor-core GEMM");
+}
+
+int pick_bt(int64_t M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+
+// Builds the activation tensor map for the chosen token tile and launches.
+template <Fmt F, int BITS>
+gwb_status dispatch_bt(int64_t M, const void *xptr, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
+                       const TcArgs &a, cudaStream_t st) {
+  const int BT = pick_bt(M);
+  CUtensorMap tx;
+  const int bk_elems = 128 / xelem;
+  gwb_status s = make_map(&tx, xdt, xptr, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * xelem, bk_elems,
+                          (uint32_t)BT, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != GWB_OK) return s;
+  switch (BT) {
+    case 16: return run_tc<F, BITS, 16>(tx, tw, a, st);
+    case 32: return run_tc<F, BITS, 32>(tx, tw, a, st);
+    case 64: return run_tc<F, BITS, 64>(tx, tw, a, st);
+    case 128: return run_tc<F, BITS, 128>(tx, tw, a, st);
+    default: return run_tc<F, BITS, 256>(tx, tw, a, st);
+  }
+}
+
+}  // namespace
+
+gwb_status launch_tc_affine(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
+                            const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
+                            cudaStream_t st) {
+  TcArgs a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
+  a.scales = scales; a.biases = biases; a.y = y;
+  CUtensorMap tw;
+  const uint64_t words = (uint64_t)K * bits / 32;
+  gwb_status s = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, (uint64_t)N, words * 4,
+                          (uint32_t)(64 * bits / 32), (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != GWB_OK) return s;
+  if (bits == 4) return dispatch_bt<Fmt::Affine, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, a, st);
+  if (bits == 8) return dispatch_bt<Fmt::Affine, 8>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, a, st);
+  return dispatch_bt<Fmt::Affine, 2>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, a, st);
+}
+
+gwb_status launch_tc_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
+                          const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
+                          uint16_t *y, cudaStream_t st) {
+  TcArgs a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
+  a.scales = scales; a.qzeros = qzeros; a.g_idx = g_idx; a.y = y;
+  CUtensorMap tw;
+  gwb_status s = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, (uint64_t)N, (uint64_t)(K / 8),
+                          (uint64_t)N * 4, (uint32_t)kTileN, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != GWB_OK) return s;
+  return dispatch_bt<Fmt::Gptq, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, tw, a, st);
+}
+
+gwb_status launch_tc_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
+                          int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st) {
+  TcArgs a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = 0;
+  a.sx = sx; a.sw = sw; a.y = y; a.acc = acc;
+  CUtensorMap tw;
+  gwb_status s = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, (uint64_t)(K / 8), (uint64_t)N,
+                          (uint64_t)(K / 8) * 4, 16u, (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != GWB_OK) return s;
+  return dispatch_bt<Fmt::I8, 4>(M, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, a, st);
+}
+
+gwb_status read_and_clear_device_error(cudaStream_t st, unsigned int *flag) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(flag, g_device_error, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "device error check: %s", cudaGetErrorString(e));
+  return GWB_OK;
+}
+
+}  // namespace gwb

@@ -1,0 +1,176 @@
+/*
+ * gwb.h -- C ABI of the group-wise low-bit linear-layer library for NVIDIA B200
+ * (sm_100a).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or retains them.  Tensors are dense and row-major
+ *    with the shapes stated per call; no strides are taken.
+ *  - bf16 and fp16 values are passed as their raw 16-bit patterns (uint16_t).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
+ *    validates its arguments synchronously, on the host, before launching
+ *    anything; on success the work is enqueued on `stream` and the call returns
+ *    without synchronizing.  A call that returns an error has launched nothing.
+ *  - Pointers must be 16-byte aligned (GWB_ERR_ALIGN otherwise); optional
+ *    pointers that may be NULL say so.
+ *  - The return value is a gwb_status; gwb_last_error() gives a readable
+ *    message for the calling thread's most recent failure.
+ *  - Device-side waits inside the tensor-core kernels are bounded; a wait that
+ *    gives up records GWB_ERR_TIMEOUT in a device flag that
+ *    gwb_check_device_error() reads and clears.
+ *  - Quantized weights follow three layouts (bits b, group size gs):
+ *      MLX affine   wq      uint32 [N, K*b/32]  codes packed along K, lowest bits
+ *                                              = lowest column
+ *                   scales  bf16   [N, K/gs]
+ *                   biases  bf16   [N, K/gs]    w[n,k] = code*scale + bias
+ *      GPTQ int4    qweight int32  [K/8, N]     packed along IN (K)
+ *                   scales  fp16   [K/gs, N]
+ *                   qzeros  int32  [K/gs, N/8]  packed along OUT, stores zero-1
+ *                   g_idx   int32  [K]          optional group of each in-feature
+ *      sym int4     wq      uint32 [N, K/8]     two's-complement nibbles along K
+ *                   sw      fp32   [N]          w[n,k] = code*sw[n]
+ *    A linear layer computes y[M,N] = x[M,K] . W^T, with W stored [N = out, K = in].
+ *
+ * Sources (page title, then section): "MLX" = metrale_gpu_runtime/mlx_int8.rs
+ * module doc "Layout" and the Hugging Face transformers "Metal" quantization
+ * page; "GPTQ" = TinyGPT "Quantization Expansion", section 1 "GPTQReader",
+ * "Format" and dequant recipe; "QAT" = the same page, section 4, "Fake-quant +
+ * STE"; "W4A8" = executorch PR #24467 "mlx::int8_int4_gemm".
+ */
+#ifndef GWB_H
+#define GWB_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gwb_status {
+    GWB_OK = 0,
+    GWB_ERR_INVALID_ARG = 1,  /* NULL where a tensor is required, negative size, ...     */
+    GWB_ERR_SHAPE = 2,        /* sizes that the layout cannot hold (K % gs, N % 8, ...)  */
+    GWB_ERR_UNSUPPORTED = 3,  /* bits not in {2,4,8}, group size not in {32,64,128}, ... */
+    GWB_ERR_ALIGN = 4,        /* a pointer is not 16-byte aligned                        */
+    GWB_ERR_CUDA = 5,         /* a CUDA runtime/driver call or kernel launch failed      */
+    GWB_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up                      */
+} gwb_status;
+
+/* Message for the calling thread's most recent non-GWB_OK return ("" if none).
+ * The string is owned by the library and valid until the next call on this thread. */
+const char *gwb_last_error(void);
+
+/* Library version string. */
+const char *gwb_version(void);
+
+/* Synchronizes `stream`, then reads and clears the device error flag that the
+ * bounded waits of the tensor-core kernels set.  Returns GWB_OK when no wait
+ * gave up since the last check, GWB_ERR_TIMEOUT otherwise, GWB_ERR_CUDA when
+ * the synchronization itself failed. */
+gwb_status gwb_check_device_error(void *stream);
+
+/* ------------------------------------------------------------------ MLX affine */
+
+/* qpack_affine -- per-group min/max affine quantization and packing (MLX layout).
+ * For each row n and group g of `group_size` consecutive columns, in fp32 with
+ * one IEEE rounding per step:
+ *   mn = min, mx = max of the group;  s = (mx - mn) / (2^bits - 1);
+ *   code = clip(round_half_even((w - mn) / s), 0, 2^bits - 1)   (0 when s == 0)
+ * scales[n,g] = bf16_rne(s), biases[n,g] = bf16_rne(mn); codes are packed
+ * 32/bits per uint32, lowest bits = lowest column.
+ * Source: MLX (affine scheme, packed uint32 layout, bf16 scales/biases).
+ *   w       fp32  [N, K]             input weights (finite values)
+ *   wq      u32   [N, K*bits/32]     output
+ *   scales  bf16  [N, K/group_size]  output
+ *   biases  bf16  [N, K/group_size]  output
+ * bits in {2,4,8}; group_size in {32,64,128}; K % group_size == 0.
+ * Results are bit-exact and independent of the launch configuration. */
+gwb_status gwb_qpack_affine(const float *w, int64_t N, int64_t K, int bits, int group_size,
+                            uint32_t *wq, uint16_t *scales, uint16_t *biases, void *stream);
+
+/* dequant_affine -- w_out[n,k] = bf16_rne(fp32(code*scale + bias)): the exact
+ * value rounded once to fp32, then to bf16.  Source: MLX (the dequant formula
+ * w[r,c] = byte*scales[r,c/G] + biases[r,c/G] and its dequantize_to output).
+ *   w_out   bf16  [N, K]             output
+ * Same layout arguments and limits as gwb_qpack_affine. */
+gwb_status gwb_dequant_affine(const uint32_t *wq, const uint16_t *scales, const uint16_t *biases,
+                              int64_t N, int64_t K, int bits, int group_size,
+                              uint16_t *w_out, void *stream);
+
+/* qmm_affine -- fused dequant + matmul (the affine_qmm_t operation):
+ *   y[m,n] = sum_k x[m,k] * (code(n,k)*scale[n,k/gs] + bias[n,k/gs])
+ * with fp32 accumulation and a bf16 (round-to-nearest-even) result.
+ * Source: MLX (Hugging Face "Metal" quantization: fused dequant + matmul
+ * affine_qmm_t; mlx_int8.rs gemv / gemm docs for y = W x and Y = X W^T).
+ *   x   bf16  [M, K]   activations;   y   bf16  [M, N]   output
+ * M >= 1.  M <= 8 runs the memory-bound split-K GEMV regime; larger M runs the
+ * tensor-core (tcgen05) GEMM regime.  For bits == 2 the packed row length
+ * K/16 words must be a multiple of 4 (K % 64 == 0).
+ * The result is deterministic for a given shape (no atomics), but not bitwise
+ * equal to any particular summation order. */
+gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
+                          const uint16_t *biases, int64_t N, int64_t K, int bits, int group_size,
+                          uint16_t *y, void *stream);
+
+/* ------------------------------------------------------------------ GPTQ */
+
+/* gptq_dequant -- the GPTQ dequant recipe, one weight at a time:
+ *   int4 = (qweight[i/8, o] >> ((i%8)*4)) & 0xF
+ *   g    = g_idx ? g_idx[i] : i / group_size
+ *   zero = ((qzeros[g, o/8] >> ((o%8)*4)) & 0xF) + 1        (the "+1" convention)
+ *   w_out[o, i] = fp16_rne(scales[g, o] * (int4 - zero))     (exact product, one rounding)
+ * Source: GPTQ (format and dequant recipe).
+ *   qweight i32 [K/8, N], scales fp16 [K/gs, N], qzeros i32 [K/gs, N/8],
+ *   g_idx   i32 [K] or NULL, w_out fp16 [N, K] (out-features major, as HF stores W)
+ * K % 8 == 0, N % 8 == 0, K % group_size == 0, group_size in {32,64,128}.
+ * g_idx values must lie in [0, K/group_size); they are not checked (an
+ * out-of-range value reads outside `scales`/`qzeros`). */
+gwb_status gwb_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
+                            const int32_t *g_idx, int64_t K, int64_t N, int group_size,
+                            uint16_t *w_out, void *stream);
+
+/* gptq_qmm -- y[m,o] = sum_i x[m,i] * W[o,i] with W as gwb_gptq_dequant defines
+ * it (each weight rounded to fp16, as the dequantized checkpoint would hold it),
+ * fp32 accumulation, fp16 result.
+ *   x  fp16 [M, K],  y  fp16 [M, N].   Limits as gwb_gptq_dequant; M >= 1. */
+gwb_status gwb_gptq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
+                        const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N,
+                        int group_size, uint16_t *y, void *stream);
+
+/* ------------------------------------------------------------------ W4A8 */
+
+/* quant_per_token_i8 -- dynamic symmetric per-token int8 (qMax = 127), fp32:
+ *   amax = max_k |x[m,k]|;  sx[m] = amax / 127;
+ *   qx[m,k] = clip(round_half_even(x[m,k] / sx[m]), -127, 127)   (0 when amax == 0)
+ * Source: W4A8 (dynamic symmetric per-token int8 activations) with the
+ * symmetric quantizer of QAT.
+ *   x bf16 [M, K] (finite), qx int8 [M, K], sx fp32 [M].   Bit-exact. */
+gwb_status gwb_quant_per_token_i8(const uint16_t *x, int64_t M, int64_t K, int8_t *qx, float *sx,
+                                  void *stream);
+
+/* qpack_sym_i4 -- symmetric per-output-channel int4 weights (qMax = 7):
+ *   sw[n] = max_k |w[n,k]| / 7;  code = clip(round_half_even(w / sw[n]), -8, 7)
+ * (0 when sw == 0), stored as two's-complement nibbles, 8 per uint32 along K,
+ * lowest nibble = lowest k.  Source: QAT (per-row symmetric scale, qMax) and W4A8.
+ *   w fp32 [N, K] (finite), wq u32 [N, K/8], sw fp32 [N].  K % 32 == 0.  Bit-exact. */
+gwb_status gwb_qpack_sym_i4(const float *w, int64_t N, int64_t K, uint32_t *wq, float *sw,
+                            void *stream);
+
+/* gemm_i8i4 -- int8 activations x int4 weights with int32 accumulation:
+ *   acc[m,n] = sum_k qx[m,k] * code(n,k)                 (exact int32)
+ *   y[m,n]   = bf16_rne(fp32(acc[m,n]) * (sx[m] * sw[n]))
+ * Source: W4A8 (INT8 x INT4 -> INT32, per-token and per-channel scales).
+ *   qx int8 [M, K], sx fp32 [M], wq u32 [N, K/8], sw fp32 [N]
+ *   y   bf16  [M, N] or NULL;  acc int32 [M, N] or NULL (at least one non-NULL)
+ * K % 32 == 0 and K <= 131072 (so that the tensor-core partial sums, which
+ * carry each int4 code multiplied by 16, stay inside int32).  The int32 result
+ * is exact; y is a single rounding of its fp32 product. */
+gwb_status gwb_gemm_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq,
+                         const float *sw, int64_t N, int64_t K, uint16_t *y, int32_t *acc,
+                         void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GWB_H */

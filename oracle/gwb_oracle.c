@@ -134,6 +134,14 @@ void orc_pack_affine(const int32_t *codes, int64_t N, int64_t K, int bits, uint3
             wq[n * words + k / pw] |= ((uint32_t)codes[n * K + k] & mask) << ((k % pw) * bits);
 }
 
+/* Comparison under the total order of finite floats in which -0 < +0, so that
+ * a group's min and max are unique bit patterns (the pages do not say which
+ * zero a group holding both would report; this is the reading taken). */
+static int less_total(float a, float b)
+{
+    return a < b || (a == b && signbit(a) && !signbit(b));
+}
+
 /* Per-group min/max affine quantizer, in fp32 with one rounding per step:
  *   mn = min, mx = max over the group's gs columns of row n
  *   s  = (mx - mn) / (2^b - 1)
@@ -154,8 +162,8 @@ void orc_qpack_affine(const float *w, int64_t N, int64_t K, int bits, int gs,
             const float *row = w + n * K + g * gs;
             float mn = row[0], mx = row[0];
             for (int j = 1; j < gs; j++) {
-                if (row[j] < mn) mn = row[j];
-                if (row[j] > mx) mx = row[j];
+                if (less_total(row[j], mn)) mn = row[j];
+                if (less_total(mx, row[j])) mx = row[j];
             }
             float range = mx - mn;
             float s = range / (float)qmax;

@@ -1,0 +1,287 @@
+"""GPU parity: the CUDA library (through the C ABI) against the CPU oracle on
+the same seeded inputs.
+
+Integer / byte work (packing, unpacking, dequantized weights, per-token int8,
+W4A8 int32 accumulators) must be bit-exact; float matmul outputs must meet the
+tolerance in tests/tol.py.  Small cases span several tiles and ragged tails in
+N, M and K; the full-size cases use the workloads' shapes, with the oracle
+evaluated on sampled output rows where all rows would take too long.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gwb_synth as synth
+import oracle
+from tol import check_float
+
+gwb = pytest.importorskip("group_wise_bit_b200")
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _np16(t):
+    return synth.bits16(t.cpu())
+
+
+def _words(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def _rows(M, N, K, seed=0, budget=3e8):
+    """All rows when the oracle finishes quickly, else the first, the last and a
+    seeded sample of rows in between (about `budget` multiply-adds in total)."""
+    if M * N * K <= budget or M <= 2:
+        return None
+    n = int(max(0, min(M - 2, budget // (N * K) - 2)))
+    r = np.random.default_rng(seed).choice(np.arange(1, M - 1), size=n, replace=False) if n else []
+    return np.unique(np.concatenate([[0, M - 1], r]).astype(np.int64))
+
+
+def _affine_max_w(sc, bi, bits):
+    s = oracle.bf16_array_to_f64(sc)
+    b = oracle.bf16_array_to_f64(bi)
+    return float(np.max(np.maximum(np.abs(b), np.abs(b + ((1 << bits) - 1) * s))))
+
+
+class Affine:
+    """A quantized MLX-affine linear built on both sides from one fp32 weight."""
+
+    def __init__(self, N, K, bits, gs, seed=0):
+        self.N, self.K, self.bits, self.gs = N, K, bits, gs
+        w = synth.weights(N, K, seed=seed)
+        self.wq_o, self.sc_o, self.bi_o, _ = oracle.qpack_affine(w.numpy(), bits, gs)
+        self.wq, self.sc, self.bi = gwb.qpack_affine(w.to(DEV), bits, gs)
+        torch.cuda.synchronize()
+        self.max_w = _affine_max_w(self.sc_o, self.bi_o, bits)
+
+    def check_pack(self):
+        assert np.array_equal(_words(self.wq), self.wq_o), "packed words differ"
+        assert np.array_equal(_np16(self.sc), self.sc_o), "scales differ"
+        assert np.array_equal(_np16(self.bi), self.bi_o), "biases differ"
+
+    def check_qmm(self, M, seed=1, outlier_frac=0.0, label=""):
+        x = synth.activations(M, self.K, seed=seed, outlier_frac=outlier_frac)
+        y = gwb.qmm_affine(x.to(DEV), self.wq, self.sc, self.bi, self.bits, self.gs)
+        rows = _rows(M, self.N, self.K)
+        y_ref = oracle.qmm_affine(synth.bits16(x), self.wq_o, self.sc_o, self.bi_o, self.N, self.K, self.bits,
+                                  self.gs, rows=rows)
+        yg = y.float().cpu().numpy()
+        if rows is not None:
+            yg = yg[rows]
+        max_x = float(x.float().abs().max())
+        return check_float(yg, y_ref, self.K, self.max_w, max_x, label or f"qmm M={M}")
+
+
+# --------------------------------------------------------------------------- packing
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("gs", [32, 64, 128])
+def test_qpack_and_dequant_affine_bit_exact(bits, gs):
+    N, K = 300, 4 * 128
+    a = Affine(N, K, bits, gs, seed=bits * 10 + gs)
+    a.check_pack()
+    w_deq = gwb.dequant_affine(a.wq, a.sc, a.bi, K, bits, gs)
+    ref = oracle.dequant_affine_bf16(a.wq_o, a.sc_o, a.bi_o, N, K, bits, gs)
+    assert np.array_equal(_np16(w_deq), ref)
+
+
+def test_qpack_affine_signed_zeros_and_constant_groups():
+    w = synth.weights(16, 128, seed=5)
+    w[0, :64] = 0.0
+    w[0, 5] = -0.0
+    w[1, :32] = 0.25
+    w[2, 64:] = -0.0
+    w[2, 70] = 0.0
+    wq_o, sc_o, bi_o, _ = oracle.qpack_affine(w.numpy(), 4, 32)
+    wq, sc, bi = gwb.qpack_affine(w.to(DEV), 4, 32)
+    assert np.array_equal(_words(wq), wq_o)
+    assert np.array_equal(_np16(sc), sc_o)
+    assert np.array_equal(_np16(bi), bi_o)
+
+
+def test_qpack_sym_i4_bit_exact():
+    w = synth.weights(333, 512, seed=9)
+    w[7] = 0.0
+    wq_o, sw_o, _ = oracle.qpack_sym_i4(w.numpy())
+    wq, sw = gwb.qpack_sym_i4(w.to(DEV))
+    assert np.array_equal(_words(wq), wq_o)
+    assert np.array_equal(sw.cpu().numpy(), sw_o)
+
+
+@pytest.mark.parametrize("M,K", [(1, 512), (7, 4096), (64, 1000), (300, 96), (5, 14336)])
+def test_quant_per_token_i8_bit_exact(M, K):
+    x = synth.activations(M, K, seed=M + K, outlier_frac=0.01)
+    if M > 3:
+        x[2] = 0
+    qx_o, sx_o = oracle.quant_per_token_i8(synth.bits16(x))
+    qx, sx = gwb.quant_per_token_i8(x.to(DEV))
+    assert np.array_equal(sx.cpu().numpy(), sx_o)
+    assert np.array_equal(qx.cpu().numpy(), qx_o)
+
+
+# --------------------------------------------------------------------------- affine qmm
+@pytest.mark.parametrize("bits,gs", [(4, 64), (4, 32), (4, 128), (8, 32), (8, 64), (8, 128), (2, 64), (2, 128)])
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_qmm_affine_gemv_small(bits, gs, M):
+    a = Affine(200, 1024, bits, gs, seed=bits + gs)
+    a.check_qmm(M, label=f"gemv b{bits} gs{gs} M{M}")
+
+
+@pytest.mark.parametrize("bits,gs", [(4, 64), (4, 32), (8, 128), (8, 64), (2, 64), (2, 32)])
+@pytest.mark.parametrize("M", [9, 16, 40, 130, 300])
+def test_qmm_affine_tensor_core_small(bits, gs, M):
+    # N = 300 ragged against the 128-row tile; K = 192 = 3 K-steps
+    a = Affine(300, 192, bits, gs, seed=bits * gs)
+    a.check_qmm(M, outlier_frac=0.01, label=f"tc b{bits} gs{gs} M{M}")
+
+
+def test_qmm_affine_k_tail_and_unsupported_gemv_combo():
+    # K = 96 (1.5 tensor-core K steps), and 2-bit gs32 at M=1 (no GEMV kernel: tensor-core path)
+    Affine(256, 96, 4, 32).check_qmm(20, label="K tail")
+    Affine(136, 256, 2, 32).check_qmm(1, label="2-bit gs32 M=1")
+
+
+def test_qmm_affine_rejects_2bit_k_not_multiple_of_64_on_tc_path():
+    a = Affine(64, 96, 2, 32)
+    x = torch.zeros(16, 96, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(gwb.GwbError, match="UNSUPPORTED"):
+        gwb.qmm_affine(x, a.wq, a.sc, a.bi, 2, 32)
+
+
+def test_qmm_affine_degenerate_inputs():
+    a = Affine(128, 256, 4, 64)
+    x = torch.zeros(4, 256, dtype=torch.bfloat16, device=DEV)
+    y = gwb.qmm_affine(x, a.wq, a.sc, a.bi, 4, 64)
+    assert torch.all(y == 0)
+    y = gwb.qmm_affine(torch.zeros(0, 256, dtype=torch.bfloat16, device=DEV), a.wq, a.sc, a.bi, 4, 64)
+    assert y.shape == (0, 128)
+
+
+# --------------------------------------------------------------------------- GPTQ
+class Gptq:
+    def __init__(self, K, N, gs, permuted, seed=0):
+        self.K, self.N, self.gs = K, N, gs
+        qw, sc, qz, gi = synth.gptq_quartet(K, N, gs, seed=seed, permuted=permuted)
+        self.h = (qw.numpy(), synth.bits16(sc), qz.numpy(), gi.numpy() if permuted else None)
+        self.d = (qw.to(DEV), sc.to(DEV), qz.to(DEV), gi.to(DEV) if permuted else None)
+
+    def check_dequant(self):
+        w = gwb.gptq_dequant(*self.d, self.gs)
+        ref = oracle.gptq_dequant_f16(*self.h, self.K, self.N, self.gs)
+        assert np.array_equal(_np16(w), ref)
+        return float(w.float().abs().max())
+
+    def check_qmm(self, M, seed=1):
+        max_w = self.check_dequant()
+        x = synth.activations(M, self.K, seed=seed, dtype=torch.float16)
+        y = gwb.gptq_qmm(x.to(DEV), *self.d, self.gs)
+        rows = _rows(M, self.N, self.K, budget=1e8)
+        y_ref = oracle.gptq_qmm(synth.bits16(x), *self.h, self.K, self.N, self.gs, rows=rows)
+        yg = y.float().cpu().numpy()
+        if rows is not None:
+            yg = yg[rows]
+        return check_float(yg, y_ref, self.K, max_w, float(x.float().abs().max()), f"gptq M={M}")
+
+
+@pytest.mark.parametrize("permuted", [False, True])
+@pytest.mark.parametrize("gs", [32, 128])
+def test_gptq_dequant_bit_exact(permuted, gs):
+    Gptq(512, 200, gs, permuted, seed=gs).check_dequant()
+
+
+@pytest.mark.parametrize("permuted", [False, True])
+@pytest.mark.parametrize("M", [1, 4, 8, 32, 150])
+def test_gptq_qmm_small(permuted, M):
+    Gptq(384, 264, 128 if M % 2 else 64, permuted, seed=M).check_qmm(M)
+
+
+# --------------------------------------------------------------------------- W4A8
+class W4A8:
+    def __init__(self, N, K, seed=0):
+        self.N, self.K = N, K
+        w = synth.weights(N, K, seed=seed)
+        self.wq_o, self.sw_o, _ = oracle.qpack_sym_i4(w.numpy())
+        self.wq, self.sw = gwb.qpack_sym_i4(w.to(DEV))
+        assert np.array_equal(_words(self.wq), self.wq_o) and np.array_equal(self.sw.cpu().numpy(), self.sw_o)
+
+    def check(self, M, seed=1):
+        x = synth.activations(M, self.K, seed=seed)
+        qx_o, sx_o = oracle.quant_per_token_i8(synth.bits16(x))
+        qx, sx = gwb.quant_per_token_i8(x.to(DEV))
+        assert np.array_equal(qx.cpu().numpy(), qx_o) and np.array_equal(sx.cpu().numpy(), sx_o)
+        y, acc = gwb.gemm_i8i4(qx, sx, self.wq, self.sw, want_y=True, want_acc=True)
+        rows = _rows(M, self.N, self.K)
+        acc_o, y_o, ovf = oracle.gemm_i8i4(qx_o, sx_o, self.wq_o, self.sw_o, self.N, self.K, rows=rows)
+        assert not ovf
+        a = acc.cpu().numpy().astype(np.int64)
+        yg = y.float().cpu().numpy()
+        if rows is not None:
+            a, yg = a[rows], yg[rows]
+        assert np.array_equal(a, acc_o), "int32 accumulators differ"
+        max_w = float(np.max(np.abs(self.sw_o)) * 7)
+        return check_float(yg, y_o, self.K, max_w, float(x.float().abs().max()), f"w4a8 M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 64, 100, 300])
+def test_w4a8_small(M):
+    W4A8(200, 384, seed=M).check(M)
+
+
+def test_w4a8_k_tail():
+    W4A8(136, 96).check(24)   # K = 96 < one 128-wide K step
+
+
+# --------------------------------------------------------------------------- full sizes
+def test_full_single_affine_linear_512():
+    a = Affine(512, 512, 4, 64)
+    a.check_pack()
+    a.check_qmm(1, label="512x512 M=1")
+
+
+DECODE_SHAPES = [(2048, 2048, 4), (512, 2048, 4), (8192, 2048, 4), (2048, 8192, 4), (128256, 2048, 4),
+                 (8192, 2048, 2), (8192, 2048, 8)]
+
+
+@pytest.mark.parametrize("N,K,bits", DECODE_SHAPES)
+def test_full_decode_gemv(N, K, bits):
+    a = Affine(N, K, bits, 64)
+    a.check_pack()
+    a.check_qmm(1, label=f"decode {N}x{K} b{bits}")
+
+
+PREFILL_SHAPES = [(4096, 4096), (1024, 4096), (14336, 4096), (4096, 14336)]
+
+
+@pytest.mark.parametrize("N,K", PREFILL_SHAPES)
+def test_full_prefill_gemm_4bit_gs64(N, K):
+    a = Affine(N, K, 4, 64)
+    a.check_pack()
+    for M in (16, 128, 2048):
+        a.check_qmm(M, outlier_frac=0.01, label=f"prefill {N}x{K} M={M}")
+
+
+@pytest.mark.parametrize("bits,gs", [(8, 32), (8, 128), (4, 32), (4, 128)])
+def test_full_prefill_other_formats(bits, gs):
+    a = Affine(4096, 4096, bits, gs)
+    a.check_pack()
+    for M in (16, 512):
+        a.check_qmm(M, outlier_frac=0.01, label=f"prefill b{bits} gs{gs} M={M}")
+
+
+@pytest.mark.parametrize("permuted", [False, True])
+def test_full_gptq(permuted):
+    g = Gptq(4096, 11008, 128, permuted)
+    for M in (1, 32, 1024):
+        g.check_qmm(M)
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096), (4096, 14336)])
+def test_full_w4a8(N, K):
+    w = W4A8(N, K)
+    for M in (8, 64, 512, 4096):
+        w.check(M)
+
+
+def test_no_device_wait_gave_up():
+    gwb.check_device_error()
