@@ -1,0 +1,418 @@
+"""Benchmark of the fused dequant + matmul hot path on B200.
+
+One step = one pass of the decode GEMV sweep at M = 1 (bf16 activations,
+MLX affine weights, group size 64): N x K in {2048x2048, 512x2048, 8192x2048,
+2048x8192, 128256x2048} at 4 bits, plus 8192x2048 at 2 and 8 bits.  The
+headline value is whole-job HBM throughput (algorithmic bytes: packed codes +
+bf16 scales and biases + activations + outputs, per call) in GB/s.  The same
+JSON line also carries the prefill GEMM at M = 2048 (4-bit, group size 64,
+shapes 4096x4096, 1024x4096, 14336x4096, 4096x14336) in TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {gwb,reference}]
+
+N > 1 is launched by torchrun: every rank runs an independent replica of the
+step on its own GPU (the path has no exchange step); the time is the max over
+ranks and the value counts the bytes of all ranks ("scaling": "weak").
+--impl reference times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import threading
+import time
+
+import numpy as np
+import torch
+
+import gwb_synth as synth
+
+DECODE = [  # (N, K, bits)
+    (2048, 2048, 4), (512, 2048, 4), (8192, 2048, 4), (2048, 8192, 4), (128256, 2048, 4),
+    (8192, 2048, 2), (8192, 2048, 8),
+]
+PREFILL = [(4096, 4096), (1024, 4096), (14336, 4096), (4096, 14336)]
+GS = 64
+M_PREFILL = 2048
+METRIC = "qmm GB/s (M=1) and TFLOP/s (M=2048), % of roofline, 4-bit gs=64, 1 B200"
+WORKLOAD = ("decode GEMV sweep, M=1, bf16 x, MLX affine gs=64: 4-bit NxK 2048x2048, 512x2048, 8192x2048, "
+            "2048x8192, 128256x2048; 2-bit and 8-bit 8192x2048")
+ROOT = os.path.dirname(os.path.abspath(__file__))
+
+
+def gemv_bytes(N, K, bits, M=1, gs=GS):
+    """Algorithmic bytes of one qmm call: packed codes, bf16 scales + biases, x and y."""
+    return N * K * bits // 8 + 2 * 2 * N * (K // gs) + 2 * M * K + 2 * M * N
+
+
+STEP_BYTES = sum(gemv_bytes(N, K, b) for N, K, b in DECODE)
+LMHEAD = (128256, 2048, 4)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def traffic_for(kernel_key):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            return json.load(f).get(kernel_key)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running (reads only)."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index):
+        self.index, self.samples, self.reasons, self.max_mhz = index, [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self._t = None
+        return self
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ GPU arm
+def build_decode(gwb, dev, n_sets=2):
+    """Quantizes every decode weight on the device (seeded N(0, 0.02)); n_sets copies rotate."""
+    sets = []
+    for s in range(n_sets):
+        layers = []
+        for i, (N, K, bits) in enumerate(DECODE):
+            g = torch.Generator(device=dev)
+            g.manual_seed(1000 * s + i)
+            w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+            wq, sc, bi = gwb.qpack_affine(w, bits, GS)
+            del w
+            x = synth.activations(1, K, seed=1).to(dev)
+            y = torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+            layers.append((wq, sc, bi, x, y, bits))
+        sets.append(layers)
+    torch.cuda.synchronize()
+    return sets
+
+
+def run_gpu(args, world, rank, local):
+    import group_wise_bit_b200 as gwb
+
+    dev = torch.device("cuda", local)
+    hbm_peak, bf16_peak, peak_kind = peaks()
+    sets = build_decode(gwb, dev)
+    lm_idx = DECODE.index(LMHEAD)
+
+    # CUDA graphs: per weight set, graph A = the six small layers, graph B = the lm_head GEMV
+    # (kept separate so events between the two replays time the dominant kernel live).
+    stream = torch.cuda.Stream(device=dev)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for layers in sets:
+            for (wq, sc, bi, x, y, bits) in layers:           # warm the launch path before capture
+                gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+            torch.cuda.synchronize()
+            ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ga, stream=stream):
+                for i, (wq, sc, bi, x, y, bits) in enumerate(layers):
+                    if i != lm_idx:
+                        gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+            with torch.cuda.graph(gb, stream=stream):
+                wq, sc, bi, x, y, bits = layers[lm_idx]
+                gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+            graphs.append((ga, gb))
+    torch.cuda.synchronize()
+
+    def step(i, ev=None):
+        ga, gb = graphs[i % len(graphs)]
+        if ev is not None:
+            ev[0].record(stream)
+        gb.replay()
+        if ev is not None:
+            ev[1].record(stream)
+        ga.replay()
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    torch.cuda.synchronize()
+
+    lm_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for i in range(args.steps):
+                step(i, lm_events[i])
+            t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms, world)
+    ms_step = ms_max / args.steps
+    value = world * STEP_BYTES * args.steps / (ms_max * 1e-3) / 1e9
+    lm_ms = float(np.mean([a.elapsed_time(b) for a, b in lm_events]))
+    lm_bytes = gemv_bytes(*LMHEAD)
+    achieved = lm_bytes / (lm_ms * 1e-3) / 1e9
+
+    # End to end through the public API: pinned host x -> device, qmm, y -> pinned host, every layer.
+    host_x = [l[3].cpu().pin_memory() for l in sets[0]]
+    host_y = [torch.empty(l[4].shape, dtype=torch.bfloat16).pin_memory() for l in sets[0]]
+    h2d = sum(t.numel() * 2 for t in host_x)
+    d2h = sum(t.numel() * 2 for t in host_y)
+
+    def e2e_step(i):
+        layers = sets[i % len(sets)]
+        for j, (wq, sc, bi, x, y, bits) in enumerate(layers):
+            x.copy_(host_x[j], non_blocking=True)
+            gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+            host_y[j].copy_(y, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * STEP_BYTES * args.steps / (e_ms * 1e-3) / 1e9
+
+    prefill = run_prefill(gwb, dev, stream, bf16_peak, peak_kind) if not args.no_prefill else None
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": 1, "group_size": GS, "bytes_per_step": STEP_BYTES,
+                   "l2": "inputs larger than L2: 192 MB of weights per step, two weight sets rotate (384 MB)",
+                   "graphs": "each step replays two CUDA graphs (lm_head GEMV; the six other GEMVs)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "k_gemv_affine<4,64,1> (lm_head 128256x2048)", "bound": "hbm",
+                     "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "peak_source": peak_kind,
+                     "bytes_per_launch": lm_bytes, "avg_launch_us": round(lm_ms * 1e3, 2),
+                     "traffic": traffic_for("k_gemv_affine_lmhead")},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "weights resident in HBM; per layer: H2D of x, qmm_affine call, D2H of y"},
+        "gpu_launches": len(DECODE) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if prefill:
+        out["prefill_m2048"] = prefill
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_prefill(gwb, dev, stream, bf16_peak, peak_kind, reps=5):
+    """M = 2048 prefill GEMMs (4-bit, gs 64), each launch timed alone with an L2 flush before it."""
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    total_flop, total_ms, per = 0.0, 0.0, []
+    for i, (N, K) in enumerate(PREFILL):
+        g = torch.Generator(device=dev)
+        g.manual_seed(77 + i)
+        w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+        wq, sc, bi = gwb.qpack_affine(w, 4, GS)
+        del w
+        x = synth.activations(M_PREFILL, K, seed=1, outlier_frac=0.01).to(dev)
+        y = torch.empty((M_PREFILL, N), dtype=torch.bfloat16, device=dev)
+        ts = []
+        with torch.cuda.stream(stream):
+            for r in range(reps + 2):
+                flush.fill_(r)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                gwb.qmm_affine(x, wq, sc, bi, 4, GS, y=y)
+                b.record(stream)
+                b.synchronize()
+                if r >= 2:
+                    ts.append(a.elapsed_time(b))
+        ms = statistics.median(ts)
+        flop = 2.0 * M_PREFILL * N * K
+        total_flop += flop
+        total_ms += ms
+        per.append({"N": N, "K": K, "us": round(ms * 1e3, 1), "tflops": round(flop / (ms * 1e-3) / 1e12, 1)})
+    tf = total_flop / (total_ms * 1e-3) / 1e12
+    return {"value": round(tf, 1), "unit": "TFLOP/s", "M": M_PREFILL, "bits": 4, "group_size": GS,
+            "l2": "256 MB buffer written before every timed launch",
+            "roofline": {"kernel": "k_tc<Affine,4,256>", "bound": "tensor", "achieved": round(tf, 1),
+                         "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(tf / bf16_peak, 4),
+                         "peak_source": peak_kind, "traffic": traffic_for("k_tc_affine4_m2048")},
+            "shapes": per}
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+def oracle_sample(frac, seed=0):
+    """A row sample of every decode layer, quantized by the oracle (untimed preparation)."""
+    import oracle
+    layers = []
+    for i, (N, K, bits) in enumerate(DECODE):
+        n = max(8, int(N * frac))
+        w = synth.weights(n, K, seed=seed + i)
+        wq, sc, bi, _ = oracle.qpack_affine(w.numpy(), bits, GS)
+        x = synth.bits16(synth.activations(1, K, seed=1))
+        layers.append((x, wq, sc, bi, n, K, bits))
+    return layers
+
+
+def oracle_pass(layers):
+    import oracle
+    nbytes = 0
+    for x, wq, sc, bi, n, K, bits in layers:
+        oracle.qmm_affine(x, wq, sc, bi, n, K, bits, GS)
+        nbytes += gemv_bytes(n, K, bits)
+    return nbytes
+
+
+def cpu_baseline(budget_s=12.0, frac=0.25):
+    layers = oracle_sample(frac)
+    t = time.perf_counter()
+    nbytes, passes = 0, 0
+    while passes < 1 or time.perf_counter() - t < budget_s:
+        nbytes += oracle_pass(layers)
+        passes += 1
+    dt = time.perf_counter() - t
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{passes} pass(es) over the first {frac:.0%} of the output rows of every decode layer "
+                      f"(M=1, gs=64), single-threaded C, fp64, {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    frac = args.ref_frac
+    layers = oracle_sample(frac)
+    for _ in range(args.warmup):
+        oracle_pass(layers)
+    t = time.perf_counter()
+    nbytes = 0
+    for _ in range(args.steps):
+        nbytes += oracle_pass(layers)
+    dt = time.perf_counter() - t
+    value = nbytes / dt / 1e9
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": 1, "group_size": GS,
+                   "sample": f"first {frac:.1%} of the output rows of every layer per step"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} steps, each over the first {frac:.1%} of the output rows of "
+                                   f"every decode layer, single-threaded C, fp64"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["gwb", "reference"], default="gwb")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-frac", type=float, default=1 / 16)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -131,8 +131,8 @@ def test_qmm_affine_gemv_small(bits, gs, M):
 @pytest.mark.parametrize("bits,gs", [(4, 64), (4, 32), (8, 128), (8, 64), (2, 64), (2, 32)])
 @pytest.mark.parametrize("M", [9, 16, 40, 130, 300])
 def test_qmm_affine_tensor_core_small(bits, gs, M):
-    # N = 300 ragged against the 128-row tile; K = 192 = 3 K-steps
-    a = Affine(300, 192, bits, gs, seed=bits * gs)
+    # N = 300 ragged against the 128-row tile; K = 384 = 6 K-steps
+    a = Affine(300, 384, bits, gs, seed=bits * gs)
     a.check_qmm(M, outlier_frac=0.01, label=f"tc b{bits} gs{gs} M{M}")
 
 
