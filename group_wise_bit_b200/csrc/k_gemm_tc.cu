@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                 : make_idesc(1, 1, kTileN, BT);
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char *base = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char *base = align_smem_1024(smem_raw);
   uint64_t *full = reinterpret_cast<uint64_t *>(base + STAGES * STAGE);
   uint64_t *afull = full + STAGES;
   uint64_t *empty = afull + STAGES;

@@ -9,15 +9,28 @@
 
 namespace gwb {
 
-// Device error flag (bit 0: a bounded wait gave up).  Read and cleared by the
-// host through gwb_check_device_error().  Only the tensor-core translation unit
-// includes this header, so the flag has a single definition.
+// Device error flag (bit 0: a bounded wait gave up).  Each translation unit
+// that includes this header has its own copy and exposes a host function that
+// reads and clears it; gwb_check_device_error() reads all of them.
 static __device__ unsigned int g_device_error = 0;
 
 constexpr unsigned long long kWaitCycles = 4000000000ull;  // ~2 s at 1.9 GHz
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 2^n as an exact fp32 value, built from its exponent field (n in [-126, 127]).
+__device__ __forceinline__ float pow2f(int n) {
+  return __int_as_float((127 + n) << 23);
+}
+
+// Rounds a dynamic shared-memory pointer up to a 1024-byte boundary of the
+// shared window by pointer arithmetic (not through an integer cast), so the
+// compiler keeps treating every derived pointer as shared memory (ld/st.shared
+// with 32-bit addresses instead of generic 64-bit accesses).
+__device__ __forceinline__ unsigned char *align_smem_1024(unsigned char *p) {
+  return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
 }
 
 // ---------------------------------------------------------------- mbarrier
@@ -66,6 +79,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     }
   }
   return true;
+}
+
+// ---------------------------------------------------------------- cp.async
+// 4- or 16-byte asynchronous global -> shared copy; src_bytes < size zero-fills the rest.
+__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_8(void *smem_dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(smem_dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_16(void *smem_dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` once this thread's prior cp.async copies complete (the
+// barrier's expected count must include this arrival).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // ---------------------------------------------------------------- proxies
@@ -170,4 +203,73 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t c_fmt, uint32_t ab_fm
   return (c_fmt << 4) | (ab_fmt << 7) | (ab_fmt << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
 }
 
+}  // namespace gwb
+
+namespace gwb {
+// ---------------------------------------------------------------- tcgen05 (TMEM operands)
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16; A is K-major in TMEM (lane =
+// row, two 16-bit elements per 32-bit column, lower k in the low half).
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Each thread writes N consecutive 32-bit columns of its own TMEM lane.
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t *r);
+template <>
+__device__ __forceinline__ void tmem_st<16>(uint32_t taddr, const uint32_t *r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_st<32>(uint32_t taddr, const uint32_t *r) {
+  tmem_st<16>(taddr, r);
+  tmem_st<16>(taddr + 16, r + 16);
+}
+template <>
+__device__ __forceinline__ void tmem_st<64>(uint32_t taddr, const uint32_t *r) {
+  tmem_st<32>(taddr, r);
+  tmem_st<32>(taddr + 32, r + 32);
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Each thread reads N consecutive 32-bit columns of its own TMEM lane.
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t *r);
+template <>
+__device__ __forceinline__ void tmem_ld<1>(uint32_t taddr, uint32_t *r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr) : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld<2>(uint32_t taddr, uint32_t *r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr) : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld<4>(uint32_t taddr, uint32_t *r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr)
+               : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld<8>(uint32_t taddr, uint32_t *r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+
+// Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 }  // namespace gwb

@@ -136,6 +136,18 @@ def test_qmm_affine_tensor_core_small(bits, gs, M):
     a.check_qmm(M, outlier_frac=0.01, label=f"tc b{bits} gs{gs} M{M}")
 
 
+@pytest.mark.parametrize("M", [1, 5])
+def test_qmm_affine_gemv_register_fed_fallback(M):
+    # an odd number of groups per row (K / gs = 3) is served by the register-fed GEMV
+    Affine(264, 192, 4, 64).check_qmm(M, label=f"register-fed GEMV M={M}")
+
+
+@pytest.mark.parametrize("bits,M", [(4, 1), (4, 3), (8, 2), (2, 1)])
+def test_qmm_affine_gemv_persistent_tiles(bits, M):
+    # 157 tiles of 128 rows on 148 persistent CTAs: some CTAs stream two tiles
+    Affine(20000, 512, bits, 64, seed=3).check_qmm(M, label=f"persistent b{bits} M={M}")
+
+
 def test_qmm_affine_k_tail_and_unsupported_gemv_combo():
     # K = 96 (1.5 tensor-core K steps), and 2-bit gs32 at M=1 (no GEMV kernel: tensor-core path)
     Affine(256, 96, 4, 32).check_qmm(20, label="K tail")
