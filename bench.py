@@ -62,12 +62,16 @@ def peaks():
 
 
 def traffic_for(kernel_key):
-    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None."""
+    """Per-launch DRAM bytes (read + write) of a kernel from the committed ncu summary, or None."""
     try:
-        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            return json.load(f).get(kernel_key)
+        with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
+            for line in f:
+                parts = line.split()
+                if parts and not parts[0].startswith("#") and parts[0] == kernel_key:
+                    return int(parts[1])
     except Exception:
-        return None
+        pass
+    return None
 
 
 class ClockSampler:
@@ -269,11 +273,11 @@ def run_gpu(args, world, rank, local):
                    "l2": "inputs larger than L2: 192 MB of weights per step, two weight sets rotate (384 MB)",
                    "graphs": "each step replays two CUDA graphs (lm_head GEMV; the six other GEMVs)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "k_gemv_affine<4,64,1> (lm_head 128256x2048)", "bound": "hbm",
+        "roofline": {"kernel": "k_gemv_stream<4,64,1> (lm_head 128256x2048)", "bound": "hbm",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "peak_source": peak_kind,
                      "bytes_per_launch": lm_bytes, "avg_launch_us": round(lm_ms * 1e3, 2),
-                     "traffic": traffic_for("k_gemv_affine_lmhead")},
+                     "traffic": traffic_for("k_gemv_stream_lmhead")},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "weights resident in HBM; per layer: H2D of x, qmm_affine call, D2H of y"},
         "gpu_launches": len(DECODE) * args.steps,
@@ -387,6 +391,50 @@ def run_reference(args, world, rank):
     print(json.dumps(out), flush=True)
 
 
+def run_layer(args):
+    """One layer only (for profiling): qmm_affine on an N x K weight at M tokens, replayed in a
+    CUDA graph of 20 launches that alternate between two weight sets (> L2)."""
+    import group_wise_bit_b200 as gwb
+    N, K, bits, M = (list(map(int, args.layer.split(","))) + [1])[:4]
+    dev = torch.device("cuda", 0)
+    sets = []
+    for s in range(2):
+        g = torch.Generator(device=dev)
+        g.manual_seed(s)
+        w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+        sets.append(gwb.qpack_affine(w, bits, GS))
+        del w
+    x = synth.activations(M, K, seed=1).to(dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    st = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(st):
+        for wq, sc, bi in sets:
+            gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=st):
+            for i in range(20):
+                wq, sc, bi = sets[i % 2]
+                gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+        for _ in range(args.warmup):
+            gr.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(args.steps):
+            gr.replay()
+        b.record(st)
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / (20 * args.steps)
+    nbytes = gemv_bytes(N, K, bits, M=M) if M <= 8 else None
+    out = {"layer": {"N": N, "K": K, "bits": bits, "group_size": GS, "M": M}, "us_per_launch": round(us, 2)}
+    if nbytes:
+        out["GB/s"] = round(nbytes / us / 1e3, 1)
+    else:
+        out["TFLOP/s"] = round(2.0 * M * N * K / us / 1e6, 1)
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -397,7 +445,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-frac", type=float, default=1 / 16)
+    ap.add_argument("--layer", default=None,
+                    help="N,K,bits[,M]: time one qmm_affine layer (group size 64) instead of the sweep")
     args = ap.parse_args()
+    if args.layer:
+        run_layer(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -50,6 +50,7 @@ struct TcArgs {
   const float *sx, *sw;     // i8: per-token / per-channel scales
   uint16_t *y;              // bf16 (affine, i8) or fp16 (gptq) [M, N]
   int32_t *acc;             // i8: optional int32 [M, N]
+  int staged_scales;        // 1: the producer copies each stage's scales (and zeros) into shared memory
 };
 
 template <Fmt F, int BITS>
@@ -59,18 +60,21 @@ struct Traits<Fmt::Affine, BITS> {
   static constexpr int BK = 64;                       // bf16: 64 elements = 128 bytes per row
   static constexpr int RAW_BYTES = kTileN * BK * BITS / 8;
   static constexpr int NMMA = BK / 16;
+  static constexpr int SC_BYTES = 1024;               // (scales, biases) x 128 rows x an aligned pair of groups
 };
 template <>
 struct Traits<Fmt::Gptq, 4> {
   static constexpr int BK = 64;
   static constexpr int RAW_BYTES = (BK / 8) * kTileN * 4;
   static constexpr int NMMA = BK / 16;
+  static constexpr int SC_BYTES = 1024;               // 2 groups x (128 fp16 scales + 16 qzeros words)
 };
 template <>
 struct Traits<Fmt::I8, 4> {
   static constexpr int BK = 128;                      // int8: 128 elements = 128 bytes per row
   static constexpr int RAW_BYTES = kTileN * BK / 2;
   static constexpr int NMMA = BK / 32;
+  static constexpr int SC_BYTES = 0;
 };
 
 __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr int BK = T::BK;
   constexpr int B_BYTES = BT * 128;
   constexpr int A_BYTES = kTileN * 128;
-  constexpr int STAGE = B_BYTES + A_BYTES + T::RAW_BYTES;
+  constexpr int STAGE = B_BYTES + A_BYTES + T::RAW_BYTES + T::SC_BYTES;
   constexpr uint32_t NCOLS = BT < 32 ? 32 : BT;
   constexpr uint32_t IDESC = (F == Fmt::I8) ? make_idesc(2, 1, kTileN, BT)
                              : (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN, BT)
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; s++) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + 32);   // producer arrive.expect_tx + one cp.async arrive per producer lane
       mbar_init(&afull[s], kDqThreads / 32);
       mbar_init(&empty[s], 1);
     }
@@ -213,22 +217,54 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nk; i++) {
-        const int s = i % STAGES, r = i / STAGES;
-        if (!mbar_wait(&empty[s], (r & 1) ^ 1)) { *abort_flag = 1; break; }
-        unsigned char *st = base + s * STAGE;
+    // Lane 0 issues the TMA loads; every lane copies a share of the stage's
+    // scales / biases (GPTQ: scales and qzeros words) with cp.async, so the
+    // dequantizers find them in shared memory when the stage completes.
+    int issued = 0;
+    for (int i = 0; i < nk; i++) {
+      const int s = i % STAGES, r = i / STAGES;
+      if (!mbar_wait(&empty[s], (r & 1) ^ 1)) { *abort_flag = 1; break; }
+      unsigned char *st = base + s * STAGE;
+      if (lane == 0) {
         mbar_arrive_expect_tx(&full[s], B_BYTES + T::RAW_BYTES);
         tma_load_2d(st, &tm_x, i * BK, m0, &full[s]);
         if constexpr (F == Fmt::Gptq) tma_load_2d(st + B_BYTES + A_BYTES, &tm_w, n0, i * (BK / 8), &full[s]);
         else tma_load_2d(st + B_BYTES + A_BYTES, &tm_w, i * (BK * BITS / 32), n0, &full[s]);
-        issued = i + 1;
       }
-      // Drain: every issued copy has landed before the CTA can exit.
-      for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; i++)
-        mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
+      unsigned char *sc = st + B_BYTES + A_BYTES + T::RAW_BYTES;
+      if constexpr (F == Fmt::Affine) {
+        if (args.staged_scales) {
+          const int G = args.K / args.gs;
+          const int gp = ((i * BK) / args.gs) & ~1;
+          for (int e = lane; e < 2 * kTileN; e += 32) {   // (array, row) -> 4 bytes: groups gp, gp+1
+            const int arr = e / kTileN, row = e % kTileN, n = n0 + row;
+            const bool ok = n < args.N && gp < G;
+            const uint16_t *src = (arr ? args.biases : args.scales) + (ok ? (int64_t)n * G + gp : 0);
+            cp_async_4(sc + e * 4, src, ok ? 4u : 0u);
+          }
+        }
+      } else if constexpr (F == Fmt::Gptq) {
+        if (args.staged_scales) {
+          const int G = args.K / args.gs;
+          const int gp = (i * BK) / args.gs;
+          {   // scales: 2 groups x 128 columns = 32 chunks of 16 bytes, one per lane
+            const int gi = lane >> 4, ch = lane & 15, g = gp + gi, n = n0 + ch * 8;
+            const bool ok = g < G && n < args.N;
+            cp_async_16(sc + lane * 16, args.scales + (ok ? (int64_t)g * args.N + n : 0), ok ? 16u : 0u);
+          }
+          {   // qzeros: 2 groups x 16 words, one word per lane
+            const int gi = lane >> 4, wz = lane & 15, g = gp + gi, n = n0 + wz * 8;
+            const bool ok = g < G && n < args.N;
+            cp_async_4(sc + 512 + lane * 4, args.qzeros + (ok ? (int64_t)g * (args.N / 8) + n / 8 : 0), ok ? 4u : 0u);
+          }
+        }
+      }
+      cp_async_arrive_noinc(&full[s]);
+      issued = i + 1;
     }
+    // Drain: every issued copy has landed before the CTA can exit.
+    for (int i = issued - STAGES < 0 ? 0 : issued - STAGES; i < issued; i++)
+      mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -269,13 +305,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float sf = 0.f, bfv = 0.f;
       uint32_t z2[4], s2[4];
       if constexpr (F == Fmt::Affine) {
-        const int G = args.K / args.gs;
-        int g = kh / args.gs;
-        g = g < G ? g : G - 1;
-        sf = bf16_val(__ldg(args.scales + (int64_t)nc * G + g));
-        bfv = bf16_val(__ldg(args.biases + (int64_t)nc * G + g));
+        if (!args.staged_scales) {
+          const int G = args.K / args.gs;
+          int g = kh / args.gs;
+          g = g < G ? g : G - 1;
+          sf = bf16_val(__ldg(args.scales + (int64_t)nc * G + g));
+          bfv = bf16_val(__ldg(args.biases + (int64_t)nc * G + g));
+        }
       } else if constexpr (F == Fmt::Gptq) {
-        if (args.g_idx == nullptr) {
+        if (args.g_idx == nullptr && !args.staged_scales) {
           const int G = args.K / args.gs;
           int g = kh / args.gs;
           g = g < G ? g : G - 1;
@@ -291,6 +329,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       unsigned char *st = base + s * STAGE;
       unsigned char *A = st + B_BYTES;
       const unsigned char *R = st + B_BYTES + A_BYTES;
+      if constexpr (F == Fmt::Affine) {
+        if (args.staged_scales) {   // this half step's group within the staged pair
+          int idx = kh / args.gs - (((i * BK) / args.gs) & ~1);
+          idx = idx < 1 ? idx : 1;
+          const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW_BYTES);
+          sf = bf16_val(sc[r * 2 + idx]);
+          bfv = bf16_val(sc[(kTileN + r) * 2 + idx]);
+        }
+      } else if constexpr (F == Fmt::Gptq) {
+        if (args.g_idx == nullptr && args.staged_scales) {
+          int idx = kh / args.gs - (i * BK) / args.gs;
+          idx = idx < 1 ? idx : 1;
+          const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW_BYTES);
+          const uint32_t *zc = reinterpret_cast<const uint32_t *>(R + T::RAW_BYTES + 512);
+          const uint32_t sv = sc[idx * kTileN + r];
+          const uint32_t zv = 0x6400u | (((zc[idx * 16 + r / 8] >> ((r % 8) * 4)) & 0xFu) + 1u);
+#pragma unroll
+          for (int p = 0; p < 4; p++) { s2[p] = sv | (sv << 16); z2[p] = zv | (zv << 16); }
+        }
+      }
       if constexpr (F == Fmt::Affine && BITS == 4) {
         const uint4 raw = *reinterpret_cast<const uint4 *>(R + (r * 8 + h * 4) * 4);
         const __nv_bfloat162 s2b = __floats2bfloat162_rn(sf, sf), b2b = __floats2bfloat162_rn(bfv, bfv);
@@ -427,7 +485,7 @@ gwb_status make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uin
 
 template <Fmt F, int BITS, int BT>
 constexpr int stages_for() {
-  constexpr int stage = BT * 128 + kTileN * 128 + Traits<F, BITS>::RAW_BYTES;
+  constexpr int stage = BT * 128 + kTileN * 128 + Traits<F, BITS>::RAW_BYTES + Traits<F, BITS>::SC_BYTES;
   constexpr int s = (kMaxSmem - 2048) / stage;
   return s > 6 ? 6 : s;
 }
@@ -436,7 +494,7 @@ template <Fmt F, int BITS, int BT>
 gwb_status run_tc(const CUtensorMap &tx, const CUtensorMap &tw, const TcArgs &a, cudaStream_t st) {
   constexpr int STAGES = stages_for<F, BITS, BT>();
   static_assert(STAGES >= 2, "shared memory too small");
-  constexpr int stage = BT * 128 + kTileN * 128 + Traits<F, BITS>::RAW_BYTES;
+  constexpr int stage = BT * 128 + kTileN * 128 + Traits<F, BITS>::RAW_BYTES + Traits<F, BITS>::SC_BYTES;
   const size_t smem = (size_t)STAGES * stage + 1024 + 256;
   auto kern = k_tc<F, BITS, BT, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -475,6 +533,8 @@ gwb_status launch_tc_affine(const uint16_t *x, int64_t M, const uint32_t *wq, co
   TcArgs a{};
   a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
   a.scales = scales; a.biases = biases; a.y = y;
+  // 4-byte copies of aligned group pairs: an even group count and 4-byte aligned arrays.
+  a.staged_scales = ((K / gs) % 2 == 0 && (((uintptr_t)scales | (uintptr_t)biases) & 3) == 0) ? 1 : 0;
   CUtensorMap tw;
   const uint64_t words = (uint64_t)K * bits / 32;
   gwb_status s = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, (uint64_t)N, words * 4,
@@ -491,6 +551,8 @@ gwb_status launch_tc_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, 
   TcArgs a{};
   a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
   a.scales = scales; a.qzeros = qzeros; a.g_idx = g_idx; a.y = y;
+  // 16-byte scale copies and 4-byte qzeros copies need those alignments.
+  a.staged_scales = (g_idx == nullptr && ((uintptr_t)scales & 15) == 0 && ((uintptr_t)qzeros & 3) == 0) ? 1 : 0;
   CUtensorMap tw;
   gwb_status s = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, (uint64_t)N, (uint64_t)(K / 8),
                           (uint64_t)N * 4, (uint32_t)kTileN, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);
