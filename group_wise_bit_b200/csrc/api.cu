@@ -82,11 +82,12 @@ const char *gwb_last_error(void) { return gwb::g_msg; }
 const char *gwb_version(void) { return "group_wise_bit_b200 0.1 (sm_100a)"; }
 
 gwb_status gwb_check_device_error(void *stream) {
-  unsigned int flag = 0, flag2 = 0, flag3 = 0;
+  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0;
   GWB_TRY(gwb::read_and_clear_device_error(as_stream(stream), &flag));
   GWB_TRY(gwb::read_and_clear_device_error_stream(as_stream(stream), &flag2));
   GWB_TRY(gwb::read_and_clear_device_error_tmem(as_stream(stream), &flag3));
-  flag |= flag2 | flag3;
+  GWB_TRY(gwb::read_and_clear_device_error_pipe(as_stream(stream), &flag4));
+  flag |= flag2 | flag3 | flag4;
   if (flag) return fail(GWB_ERR_TIMEOUT, "a bounded device-side wait gave up (flag 0x%x)", flag);
   return GWB_OK;
 }
@@ -129,8 +130,10 @@ gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, cons
   GWB_TRY(need(scales, "scales"));
   GWB_TRY(need(biases, "biases"));
   if (M <= 8 && gwb::gemv_affine_supported(bits, group_size)) {
-    const gwb_status s =
-        gwb::launch_gemv_stream(x, (int)M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
+    gwb_status s =
+        gwb::launch_gemv_pipe(x, (int)M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
+    if (s != GWB_ERR_UNSUPPORTED) return s;
+    s = gwb::launch_gemv_stream(x, (int)M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
     if (s != GWB_ERR_UNSUPPORTED) return s;
     return gwb::launch_gemv_affine(x, (int)M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
   }

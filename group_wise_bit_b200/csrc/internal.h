@@ -40,6 +40,12 @@ gwb_status launch_gemv_stream(const uint16_t *x, int M, const uint32_t *wq, cons
                               const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
                               cudaStream_t st);
 gwb_status read_and_clear_device_error_stream(cudaStream_t st, unsigned int *flag);
+// Producer/consumer decode GEMV (the main decode kernel); GWB_ERR_UNSUPPORTED
+// (without a message) for layouts it does not cover (K / gs not a multiple of 8).
+gwb_status launch_gemv_pipe(const uint16_t *x, int M, const uint32_t *wq, const uint16_t *scales,
+                            const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
+                            cudaStream_t st);
+gwb_status read_and_clear_device_error_pipe(cudaStream_t st, unsigned int *flag);
 // TMEM-operand tensor-core GEMV (the main decode kernel); GWB_ERR_UNSUPPORTED
 // (without a message) when the layout is outside what it covers.
 gwb_status launch_gemv_tmem(const uint16_t *x, int M, const uint32_t *wq, const uint16_t *scales,

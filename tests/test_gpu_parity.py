@@ -148,6 +148,19 @@ def test_qmm_affine_gemv_persistent_tiles(bits, M):
     Affine(20000, 512, bits, 64, seed=3).check_qmm(M, label=f"persistent b{bits} M={M}")
 
 
+@pytest.mark.parametrize("N,K,bits,gs,M", [
+    (264, 768, 4, 32, 1),      # 1.5 stages of 512 k: the last stage is zero-filled past K
+    (264, 768, 4, 32, 5),
+    (136, 1536, 2, 64, 2),     # 1.5 stages of 1024 k
+    (200, 384, 4, 64, 1),      # K / gs = 6 (not a multiple of 8): the per-warp-ring GEMV
+    (200, 384, 4, 64, 8),
+    (256, 4096, 8, 64, 7),     # 16 strips: K split over a cluster, 7 tokens
+    (48, 8192, 4, 128, 4),     # 3 strips: the widest K split
+])
+def test_qmm_affine_gemv_layout_edges(N, K, bits, gs, M):
+    Affine(N, K, bits, gs, seed=N + K).check_qmm(M, label=f"gemv edge {N}x{K} b{bits} gs{gs} M{M}")
+
+
 def test_qmm_affine_k_tail_and_unsupported_gemv_combo():
     # K = 96 (1.5 tensor-core K steps), and 2-bit gs32 at M=1 (no GEMV kernel: tensor-core path)
     Affine(256, 96, 4, 32).check_qmm(20, label="K tail")
