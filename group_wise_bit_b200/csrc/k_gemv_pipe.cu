@@ -54,6 +54,7 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kCW = 8;                       // warps per CTA
+constexpr int kCWLog = 3;
 constexpr int kThreads = kCW * 32;
 constexpr int kSmemPerSM = 232448;
 constexpr int kSMs = 148;
@@ -117,11 +118,13 @@ __device__ __forceinline__ void tma_load_2d_l(uint32_t dst, const CUtensorMap *m
       : "memory");
 }
 
-// Hint: bring a tile into L2 (no shared memory, no completion to wait for).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
+__device__ __forceinline__ void tma_load_3d_l(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y, int32_t z,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -196,6 +199,10 @@ struct PipeArgs {
   uint16_t *y;
   int M, N, K;
   int NS;          // strips of 16 rows
+  int ns_per, ns_rem;   // strips per CTA: ns_per, and one more for the first ns_rem CTAs
+  int w3d;         // packed words: one 3-D box per stage (else two 2-D boxes)
+  int sb_joint;    // scales and biases: one 3-D box per stage (else one each)
+  int sb_swap;     // joint box: biases come first (they sit below the scales in memory)
   int NCS;         // stages per strip in this CTA's K-slice
   int D;           // ring depth per consumer warp
   int out_strips;  // split-K only: strips per CTA that the OUT buffer holds
@@ -207,12 +214,11 @@ struct PartRec {   // a strip result that one warp holds only part of
 
 template <int BITS, int GS, int MP>
 __global__ void __launch_bounds__(kThreads, 2)
-    k_gemv_pipe(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+    k_gemv_pipe(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sb,
                 const __grid_constant__ CUtensorMap tm_b, const PipeArgs a) {
   using C = PCfg<BITS, GS>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ float red[kCW][8];
-  __shared__ float s_scale[8], s_inv[8];
   __shared__ PartRec rec[kCW][2];
   __shared__ volatile int abort_flag;
   unsigned char *base = align_smem_1024(smem_raw);
@@ -227,49 +233,36 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint4 *XB = reinterpret_cast<uint4 *>(ringSB + kCW * D * 2 * C::SBB);   // [GR][NMMA/2][4][MP]
   float4 *XNF = reinterpret_cast<float4 *>(XB + GR * (C::NMMA / 2) * 4 * MP);   // [GR][4]
   uint2 *XF = reinterpret_cast<uint2 *>(XNF + GR * 4);                // [NCS][NBM][32]
-  float *XSM = reinterpret_cast<float *>(XF + NCS * C::NBM * 32);     // [GR][8] sums, [GR][8] magic sums
-  float *PART = XSM + GR * 16;                                        // [kCW][2][16][MP]
+  float *PART = reinterpret_cast<float *>(XF + NCS * C::NBM * 32);    // [kCW][2][16][MP]
   float *OUT = PART + kCW * 2 * 16 * MP;                              // split-K: [strips][16][MP]
   uint64_t *full = reinterpret_cast<uint64_t *>(OUT + (S > 1 ? a.out_strips * 16 * MP : 0));
 
-  // ---- this CTA's strips; consumer warp w owns stages [ub(w), ub(w + 1))
-  const int sb = (int)((int64_t)blockIdx.x * a.NS / gridDim.x);
-  const int se = (int)((int64_t)(blockIdx.x + 1) * a.NS / gridDim.x);
+  // ---- this CTA's strips [sb, se) (the first ns_rem CTAs take one more), and
+  // warp w's stages [ub(w), ub(w + 1)) of them
+  const int bx = blockIdx.x;
+  const int sb = bx * a.ns_per + (bx < a.ns_rem ? bx : a.ns_rem);
+  const int se = sb + a.ns_per + (bx < a.ns_rem ? 1 : 0);
   const int ucta = (se - sb) * NCS;
-  auto ub = [&](int w) { return (int)((int64_t)w * ucta / kCW); };
+  auto ub = [&](int w) { return (int)(((int64_t)w * ucta) >> kCWLog); };
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kCW * D; i++) mbar_init(&full[i], 1);
-    fence_mbar_init();
-    abort_flag = 0;
-  }
+  if (threadIdx.x < kCW * D) mbar_init(&full[threadIdx.x], 1);
   if (threadIdx.x < kCW * 2) rec[threadIdx.x >> 1][threadIdx.x & 1] = PartRec{-1, -1};
-  for (int e = threadIdx.x; e < GR * 16; e += kThreads) XSM[e] = 0.0f;
+  for (int e = threadIdx.x; e < NCS * C::NBM * 32; e += kThreads) XF[e] = make_uint2(0u, 0u);
   if (threadIdx.x == 0) {
+    abort_flag = 0;
     tma_prefetch_desc(&tm_w);
-    tma_prefetch_desc(&tm_s);
-    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_sb);
+    if (!a.sb_joint) tma_prefetch_desc(&tm_b);
   }
+  fence_mbar_init();
   __syncthreads();
   pdl_launch_dependents();
-  const int units = ub(warp + 1) - ub(warp);
-  if (lane == 0) {
-    // While the previous kernel finishes: pull this warp's first stages into L2.
-    // Only a hint; the loads proper are issued after the wait below.
-    for (int i = 0; i < (units < D ? units : D); i++) {
-      const int u = ub(warp) + i;
-      const int strip = sb + u / NCS, ks = k0 + (u % NCS) * C::KST;
-      const int gsx = ks / GS, gbox = C::GST < 8 ? (gsx & ~7) : gsx;
-      tma_prefetch_l2_2d(&tm_w, ks / C::CPW, strip * 16);
-      tma_prefetch_l2_2d(&tm_w, ks / C::CPW + 32, strip * 16);
-      tma_prefetch_l2_2d(&tm_s, gbox, strip * 16);
-      tma_prefetch_l2_2d(&tm_b, gbox, strip * 16);
-    }
-  }
   pdl_wait();   // the previous kernel's writes (x, and possibly the weights) are visible from here on
 
-  // loads stage i of consumer warp w into its ring slot i % D
-  // loads the stage (strip, st) of this warp into its ring slot
+  // loads the stage (strip, st) of this warp into its ring slot: packed words
+  // as one 3-D box ([2 segments][16 rows][128 bytes], or two 2-D boxes) and the
+  // scale and bias boxes as one 3-D box ([2 arrays][16 rows][SBG], or two)
+  const int units = ub(warp + 1) - ub(warp);
   auto issue = [&](int strip, int st, int slot) {
     const int ks = k0 + st * C::KST;
     const uint32_t bar = smem_u32(&full[slot]);
@@ -278,10 +271,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int gsx = ks / GS;
     const int gbox = C::GST < 8 ? (gsx & ~7) : gsx;
     mbar_arrive_expect_tx(&full[slot], C::WB + 2 * C::SBB);
-    tma_load_2d_l(dw, &tm_w, ks / C::CPW, strip * 16, bar);
-    tma_load_2d_l(dw + 2048, &tm_w, ks / C::CPW + 32, strip * 16, bar);
-    tma_load_2d_l(ds, &tm_s, gbox, strip * 16, bar);
-    tma_load_2d_l(ds + C::SBB, &tm_b, gbox, strip * 16, bar);
+    if (a.w3d) {
+      tma_load_3d_l(dw, &tm_w, 0, strip * 16, ks / (32 * C::CPW), bar);
+    } else {
+      tma_load_2d_l(dw, &tm_w, ks / C::CPW, strip * 16, bar);
+      tma_load_2d_l(dw + 2048, &tm_w, ks / C::CPW + 32, strip * 16, bar);
+    }
+    if (a.sb_joint) {
+      tma_load_3d_l(ds, &tm_sb, gbox, strip * 16, 0, bar);
+    } else {
+      tma_load_2d_l(ds, &tm_sb, gbox, strip * 16, bar);
+      tma_load_2d_l(ds + C::SBB, &tm_b, gbox, strip * 16, bar);
+    }
   };
   // issue-side position (strip, stage) of this warp, advanced without divisions
   int is_strip = sb + ub(warp) / NCS, is_st = ub(warp) % NCS;
@@ -290,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (++is_st == NCS) { is_st = 0; ++is_strip; }
   }
 
-  // ---- activations of the K-slice.  Pass A: |x| max per token.
+  // ---- activations of the K-slice.  Pass A: |x| max per token (per warp).
   {
     float m[MP];
 #pragma unroll
@@ -318,24 +319,21 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   __syncthreads();
-  if (threadIdx.x < 8) {
-    const int t = threadIdx.x;
+  // Per-token power of two e: the largest |x| * 2^e lands in [2^13, 2^14), so
+  // the rescaled activations fit fp16 (every thread derives it from red[]).
+  auto token_exp = [&](int t) -> int {
     float m = 0.0f;
-    if (t < a.M)
-      for (int w = 0; w < kCW; w++) m = fmaxf(m, red[w][t]);
-    int e = 0;
-    if (m > 0.0f) {
-      int ex;
-      frexpf(m, &ex);            // m in [2^(ex-1), 2^ex): scaled max lands in [2^13, 2^14)
-      e = 14 - ex;
-      e = e > 120 ? 120 : (e < -120 ? -120 : e);
-    }
-    s_scale[t] = pow2f(e);
-    s_inv[t] = pow2f(-e);
-  }
-  __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kCW; w++) m = fmaxf(m, red[w][t]);
+    if (!(m > 0.0f)) return 0;
+    const int be = (int)((__float_as_uint(m) >> 23) & 0xffu);   // m in [2^(be-127), 2^(be-126))
+    const int e = 140 - be;                                       // 14 - (be - 126)
+    return e > 120 ? 120 : (e < -120 ? -120 : e);
+  };
   // Pass B: one thread per (group, token, quad lane c): the B fragments of the
-  // lane's codes and its share of the group's sums (combined over c in order).
+  // lane's codes, and (combined over c in order) the group's activation sum X
+  // and magic sum XN, written straight into the accumulator start quads (XNF)
+  // and the split-bf16 B operand of the bias MMAs (XF).
   {
     const int total = GR * MP * 4;
     for (int b0 = 0; b0 < total; b0 += kThreads) {
@@ -344,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int c = idx & 3, t = (idx >> 2) % MP, g = (idx >> 2) / MP;
       const int kg = k0 + g * GS;                    // first k of the group
       const bool live = valid && t < a.M && kg < a.K;
+      const float sc = pow2f(live ? token_exp(t) : 0);
       float sx = 0.0f, sn = 0.0f;
       uint32_t pr[C::NREG];
 #pragma unroll
@@ -369,8 +368,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int p = 0; p < C::CPW; p++) {
           const uint32_t bits = (p & 1) ? (raw[p >> 1] >> 16) : (raw[p >> 1] & 0xffffu);
-          const float v = bf16_val(bits) * s_scale[t < 8 ? t : 0];
-          h[p] = __half_as_ushort(__float2half_rn(v));
+          h[p] = __half_as_ushort(__float2half_rn(bf16_val(bits) * sc));
           sx += __half2float(__ushort_as_half(h[p]));
         }
 #pragma unroll
@@ -392,37 +390,23 @@ __global__ void __launch_bounds__(kThreads, 2)
       sn += __shfl_xor_sync(kFull, sn, 1);
       sx += __shfl_xor_sync(kFull, sx, 2);
       sn += __shfl_xor_sync(kFull, sn, 2);
-      if (live && c == 0) {
-        XSM[g * 8 + t] = sx;
-        XSM[GR * 8 + g * 8 + t] = -1024.0f * sn;
+      if (valid && c == 0) {
+        const float xn = live ? -1024.0f * sn : 0.0f, X = live ? sx : 0.0f;
+        // accumulator quad of quad lane t / 2: components t % 2 and t % 2 + 2
+        float *q = reinterpret_cast<float *>(XNF + g * 4 + (t >> 1));
+        q[t & 1] = xn;
+        q[(t & 1) + 2] = xn;
+        // bias-MMA B operand: stage st, box column jj = 8 bm + 2 c' + h, lane t * 4 + c'
+        const int st = g / C::GST;
+        const int gbox = C::GST < 8 ? ((g0 + st * C::GST) & ~7) - g0 : st * C::GST;
+        const int jj = g - gbox, bm = jj >> 3, cq = (jj & 7) >> 1, hh = jj & 1;
+        const __nv_bfloat16 xh = __float2bfloat16_rn(X);
+        const __nv_bfloat16 xl = __float2bfloat16_rn(X - __bfloat162float(xh));
+        uint16_t *f = reinterpret_cast<uint16_t *>(XF + (st * C::NBM + bm) * 32 + t * 4 + cq);
+        f[hh] = __bfloat16_as_ushort(xh);
+        f[2 + hh] = __bfloat16_as_ushort(xl);
       }
     }
-  }
-  __syncthreads();
-  // Pass C: magic-sum fragments (MMA accumulator start values) and the split
-  // bf16 activation sums that are the B operand of the bias MMAs.
-  for (int e = threadIdx.x; e < GR * 4; e += kThreads) {   // the accumulator quad of (group, quad lane c)
-    const int g = e >> 2, c = e & 3;
-    const float *xn = XSM + GR * 8;
-    XNF[e] = make_float4(xn[g * 8 + 2 * c], xn[g * 8 + 2 * c + 1], xn[g * 8 + 2 * c], xn[g * 8 + 2 * c + 1]);
-  }
-  for (int e = threadIdx.x; e < NCS * C::NBM * 32; e += kThreads) {
-    const int ln = e & 31, bm = (e >> 5) % C::NBM, st = (e >> 5) / C::NBM;
-    const int t = ln >> 2, c = ln & 3;
-    const int gst0 = st * C::GST;                          // first slice group of the stage
-    const int gbox = C::GST < 8 ? ((g0 + gst0) & ~7) - g0 : gst0;   // slice group of box column 0
-    uint32_t hi2 = 0u, lo2 = 0u;
-#pragma unroll
-    for (int q = 0; q < 2; q++) {
-      const int gr = gbox + bm * 8 + 2 * c + q;
-      float X = 0.0f;
-      if (t < MP && gr >= gst0 && gr < gst0 + C::GST) X = XSM[gr * 8 + t];
-      const __nv_bfloat16 h = __float2bfloat16_rn(X);
-      const __nv_bfloat16 l = __float2bfloat16_rn(X - __bfloat162float(h));
-      hi2 |= (uint32_t)__bfloat16_as_ushort(h) << (16 * q);
-      lo2 |= (uint32_t)__bfloat16_as_ushort(l) << (16 * q);
-    }
-    XF[e] = make_uint2(hi2, lo2);
   }
   __syncthreads();
 
@@ -438,6 +422,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     // fills MMA columns >= MP, which are never stored.
     const uint4 *xbl = XB + c * MP + (MP == 1 ? 0 : g8 % MP);
     const uint32_t mag = mag_reg(BITS == 8 ? 0x64646464u : 0x64006400u);
+    // undoes the per-token rescale of the lane's two tokens
+    const float inv0 = pow2f(2 * c < a.M ? -token_exp(2 * c) : 0);
+    const float inv1 = pow2f(2 * c + 1 < a.M ? -token_exp(2 * c + 1) : 0);
     constexpr int xbs = 4 * MP;
 
     constexpr int SW = C::SBG / 2;          // 32-bit words per scale-box row
@@ -452,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const bool whole = fst == 0 && lst == NCS - 1;
       float v[4];
 #pragma unroll
-      for (int i = 0; i < 4; i++) v[i] = (acc[i] + accb[i]) * s_inv[2 * c + (i & 1)];
+      for (int i = 0; i < 4; i++) v[i] = (acc[i] + accb[i]) * ((i & 1) ? inv1 : inv0);
       if (whole && S == 1) {
         const int rA = strip_ * 16 + g8;
 #pragma unroll
@@ -487,6 +474,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t sw = smem_u32(ringW + (warp * D + slot) * C::WB) + rowoff;
       const uint32_t *sp = reinterpret_cast<const uint32_t *>(ringSB + (warp * D + slot) * 2 * C::SBB);
       const uint32_t *bp = sp + C::SBB / 4;
+      if (a.sb_swap) {
+        const uint32_t *tmp = sp;
+        sp = bp;
+        bp = tmp;
+      }
       const int jb = C::GST < 8 ? ((g0 + st * C::GST) & 7) : 0;   // box column of the stage's first group
       // ---- everything this stage needs from shared memory, then release the slot
       uint32_t wd[16][2];
@@ -729,9 +721,10 @@ gwb_status run_pipe(const uint16_t *x, int M, const uint32_t *wq, const uint16_t
 
   // Plan for a K split over S CTAs of a cluster: P CTAs along the strips (at
   // most one wave), ring depth D and shared memory.
-  // With enough stages for every warp, two CTAs share an SM (twice the warps
-  // to hide latency, half the ring each).
-  struct Plan { int S, P, D, NCS, out_strips; size_t smem; };
+  // Launch plan for a K split over S CTAs of a cluster: P CTAs along the
+  // strips (one wave), ring depth D and shared memory; per_sm = 2 puts two
+  // CTAs on an SM (twice the warps to hide latency, half the ring each).
+  struct Plan { int S, P, D, NCS, out_strips; size_t smem; int est; };
   auto plan_for = [&](int S, int per_sm, Plan &pl) -> bool {
     if (nst % S != 0) return false;
     const int NCS = nst / S, KR = NCS * C::KST, GR = KR / GS;
@@ -741,52 +734,91 @@ gwb_status run_pipe(const uint16_t *x, int M, const uint32_t *wq, const uint16_t
       if (mc < 1) return false;
       P = P < mc ? P : mc;
     }
-    const int out_strips = S > 1 ? (NS + P - 1) / P : 0;
+    const int out_strips = (NS + P - 1) / P;
     const size_t fixed = (size_t)GR * (C::NMMA / 2) * 4 * MP * 16 + (size_t)GR * 4 * 16 +
-                         (size_t)NCS * C::NBM * 32 * 8 + (size_t)GR * 16 * 4 + (size_t)kCW * 2 * 16 * MP * 4 +
-                         (size_t)out_strips * 16 * MP * 4;
+                         (size_t)NCS * C::NBM * 32 * 8 + (size_t)kCW * 2 * 16 * MP * 4 +
+                         (S > 1 ? (size_t)out_strips * 16 * MP * 4 : 0);
     const size_t per = (size_t)kCW * (C::WB + 2 * C::SBB + 8);
     const size_t avail = (size_t)kSmemPerSM / per_sm - 4096 - 1024;
     if (fixed + 2 * per > avail) return false;
     int D = (int)((avail - fixed) / per);
     D = D > 6 ? 6 : D;
-    pl = Plan{S, P, D, NCS, out_strips, 1024 + fixed + (size_t)D * per};
+    // estimated critical path: stages of the busiest warp, plus the cost of a
+    // cluster barrier pair (about two stages)
+    const int est = (out_strips * NCS + kCW - 1) / kCW + (S > 1 ? 2 : 0);
+    pl = Plan{S, P, D, NCS, out_strips, 1024 + fixed + (size_t)D * per, est};
     return true;
   };
-  // Every SM gets a strip: no split.  Otherwise the split that covers the most SMs.
-  Plan best{0, 0, 0, 0, 0, 0};
+  Plan best{0, 0, 0, 0, 0, 0, 0};
   bool have = false;
-  if ((int64_t)NS * nst >= 2LL * kSMs * kCW * 4) have = plan_for(1, 2, best);
-  if (!have) have = plan_for(1, 1, best);
-  if (!have || best.P < kSMs) {
-    for (int S = 2; S <= 8; S *= 2) {
-      Plan pl{0, 0, 0, 0, 0, 0};
-      if (plan_for(S, 1, pl) && (!have || pl.S * pl.P > best.S * best.P)) {
-        best = pl;
-        have = true;
-      }
+  auto consider = [&](int S, int per_sm) {
+    Plan pl{0, 0, 0, 0, 0, 0, 0};
+    if (plan_for(S, per_sm, pl) && (!have || pl.est < best.est)) {
+      best = pl;
+      have = true;
     }
-  }
+  };
+  if ((int64_t)NS * nst >= 2LL * kSMs * kCW * 4) consider(1, 2);
+  consider(1, 1);
+  for (int S = 2; S <= 8; S *= 2) consider(S, 1);
   if (!have) return GWB_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(reinterpret_cast<const void *>(kern), best.smem))
     return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute failed for %zu bytes of shared memory", best.smem);
 
-  CUtensorMap tw, ts, tb;
-  const uint64_t words = (uint64_t)K / C::CPW;
-  CUresult r = encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, (uint64_t)N, words * 4, 32u, 16u,
-                         CU_TENSOR_MAP_SWIZZLE_128B);
-  if (r == CUDA_SUCCESS)
-    r = encode_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT16, scales, (uint64_t)G, (uint64_t)N, (uint64_t)G * 2,
-                  (uint32_t)C::SBG, 16u, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (r == CUDA_SUCCESS)
-    r = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT16, biases, (uint64_t)G, (uint64_t)N, (uint64_t)G * 2,
-                  (uint32_t)C::SBG, 16u, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (r != CUDA_SUCCESS) return fail(GWB_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-
   PipeArgs a{};
   a.x = x; a.y = y;
   a.M = M; a.N = (int)N; a.K = (int)K;
-  a.NS = NS; a.NCS = best.NCS; a.D = best.D; a.out_strips = best.out_strips;
+  a.NS = NS; a.NCS = best.NCS; a.D = best.D; a.out_strips = best.S > 1 ? best.out_strips : 0;
+  a.ns_per = NS / best.P;
+  a.ns_rem = NS % best.P;
+
+  // Packed words: one 3-D box per stage ([2 segments][16 rows][32 words]);
+  // two 2-D boxes if the driver refuses that view.
+  CUtensorMap tw, tsb, tb;
+  const uint64_t words = (uint64_t)K / C::CPW;
+  a.w3d = 0;
+  if (words % 32 == 0) {
+    const cuuint64_t dims[3] = {32, (cuuint64_t)N, words / 32};
+    const cuuint64_t strides[2] = {words * 4, 128};
+    const cuuint32_t box[3] = {32, 16, 2};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (encode_fn()(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t *>(wq), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+      a.w3d = 1;
+  }
+  CUresult r = CUDA_SUCCESS;
+  if (!a.w3d)
+    r = encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, (uint64_t)N, words * 4, 32u, 16u,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+  // Scales and biases: one 3-D box per stage over both arrays (the third
+  // dimension steps from the lower array to the higher one), else one each.
+  const uintptr_t ps = reinterpret_cast<uintptr_t>(scales), pb = reinterpret_cast<uintptr_t>(biases);
+  const uint64_t diff = ps > pb ? ps - pb : pb - ps;
+  a.sb_joint = 0;
+  a.sb_swap = pb < ps ? 1 : 0;
+  if (r == CUDA_SUCCESS && diff != 0 && diff % 16 == 0 && diff < (1ull << 39)) {
+    const cuuint64_t dims[3] = {(cuuint64_t)G, (cuuint64_t)N, 2};
+    const cuuint64_t strides[2] = {(cuuint64_t)G * 2, diff};
+    const cuuint32_t box[3] = {(cuuint32_t)C::SBG, 16, 2};
+    const cuuint32_t es[3] = {1, 1, 1};
+    const void *lo = a.sb_swap ? biases : scales;
+    if (encode_fn()(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(lo), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+      a.sb_joint = 1;
+  }
+  if (r == CUDA_SUCCESS && !a.sb_joint) {
+    a.sb_swap = 0;
+    r = encode_2d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT16, scales, (uint64_t)G, (uint64_t)N, (uint64_t)G * 2,
+                  (uint32_t)C::SBG, 16u, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (r == CUDA_SUCCESS)
+      r = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT16, biases, (uint64_t)G, (uint64_t)N, (uint64_t)G * 2,
+                    (uint32_t)C::SBG, 16u, CU_TENSOR_MAP_SWIZZLE_NONE);
+  } else {
+    tb = tsb;   // unused
+  }
+  if (r != CUDA_SUCCESS) return fail(GWB_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)best.P, (unsigned)best.S);
@@ -807,7 +839,7 @@ gwb_status run_pipe(const uint16_t *x, int M, const uint32_t *wq, const uint16_t
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, ts, tb, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tw, tsb, tb, a);
   if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "decode GEMV launch: %s", cudaGetErrorString(e));
   return GWB_OK;
 }
