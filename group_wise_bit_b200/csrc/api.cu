@@ -82,12 +82,13 @@ const char *gwb_last_error(void) { return gwb::g_msg; }
 const char *gwb_version(void) { return "group_wise_bit_b200 0.1 (sm_100a)"; }
 
 gwb_status gwb_check_device_error(void *stream) {
-  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0;
+  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0, flag5 = 0;
   GWB_TRY(gwb::read_and_clear_device_error(as_stream(stream), &flag));
   GWB_TRY(gwb::read_and_clear_device_error_stream(as_stream(stream), &flag2));
   GWB_TRY(gwb::read_and_clear_device_error_tmem(as_stream(stream), &flag3));
   GWB_TRY(gwb::read_and_clear_device_error_pipe(as_stream(stream), &flag4));
-  flag |= flag2 | flag3 | flag4;
+  GWB_TRY(gwb::read_and_clear_device_error_tc2(as_stream(stream), &flag5));
+  flag |= flag2 | flag3 | flag4 | flag5;
   if (flag) return fail(GWB_ERR_TIMEOUT, "a bounded device-side wait gave up (flag 0x%x)", flag);
   return GWB_OK;
 }
@@ -139,6 +140,11 @@ gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, cons
   }
   if (bits == 2 && K % 64 != 0)
     return fail(GWB_ERR_UNSUPPORTED, "bits=2 needs K %% 64 == 0 on the tensor-core path (K=%lld)", (long long)K);
+  if (M >= 128) {
+    const gwb_status s =
+        gwb::launch_tc2_affine(x, M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
+    if (s != GWB_ERR_UNSUPPORTED) return s;
+  }
   return gwb::launch_tc_affine(x, M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
 }
 
@@ -172,6 +178,11 @@ gwb_status gwb_gptq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, co
   if (g_idx && !aligned16(g_idx)) return fail(GWB_ERR_ALIGN, "g_idx is not 16-byte aligned");
   if (M <= 8)
     return gwb::launch_gemv_gptq(x, (int)M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream));
+  if (M >= 128) {
+    const gwb_status s =
+        gwb::launch_tc2_gptq(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream));
+    if (s != GWB_ERR_UNSUPPORTED) return s;
+  }
   return gwb::launch_tc_gptq(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream));
 }
 
@@ -223,6 +234,7 @@ gwb_status gwb_gemm_i8i4(const int8_t *qx, const float *sx, int64_t M, const uin
   GWB_TRY(need(sx, "sx"));
   GWB_TRY(need(wq, "wq"));
   GWB_TRY(need(sw, "sw"));
+  if (M >= 128) return gwb::launch_tc2_i8i4(qx, sx, M, wq, sw, N, K, y, acc, as_stream(stream));
   return gwb::launch_tc_i8i4(qx, sx, M, wq, sw, N, K, y, acc, as_stream(stream));
 }
 

@@ -1,0 +1,508 @@
+// Persistent tensor-core (tcgen05) GEMM for the prefill regime (M >= 128) of
+// the fused dequant + matmul, for the MLX affine layout (bf16, kind::f16), the
+// GPTQ layout without g_idx (fp16, kind::f16) and W4A8 (int8, kind::i8).
+//
+// As in the per-tile kernel the product is computed transposed ("swap AB"):
+// the tensor core's M side is 128 output features, its N side BT tokens.  Each
+// CTA (one per SM) walks a static list of 128 x BT output tiles (features
+// fastest, so the CTAs in flight share one activation tile through L2), and
+// its warps form a pipeline of three decoupled shared-memory rings:
+//
+//   warp 0      TMA producer of the activation ring X (BT x BK, 128-byte
+//               swizzle, zero-filled past M and K);
+//   warp 2      producer of the packed-weight ring R: lane 0 issues the TMA
+//               tile load of the step's packed words, all lanes copy the
+//               step's group scales / biases (GPTQ: scales and qzeros) with
+//               cp.async onto the same mbarrier;
+//   warps 3-10  dequantizers: R stage -> the 128 x BK A operand (bf16, fp16 or
+//               int8) in the 128-byte-swizzled K-major layout, into ring A;
+//               the R ring is deeper than X and A, so the dequantizers run
+//               ahead of the tensor core instead of waiting for each load;
+//   warp 1      TMEM allocation and the single MMA-issuing thread: per K step
+//               BK/16 (int8: BK/32) tcgen05.mma into one of two TMEM
+//               accumulators, then commits the X and A slots back;
+//   warps 11-14 epilogue: drain the finished accumulator with tcgen05.ld and
+//               write the output tile while the next tile accumulates in the
+//               other TMEM buffer.
+//
+// Every mbarrier wait is bounded (ptx.cuh); on a timeout the CTA stops issuing
+// work, drains what it issued, frees its TMEM and exits.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "dequant.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gwb {
+namespace {
+using namespace dq;
+
+constexpr int kWarps = 15;
+constexpr int kThreads = kWarps * 32;
+constexpr int kDqWarps = 8;
+constexpr int kFirstDq = 3, kFirstEpi = 11;
+constexpr int kTileN = 128;      // output features per tile (tensor-core M)
+constexpr int kMaxSmem = 232448;
+constexpr int kSMs = 148;
+
+enum class Fmt { Affine, Gptq, I8 };
+
+struct Args {
+  int M, N, K, gs;
+  int Nt, T;                // feature tiles, tiles
+  const uint16_t *scales;   // affine: bf16 [N, K/gs];   gptq: fp16 [K/gs, N]
+  const uint16_t *biases;   // affine: bf16 [N, K/gs]
+  const int32_t *qzeros;    // gptq: [K/gs, N/8]
+  const float *sx, *sw;     // i8: per-token / per-channel scales
+  uint16_t *y;              // bf16 (affine, i8) or fp16 (gptq) [M, N]
+  int32_t *acc;             // i8: optional int32 [M, N]
+};
+
+template <Fmt F, int BITS>
+struct Tr;
+template <int BITS>
+struct Tr<Fmt::Affine, BITS> {
+  static constexpr int BK = 64;                       // 64 bf16 = 128 bytes per row
+  static constexpr int RAW = kTileN * BK * BITS / 8;  // packed words of a step
+  static constexpr int SC = 1024;                     // scales + biases: 128 rows x an aligned pair of groups
+  static constexpr int NMMA = BK / 16;
+  static constexpr int CP = 32;                       // cp.async arrivals per step
+};
+template <>
+struct Tr<Fmt::Gptq, 4> {
+  static constexpr int BK = 64;
+  static constexpr int RAW = (BK / 8) * kTileN * 4;
+  static constexpr int SC = 1024;                     // 2 groups x (128 fp16 scales + 16 qzeros words)
+  static constexpr int NMMA = BK / 16;
+  static constexpr int CP = 32;
+};
+template <>
+struct Tr<Fmt::I8, 4> {
+  static constexpr int BK = 128;                      // 128 int8 = 128 bytes per row
+  static constexpr int RAW = kTileN * BK / 2;
+  static constexpr int SC = 0;
+  static constexpr int NMMA = BK / 32;
+  static constexpr int CP = 0;
+};
+
+// Ring depths: 3 A slots, as many X slots as fit next to an R ring of up to 8.
+template <Fmt F, int BITS, int BT>
+struct Plan2 {
+  static constexpr int XB = BT * 128;
+  static constexpr int AB = kTileN * 128;
+  static constexpr int RB = (Tr<F, BITS>::RAW + Tr<F, BITS>::SC + 127) / 128 * 128;
+  static constexpr int SA = 3;
+  static constexpr int BUDGET = kMaxSmem - 1024 - 1024 - 1024;   // alignment, barriers, static
+  static constexpr int SX = (BUDGET - SA * AB - 4 * RB) / XB > 6 ? 6 : (BUDGET - SA * AB - 4 * RB) / XB;
+  static constexpr int SR0 = (BUDGET - SA * AB - SX * XB) / RB;
+  static constexpr int SR = SR0 > 8 ? 8 : SR0;
+  static constexpr int SMEM = SX * XB + SA * AB + SR * RB + 1024 + 1024;
+  static_assert(SX >= 2 && SR >= 4, "shared memory too small");
+};
+
+// Dequantizes K step `k` of the tile at feature n0 (rows r, half h of the step)
+// from the R stage into the A stage.
+template <Fmt F, int BITS>
+__device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h, const unsigned char *R,
+                                             unsigned char *A) {
+  using T = Tr<F, BITS>;
+  constexpr int BK = T::BK;
+  const int kh = k * BK + h * (BK / 2);    // first k of this thread's half step
+  if constexpr (F == Fmt::Affine) {
+    int idx = kh / a.gs - (((k * BK) / a.gs) & ~1);   // group within the staged pair
+    idx = idx < 1 ? idx : 1;
+    const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW);
+    const float sf = bf16_val(sc[r * 2 + idx]);
+    const float bfv = bf16_val(sc[(kTileN + r) * 2 + idx]);
+    if constexpr (BITS == 4) {
+      const uint4 raw = *reinterpret_cast<const uint4 *>(R + (r * 8 + h * 4) * 4);
+      const __nv_bfloat162 s2b = __floats2bfloat162_rn(sf, sf), b2b = __floats2bfloat162_rn(bfv, bfv);
+      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int j = 0; j < 4; j++) *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + j)) = dq_affine4(wv[j], s2b, b2b);
+    } else if constexpr (BITS == 2) {
+      const uint2 raw = *reinterpret_cast<const uint2 *>(R + (r * 4 + h * 2) * 4);
+      const __nv_bfloat162 s2q = __floats2bfloat162_rn(sf, sf * 0.25f), b2b = __floats2bfloat162_rn(bfv, bfv);
+      uint4 c0, c1;
+      dq_affine2(raw.x, s2q, b2b, c0, c1);
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 0)) = c0;
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 1)) = c1;
+      dq_affine2(raw.y, s2q, b2b, c0, c1);
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 2)) = c0;
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 3)) = c1;
+    } else {
+      const uint4 *rp = reinterpret_cast<const uint4 *>(R + (r * 16 + h * 8) * 4);
+      const uint4 ra = rp[0], rb = rp[1];
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 0)) = dq_affine8(ra.x, ra.y, sf, bfv);
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 1)) = dq_affine8(ra.z, ra.w, sf, bfv);
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 2)) = dq_affine8(rb.x, rb.y, sf, bfv);
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 3)) = dq_affine8(rb.z, rb.w, sf, bfv);
+    }
+  } else if constexpr (F == Fmt::Gptq) {
+    int idx = kh / a.gs - (k * BK) / a.gs;
+    idx = idx < 1 ? idx : 1;
+    const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW);
+    const uint32_t *zc = reinterpret_cast<const uint32_t *>(R + T::RAW + 512);
+    const uint32_t sv = sc[idx * kTileN + r];
+    const uint32_t zv = 0x6400u | (((zc[idx * 16 + r / 8] >> ((r % 8) * 4)) & 0xFu) + 1u);
+    uint32_t s2[4], z2[4];
+#pragma unroll
+    for (int p = 0; p < 4; p++) { s2[p] = sv | (sv << 16); z2[p] = zv | (zv << 16); }
+    const uint32_t *Rw = reinterpret_cast<const uint32_t *>(R);
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const int kq = 4 * h + j;                  // k-octet within the step = chunk index
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, kq)) = dq_gptq(Rw[kq * kTileN + r], z2, s2);
+    }
+  } else {
+    const uint4 *rp = reinterpret_cast<const uint4 *>(R + (r * 16 + h * 8) * 4);
+    const uint4 ra = rp[0], rb = rp[1];
+    const uint32_t wv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      const uint2 lo = dq_i4(wv[2 * j]), hi = dq_i4(wv[2 * j + 1]);
+      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + j)) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    }
+  }
+}
+
+template <Fmt F, int BITS, int BT>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_tc2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Args a) {
+  using T = Tr<F, BITS>;
+  using P = Plan2<F, BITS, BT>;
+  constexpr int BK = T::BK;
+  constexpr int SX = P::SX, SA = P::SA, SR = P::SR;
+  constexpr uint32_t NCOLS = 2 * BT;                  // two accumulators of BT fp32 / s32 columns
+  constexpr uint32_t IDESC = (F == Fmt::I8) ? make_idesc(2, 1, kTileN, BT)
+                             : (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN, BT)
+                                                : make_idesc(1, 1, kTileN, BT);
+
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *base = align_smem_1024(smem_raw);
+  unsigned char *ringX = base;
+  unsigned char *ringA = ringX + SX * P::XB;
+  unsigned char *ringR = ringA + SA * P::AB;
+  uint64_t *xfull = reinterpret_cast<uint64_t *>(ringR + SR * P::RB);
+  uint64_t *xempty = xfull + SX;
+  uint64_t *afull = xempty + SX;
+  uint64_t *aempty = afull + SA;
+  uint64_t *rfull = aempty + SA;
+  uint64_t *rempty = rfull + SR;
+  uint64_t *accfull = rempty + SR;
+  uint64_t *accempty = accfull + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = (a.K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SX; s++) { mbar_init(&xfull[s], 1); mbar_init(&xempty[s], 1); }
+    for (int s = 0; s < SA; s++) { mbar_init(&afull[s], kDqWarps); mbar_init(&aempty[s], 1); }
+    for (int s = 0; s < SR; s++) { mbar_init(&rfull[s], 1 + T::CP); mbar_init(&rempty[s], kDqWarps); }
+    for (int b = 0; b < 2; b++) { mbar_init(&accfull[b], 1); mbar_init(&accempty[b], 4); }
+    *abort_flag = 0;
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, NCOLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ X producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < a.T && ok; t += gridDim.x) {
+        const int m0 = (t / a.Nt) * BT;
+        for (int k = 0; k < nk; k++, it++) {
+          const int s = it % SX;
+          if (*abort_flag || !mbar_wait(&xempty[s], ((it / SX) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
+          mbar_arrive_expect_tx(&xfull[s], P::XB);
+          tma_load_2d(ringX + s * P::XB, &tm_x, k * BK, m0, &xfull[s]);
+        }
+      }
+      // every issued load lands before the CTA may exit
+      for (int i = it - SX < 0 ? 0 : it - SX; i < it; i++) mbar_wait(&xfull[i % SX], (i / SX) & 1);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ R producer
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < a.T && ok; t += gridDim.x) {
+      const int n0 = (t % a.Nt) * kTileN;
+      for (int k = 0; k < nk; k++, it++) {
+        const int s = it % SR;
+        if (*abort_flag || !mbar_wait(&rempty[s], ((it / SR) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
+        unsigned char *st = ringR + s * P::RB;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&rfull[s], T::RAW);
+          if constexpr (F == Fmt::Gptq) tma_load_2d(st, &tm_w, n0, k * (BK / 8), &rfull[s]);
+          else if constexpr (F == Fmt::I8) tma_load_2d(st, &tm_w, k * (BK / 8), n0, &rfull[s]);
+          else tma_load_2d(st, &tm_w, k * (BK * BITS / 32), n0, &rfull[s]);
+        }
+        unsigned char *sc = st + T::RAW;
+        if constexpr (F == Fmt::Affine) {
+          const int G = a.K / a.gs;
+          const int gp = ((k * BK) / a.gs) & ~1;
+          for (int e = lane; e < 2 * kTileN; e += 32) {   // (array, row) -> 4 bytes: groups gp, gp+1
+            const int arr = e / kTileN, row = e % kTileN, n = n0 + row;
+            const bool okc = n < a.N && gp < G;
+            const uint16_t *src = (arr ? a.biases : a.scales) + (okc ? (int64_t)n * G + gp : 0);
+            cp_async_4(sc + e * 4, src, okc ? 4u : 0u);
+          }
+          cp_async_arrive_noinc(&rfull[s]);
+        } else if constexpr (F == Fmt::Gptq) {
+          const int G = a.K / a.gs;
+          const int gp = (k * BK) / a.gs;
+          {   // scales: 2 groups x 128 columns = 32 chunks of 16 bytes, one per lane
+            const int gi = lane >> 4, ch = lane & 15, g = gp + gi, n = n0 + ch * 8;
+            const bool okc = g < G && n < a.N;
+            cp_async_16(sc + lane * 16, a.scales + (okc ? (int64_t)g * a.N + n : 0), okc ? 16u : 0u);
+          }
+          {   // qzeros: 2 groups x 16 words, one word per lane
+            const int gi = lane >> 4, wz = lane & 15, g = gp + gi, n = n0 + wz * 8;
+            const bool okc = g < G && n < a.N;
+            cp_async_4(sc + 512 + lane * 4, a.qzeros + (okc ? (int64_t)g * (a.N / 8) + n / 8 : 0), okc ? 4u : 0u);
+          }
+          cp_async_arrive_noinc(&rfull[s]);
+        }
+      }
+    }
+    if (lane == 0)
+      for (int i = it - SR < 0 ? 0 : it - SR; i < it; i++) mbar_wait(&rfull[i % SR], (i / SR) & 1);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int xi = 0, tc = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < a.T && ok; t += gridDim.x, tc++) {
+        const int buf = tc & 1;
+        if (*abort_flag || !mbar_wait(&accempty[buf], ((tc >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * BT);
+        for (int k = 0; k < nk; k++, xi++) {
+          const int sx = xi % SX, sa = xi % SA;
+          if (*abort_flag || !mbar_wait(&afull[sa], (xi / SA) & 1) || !mbar_wait(&xfull[sx], (xi / SX) & 1)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(ringA + sa * P::AB), b0 = smem_u32(ringX + sx * P::XB);
+#pragma unroll
+          for (int kk = 0; kk < T::NMMA; kk++) {
+            const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
+            if constexpr (F == Fmt::I8) umma_i8(d, ad, bd, IDESC, (k | kk) != 0);
+            else umma_f16(d, ad, bd, IDESC, (k | kk) != 0);
+          }
+          umma_commit(&xempty[sx]);
+          umma_commit(&aempty[sa]);
+        }
+        if (!ok) break;
+        umma_commit(&accfull[buf]);
+      }
+      // the last commits' arrivals land before the CTA may exit
+      for (int i = xi - SX < 0 ? 0 : xi - SX; i < xi; i++) mbar_wait(&xempty[i % SX], (i / SX) & 1);
+      for (int i = xi - SA < 0 ? 0 : xi - SA; i < xi; i++) mbar_wait(&aempty[i % SA], (i / SA) & 1);
+    }
+  } else if (warp < kFirstEpi) {
+    // ------------------------------------------------------------ dequantizers
+    const int d = threadIdx.x - kFirstDq * 32;
+    const int r = d & (kTileN - 1), h = d >> 7;   // tile row, half of the K step
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < a.T && ok; t += gridDim.x) {
+      for (int k = 0; k < nk; k++, it++) {
+        const int sr = it % SR, sa = it % SA;
+        if (*abort_flag || !mbar_wait(&rfull[sr], (it / SR) & 1) || !mbar_wait(&aempty[sa], ((it / SA) & 1) ^ 1)) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        dequant_step<F, BITS>(a, k, r, h, ringR + sr * P::RB, ringA + sa * P::AB);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&afull[sa]);
+          mbar_arrive(&rempty[sr]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                        // TMEM lanes 32q .. 32q + 31 (this warp's quarter)
+    int tc = 0;
+    for (int t = blockIdx.x; t < a.T; t += gridDim.x, tc++) {
+      const int buf = tc & 1;
+      const int n0 = (t % a.Nt) * kTileN, m0 = (t / a.Nt) * BT;
+      if (*abort_flag || !mbar_wait(&accfull[buf], (tc >> 1) & 1)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const int row = n0 + 32 * q + lane;
+      float swn = 0.f;
+      if constexpr (F == Fmt::I8) swn = row < a.N ? a.sw[row] : 0.f;
+      for (int ch = 0; ch < BT / 16; ch++) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BT + ch * 16), v);
+        tmem_ld_wait();
+        if (row < a.N) {
+#pragma unroll
+          for (int j = 0; j < 16; j++) {
+            const int m = m0 + ch * 16 + j;
+            if (m < a.M) {
+              const int64_t o = (int64_t)m * a.N + row;
+              if constexpr (F == Fmt::I8) {
+                const int acc = static_cast<int>(v[j]) >> 4;   // the tensor core summed 16 * code
+                if (a.acc) a.acc[o] = acc;
+                if (a.y) a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn((float)acc * (a.sx[m] * swn)));
+              } else if constexpr (F == Fmt::Gptq) {
+                a.y[o] = __half_as_ushort(__float2half_rn(__uint_as_float(v[j])));
+              } else {
+                a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, NCOLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+gwb_status map2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t inner, uint64_t outer,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return fail(GWB_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GWB_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return GWB_OK;
+}
+
+template <Fmt F, int BITS, int BT>
+gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw, Args a,
+                   cudaStream_t st) {
+  using P = Plan2<F, BITS, BT>;
+  CUtensorMap tx;
+  gwb_status s = map2d(&tx, xdt, xptr, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * xelem, 128u / xelem,
+                       (uint32_t)BT, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != GWB_OK) return s;
+  a.Nt = (a.N + kTileN - 1) / kTileN;
+  a.T = a.Nt * ((a.M + BT - 1) / BT);
+  auto kern = k_tc2<F, BITS, BT>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
+  });
+  if (attr_err != cudaSuccess) return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
+  const int grid = a.T < kSMs ? a.T : kSMs;
+  kern<<<grid, kThreads, P::SMEM, st>>>(tx, tw, a);
+  return check_launch("persistent tensor-core GEMM");
+}
+
+// Token tile: 256 (half the activation traffic per flop, and twice the tensor
+// work per dequantized K step) unless the tokens fit one 128-token tile.
+int pick_bt2(int64_t M) { return M <= 128 ? 128 : 256; }
+
+template <Fmt F, int BITS>
+gwb_status dispatch2(int64_t M, const void *x, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
+                     const Args &a, cudaStream_t st) {
+  if (pick_bt2(M) == 128) return run_tc2<F, BITS, 128>(x, xdt, xelem, tw, a, st);
+  return run_tc2<F, BITS, 256>(x, xdt, xelem, tw, a, st);
+}
+
+}  // namespace
+
+gwb_status launch_tc2_affine(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
+                             const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
+                             cudaStream_t st) {
+  // scales are staged in 4-byte copies of aligned group pairs
+  if ((K / gs) % 2 != 0 || (((uintptr_t)scales | (uintptr_t)biases) & 3) != 0) return GWB_ERR_UNSUPPORTED;
+  Args a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
+  a.scales = scales; a.biases = biases; a.y = y;
+  CUtensorMap tw;
+  const uint64_t words = (uint64_t)K * bits / 32;
+  gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, (uint64_t)N, words * 4,
+                       (uint32_t)(64 * bits / 32), (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != GWB_OK) return s;
+  if (bits == 4) return dispatch2<Fmt::Affine, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, a, st);
+  if (bits == 8) return dispatch2<Fmt::Affine, 8>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, a, st);
+  return dispatch2<Fmt::Affine, 2>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, a, st);
+}
+
+gwb_status launch_tc2_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
+                           const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *y,
+                           cudaStream_t st) {
+  if (g_idx != nullptr || ((uintptr_t)scales & 15) != 0 || ((uintptr_t)qzeros & 3) != 0) return GWB_ERR_UNSUPPORTED;
+  Args a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
+  a.scales = scales; a.qzeros = qzeros; a.y = y;
+  CUtensorMap tw;
+  gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, (uint64_t)N, (uint64_t)(K / 8), (uint64_t)N * 4,
+                       (uint32_t)kTileN, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != GWB_OK) return s;
+  return dispatch2<Fmt::Gptq, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, tw, a, st);
+}
+
+gwb_status launch_tc2_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
+                           int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st) {
+  Args a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = 0;
+  a.sx = sx; a.sw = sw; a.y = y; a.acc = acc;
+  CUtensorMap tw;
+  gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, (uint64_t)(K / 8), (uint64_t)N, (uint64_t)(K / 8) * 4,
+                       16u, (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != GWB_OK) return s;
+  return dispatch2<Fmt::I8, 4>(M, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, a, st);
+}
+
+gwb_status read_and_clear_device_error_tc2(cudaStream_t st, unsigned int *flag) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(flag, g_device_error, sizeof(unsigned int));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "device error check: %s", cudaGetErrorString(e));
+  return GWB_OK;
+}
+
+}  // namespace gwb
