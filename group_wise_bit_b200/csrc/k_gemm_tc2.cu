@@ -25,8 +25,16 @@
 //               write the output tile while the next tile accumulates in the
 //               other TMEM buffer.
 //
+// With PAIR = 2 two CTAs of a cluster share one 256 x BT tile through the
+// tensor core's two-SM mode (tcgen05 cta_group::2): each CTA dequantizes its
+// own 128 feature rows (its half of A) and loads half of the BT tokens (its
+// half of B), so every SM moves half the activation bytes per flop.  The
+// leader CTA (rank 0) issues the MMAs; its barriers collect both CTAs' TMA
+// bytes and dequantizer arrivals, and its commits release the slots of both.
+//
 // Every mbarrier wait is bounded (ptx.cuh); on a timeout the CTA stops issuing
 // work, drains what it issued, frees its TMEM and exits.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -37,9 +45,72 @@
 #include "internal.h"
 #include "ptx.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace gwb {
 namespace {
 using namespace dq;
+
+// ---------------------------------------------------------------- two-SM helpers
+__device__ __forceinline__ uint32_t cta_rank_in_cluster() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory location in CTA `rank`
+__device__ __forceinline__ uint32_t map_rank(const void *p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// Arrive on a barrier of either CTA of the pair (release at CTA scope: the data
+// it publishes, a dequantized A half, is read by this CTA's own tensor core).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA tile load into this CTA's shared memory whose bytes complete on a barrier
+// of either CTA of the pair (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, int32_t x, int32_t y,
+                                                 uint32_t bar_cluster_addr) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster_addr)
+      : "memory");
+}
+__device__ __forceinline__ void umma_f16_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_i8_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Arrive once on the barrier at this offset in both CTAs of the pair when the
+// pair's MMAs issued so far complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
 
 constexpr int kWarps = 15;
 constexpr int kThreads = kWarps * 32;
@@ -53,6 +124,7 @@ enum class Fmt { Affine, Gptq, I8 };
 
 struct Args {
   int M, N, K, gs;
+  int gs_log2;              // group size = 1 << gs_log2
   int Nt, T;                // feature tiles, tiles
   const uint16_t *scales;   // affine: bf16 [N, K/gs];   gptq: fp16 [K/gs, N]
   const uint16_t *biases;   // affine: bf16 [N, K/gs]
@@ -89,15 +161,19 @@ struct Tr<Fmt::I8, 4> {
   static constexpr int CP = 0;
 };
 
-// Ring depths: 3 A slots, as many X slots as fit next to an R ring of up to 8.
-template <Fmt F, int BITS, int BT>
+// Ring depths.  A CTA pair holds half the tokens per CTA, which leaves room for
+// 6 dequantized slots (the dequantizers then run well ahead of the tensor core)
+// next to 4 activation slots; a single CTA keeps 3 A slots and fits as many
+// activation slots as it can.  The packed-weight ring takes what is left, up to 8.
+template <Fmt F, int BITS, int BT, int PAIR>
 struct Plan2 {
-  static constexpr int XB = BT * 128;
+  static constexpr int XB = BT / PAIR * 128;
   static constexpr int AB = kTileN * 128;
   static constexpr int RB = (Tr<F, BITS>::RAW + Tr<F, BITS>::SC + 127) / 128 * 128;
-  static constexpr int SA = 3;
+  static constexpr int SA = PAIR == 2 ? 6 : 3;
   static constexpr int BUDGET = kMaxSmem - 1024 - 1024 - 1024;   // alignment, barriers, static
-  static constexpr int SX = (BUDGET - SA * AB - 4 * RB) / XB > 6 ? 6 : (BUDGET - SA * AB - 4 * RB) / XB;
+  static constexpr int SXF = (BUDGET - SA * AB - 4 * RB) / XB > 6 ? 6 : (BUDGET - SA * AB - 4 * RB) / XB;
+  static constexpr int SX = PAIR == 2 && SXF > 4 ? 4 : SXF;
   static constexpr int SR0 = (BUDGET - SA * AB - SX * XB) / RB;
   static constexpr int SR = SR0 > 8 ? 8 : SR0;
   static constexpr int SMEM = SX * XB + SA * AB + SR * RB + 1024 + 1024;
@@ -113,7 +189,7 @@ __device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h,
   constexpr int BK = T::BK;
   const int kh = k * BK + h * (BK / 2);    // first k of this thread's half step
   if constexpr (F == Fmt::Affine) {
-    int idx = kh / a.gs - (((k * BK) / a.gs) & ~1);   // group within the staged pair
+    int idx = (kh >> a.gs_log2) - (((k * BK) >> a.gs_log2) & ~1);   // group within the staged pair
     idx = idx < 1 ? idx : 1;
     const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW);
     const float sf = bf16_val(sc[r * 2 + idx]);
@@ -143,7 +219,7 @@ __device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h,
       *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 3)) = dq_affine8(rb.z, rb.w, sf, bfv);
     }
   } else if constexpr (F == Fmt::Gptq) {
-    int idx = kh / a.gs - (k * BK) / a.gs;
+    int idx = (kh >> a.gs_log2) - ((k * BK) >> a.gs_log2);
     idx = idx < 1 ? idx : 1;
     const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW);
     const uint32_t *zc = reinterpret_cast<const uint32_t *>(R + T::RAW + 512);
@@ -170,17 +246,18 @@ __device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h,
   }
 }
 
-template <Fmt F, int BITS, int BT>
+template <Fmt F, int BITS, int BT, int PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     k_tc2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Args a) {
   using T = Tr<F, BITS>;
-  using P = Plan2<F, BITS, BT>;
+  using P = Plan2<F, BITS, BT, PAIR>;
   constexpr int BK = T::BK;
   constexpr int SX = P::SX, SA = P::SA, SR = P::SR;
+  constexpr int XT = BT / PAIR;                        // tokens of this CTA's activation slot
   constexpr uint32_t NCOLS = 2 * BT;                  // two accumulators of BT fp32 / s32 columns
-  constexpr uint32_t IDESC = (F == Fmt::I8) ? make_idesc(2, 1, kTileN, BT)
-                             : (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN, BT)
-                                                : make_idesc(1, 1, kTileN, BT);
+  constexpr uint32_t IDESC = (F == Fmt::I8) ? make_idesc(2, 1, kTileN * PAIR, BT)
+                             : (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN * PAIR, BT)
+                                                : make_idesc(1, 1, kTileN * PAIR, BT);
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *base = align_smem_1024(smem_raw);
@@ -200,49 +277,69 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = (a.K + BK - 1) / BK;
+  // tile walk: this CTA's pair (or itself) and its rank within the pair
+  const int rank = PAIR == 2 ? (int)cta_rank_in_cluster() : 0;
+  const int unit = blockIdx.x / PAIR, units = gridDim.x / PAIR;
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; s++) { mbar_init(&xfull[s], 1); mbar_init(&xempty[s], 1); }
-    for (int s = 0; s < SA; s++) { mbar_init(&afull[s], kDqWarps); mbar_init(&aempty[s], 1); }
+    for (int s = 0; s < SA; s++) { mbar_init(&afull[s], kDqWarps * PAIR); mbar_init(&aempty[s], 1); }
     for (int s = 0; s < SR; s++) { mbar_init(&rfull[s], 1 + T::CP); mbar_init(&rempty[s], kDqWarps); }
-    for (int b = 0; b < 2; b++) { mbar_init(&accfull[b], 1); mbar_init(&accempty[b], 4); }
+    for (int b = 0; b < 2; b++) { mbar_init(&accfull[b], 1); mbar_init(&accempty[b], 4 * PAIR); }
     *abort_flag = 0;
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, NCOLS);
-    tmem_relinquish();
+    if constexpr (PAIR == 2) {
+      tmem_alloc_pair(tmem_slot, NCOLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, NCOLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR == 2) cg::this_cluster().sync();   // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the leader's copies of the barriers both CTAs report to
+  const uint32_t lead_afull = PAIR == 2 ? map_rank(afull, 0) : 0u;
+  const uint32_t lead_accempty = PAIR == 2 ? map_rank(accempty, 0) : 0u;
+  const uint32_t lead_xfull = PAIR == 2 ? map_rank(xfull, 0) : 0u;
 
   if (warp == 0) {
     // ------------------------------------------------------------ X producer
     if (lane == 0) {
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < a.T && ok; t += gridDim.x) {
-        const int m0 = (t / a.Nt) * BT;
+      for (int t = unit; t < a.T && ok; t += units) {
+        const int mx = (t / a.Nt) * BT + rank * XT;    // first token of this CTA's half
         for (int k = 0; k < nk; k++, it++) {
           const int s = it % SX;
           if (*abort_flag || !mbar_wait(&xempty[s], ((it / SX) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
-          mbar_arrive_expect_tx(&xfull[s], P::XB);
-          tma_load_2d(ringX + s * P::XB, &tm_x, k * BK, m0, &xfull[s]);
+          if constexpr (PAIR == 2) {
+            if (leader) mbar_arrive_expect_tx(&xfull[s], 2 * P::XB);
+            tma_load_2d_pair(ringX + s * P::XB, &tm_x, k * BK, mx, lead_xfull + s * 8);
+          } else {
+            mbar_arrive_expect_tx(&xfull[s], P::XB);
+            tma_load_2d(ringX + s * P::XB, &tm_x, k * BK, mx, &xfull[s]);
+          }
         }
       }
-      // every issued load lands before the CTA may exit
-      for (int i = it - SX < 0 ? 0 : it - SX; i < it; i++) mbar_wait(&xfull[i % SX], (i / SX) & 1);
+      // every issued load lands before the CTA may exit (the leader sees both halves)
+      if (leader)
+        for (int i = it - SX < 0 ? 0 : it - SX; i < it; i++) mbar_wait(&xfull[i % SX], (i / SX) & 1);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ R producer
     int it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < a.T && ok; t += gridDim.x) {
-      const int n0 = (t % a.Nt) * kTileN;
+    for (int t = unit; t < a.T && ok; t += units) {
+      const int n0 = (t % a.Nt) * kTileN * PAIR + rank * kTileN;
       for (int k = 0; k < nk; k++, it++) {
         const int s = it % SR;
         if (*abort_flag || !mbar_wait(&rempty[s], ((it / SR) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
@@ -256,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         unsigned char *sc = st + T::RAW;
         if constexpr (F == Fmt::Affine) {
           const int G = a.K / a.gs;
-          const int gp = ((k * BK) / a.gs) & ~1;
+          const int gp = ((k * BK) >> a.gs_log2) & ~1;
           for (int e = lane; e < 2 * kTileN; e += 32) {   // (array, row) -> 4 bytes: groups gp, gp+1
             const int arr = e / kTileN, row = e % kTileN, n = n0 + row;
             const bool okc = n < a.N && gp < G;
@@ -266,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           cp_async_arrive_noinc(&rfull[s]);
         } else if constexpr (F == Fmt::Gptq) {
           const int G = a.K / a.gs;
-          const int gp = (k * BK) / a.gs;
+          const int gp = (k * BK) >> a.gs_log2;
           {   // scales: 2 groups x 128 columns = 32 chunks of 16 bytes, one per lane
             const int gi = lane >> 4, ch = lane & 15, g = gp + gi, n = n0 + ch * 8;
             const bool okc = g < G && n < a.N;
@@ -284,11 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0)
       for (int i = it - SR < 0 ? 0 : it - SR; i < it; i++) mbar_wait(&rfull[i % SR], (i / SR) & 1);
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (the leader's)
+    if (lane == 0 && leader) {
       int xi = 0, tc = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < a.T && ok; t += gridDim.x, tc++) {
+      for (int t = unit; t < a.T && ok; t += units, tc++) {
         const int buf = tc & 1;
         if (*abort_flag || !mbar_wait(&accempty[buf], ((tc >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
         tc_fence_after();
@@ -305,14 +402,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < T::NMMA; kk++) {
             const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
-            if constexpr (F == Fmt::I8) umma_i8(d, ad, bd, IDESC, (k | kk) != 0);
-            else umma_f16(d, ad, bd, IDESC, (k | kk) != 0);
+            if constexpr (PAIR == 2) {
+              if constexpr (F == Fmt::I8) umma_i8_pair(d, ad, bd, IDESC, (k | kk) != 0);
+              else umma_f16_pair(d, ad, bd, IDESC, (k | kk) != 0);
+            } else {
+              if constexpr (F == Fmt::I8) umma_i8(d, ad, bd, IDESC, (k | kk) != 0);
+              else umma_f16(d, ad, bd, IDESC, (k | kk) != 0);
+            }
           }
-          umma_commit(&xempty[sx]);
-          umma_commit(&aempty[sa]);
+          if constexpr (PAIR == 2) {
+            umma_commit_pair(&xempty[sx]);
+            umma_commit_pair(&aempty[sa]);
+          } else {
+            umma_commit(&xempty[sx]);
+            umma_commit(&aempty[sa]);
+          }
         }
         if (!ok) break;
-        umma_commit(&accfull[buf]);
+        if constexpr (PAIR == 2) umma_commit_pair(&accfull[buf]);
+        else umma_commit(&accfull[buf]);
       }
       // the last commits' arrivals land before the CTA may exit
       for (int i = xi - SX < 0 ? 0 : xi - SX; i < xi; i++) mbar_wait(&xempty[i % SX], (i / SX) & 1);
@@ -324,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = d & (kTileN - 1), h = d >> 7;   // tile row, half of the K step
     int it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < a.T && ok; t += gridDim.x) {
+    for (int t = unit; t < a.T && ok; t += units) {
       for (int k = 0; k < nk; k++, it++) {
         const int sr = it % SR, sa = it % SA;
         if (*abort_flag || !mbar_wait(&rfull[sr], (it / SR) & 1) || !mbar_wait(&aempty[sa], ((it / SA) & 1) ^ 1)) {
@@ -336,7 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&afull[sa]);
+          if constexpr (PAIR == 2) mbar_arrive_remote(lead_afull + sa * 8);
+          else mbar_arrive(&afull[sa]);
           mbar_arrive(&rempty[sr]);
         }
       }
@@ -345,9 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                        // TMEM lanes 32q .. 32q + 31 (this warp's quarter)
     int tc = 0;
-    for (int t = blockIdx.x; t < a.T; t += gridDim.x, tc++) {
+    for (int t = unit; t < a.T; t += units, tc++) {
       const int buf = tc & 1;
-      const int n0 = (t % a.Nt) * kTileN, m0 = (t / a.Nt) * BT;
+      const int n0 = (t % a.Nt) * kTileN * PAIR + rank * kTileN, m0 = (t / a.Nt) * BT;
       if (*abort_flag || !mbar_wait(&accfull[buf], (tc >> 1) & 1)) { *abort_flag = 1; break; }
       tc_fence_after();
       const int row = n0 + 32 * q + lane;
@@ -378,14 +487,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[buf]);
+      if (lane == 0) {
+        if constexpr (PAIR == 2) mbar_arrive_remote(lead_accempty + buf * 8);
+        else mbar_arrive(&accempty[buf]);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR == 2) cg::this_cluster().sync();   // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, NCOLS);
+    if constexpr (PAIR == 2) tmem_dealloc_pair(tmem, NCOLS);
+    else tmem_dealloc(tmem, NCOLS);
   }
 }
 
@@ -417,37 +531,48 @@ gwb_status map2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64
   return GWB_OK;
 }
 
-template <Fmt F, int BITS, int BT>
+template <Fmt F, int BITS, int BT, int PAIR>
 gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw, Args a,
                    cudaStream_t st) {
-  using P = Plan2<F, BITS, BT>;
+  using P = Plan2<F, BITS, BT, PAIR>;
   CUtensorMap tx;
   gwb_status s = map2d(&tx, xdt, xptr, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * xelem, 128u / xelem,
-                       (uint32_t)BT, CU_TENSOR_MAP_SWIZZLE_128B);
+                       (uint32_t)(BT / PAIR), CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != GWB_OK) return s;
-  a.Nt = (a.N + kTileN - 1) / kTileN;
+  a.Nt = (a.N + kTileN * PAIR - 1) / (kTileN * PAIR);
   a.T = a.Nt * ((a.M + BT - 1) / BT);
-  auto kern = k_tc2<F, BITS, BT>;
+  auto kern = k_tc2<F, BITS, BT, PAIR>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
   });
   if (attr_err != cudaSuccess) return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
-  const int grid = a.T < kSMs ? a.T : kSMs;
-  kern<<<grid, kThreads, P::SMEM, st>>>(tx, tw, a);
-  return check_launch("persistent tensor-core GEMM");
+  const int units = kSMs / PAIR;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(PAIR * (a.T < units ? a.T : units)));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = P::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)PAIR;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = PAIR == 2 ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tw, a);
+  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "persistent tensor-core GEMM: %s", cudaGetErrorString(e));
+  return GWB_OK;
 }
 
-// Token tile: 256 (half the activation traffic per flop, and twice the tensor
-// work per dequantized K step) unless the tokens fit one 128-token tile.
-int pick_bt2(int64_t M) { return M <= 128 ? 128 : 256; }
-
+// Tokens above one 128-token tile: 256 x 256 tiles on CTA pairs (two-SM MMA,
+// half the activation bytes per SM); else 128 x 128 tiles on single CTAs.
 template <Fmt F, int BITS>
 gwb_status dispatch2(int64_t M, const void *x, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
                      const Args &a, cudaStream_t st) {
-  if (pick_bt2(M) == 128) return run_tc2<F, BITS, 128>(x, xdt, xelem, tw, a, st);
-  return run_tc2<F, BITS, 256>(x, xdt, xelem, tw, a, st);
+  if (M <= 128) return run_tc2<F, BITS, 128, 1>(x, xdt, xelem, tw, a, st);
+  return run_tc2<F, BITS, 256, 2>(x, xdt, xelem, tw, a, st);
 }
 
 }  // namespace
@@ -459,6 +584,7 @@ gwb_status launch_tc2_affine(const uint16_t *x, int64_t M, const uint32_t *wq, c
   if ((K / gs) % 2 != 0 || (((uintptr_t)scales | (uintptr_t)biases) & 3) != 0) return GWB_ERR_UNSUPPORTED;
   Args a{};
   a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
+  a.gs_log2 = gs == 32 ? 5 : (gs == 64 ? 6 : 7);
   a.scales = scales; a.biases = biases; a.y = y;
   CUtensorMap tw;
   const uint64_t words = (uint64_t)K * bits / 32;
@@ -476,6 +602,7 @@ gwb_status launch_tc2_gptq(const uint16_t *x, int64_t M, const int32_t *qweight,
   if (g_idx != nullptr || ((uintptr_t)scales & 15) != 0 || ((uintptr_t)qzeros & 3) != 0) return GWB_ERR_UNSUPPORTED;
   Args a{};
   a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
+  a.gs_log2 = gs == 32 ? 5 : (gs == 64 ? 6 : 7);
   a.scales = scales; a.qzeros = qzeros; a.y = y;
   CUtensorMap tw;
   gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, (uint64_t)N, (uint64_t)(K / 8), (uint64_t)N * 4,
