@@ -92,6 +92,14 @@ __device__ __forceinline__ void umma_i8_pair(uint32_t d, uint64_t a, uint64_t b,
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
+// 3-D tile load (x, y, z = 0 .. box) into this CTA's shared memory.
+__device__ __forceinline__ void tma_load_3d_sb(void *dst, const CUtensorMap *map, int32_t x, int32_t y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(0), "r"(smem_u32(bar))
+      : "memory");
+}
 // Arrive once on the barrier at this offset in both CTAs of the pair when the
 // pair's MMAs issued so far complete.
 __device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
@@ -125,6 +133,8 @@ enum class Fmt { Affine, Gptq, I8 };
 struct Args {
   int M, N, K, gs;
   int gs_log2;              // group size = 1 << gs_log2
+  int sc_tma;               // affine: scales + biases arrive by TMA as [2 arrays][128 rows][8 groups]
+  int sc_swap;              //   ... with the biases first (they sit below the scales in memory)
   int Nt, T;                // feature tiles, tiles
   const uint16_t *scales;   // affine: bf16 [N, K/gs];   gptq: fp16 [K/gs, N]
   const uint16_t *biases;   // affine: bf16 [N, K/gs]
@@ -140,9 +150,9 @@ template <int BITS>
 struct Tr<Fmt::Affine, BITS> {
   static constexpr int BK = 64;                       // 64 bf16 = 128 bytes per row
   static constexpr int RAW = kTileN * BK * BITS / 8;  // packed words of a step
-  static constexpr int SC = 1024;                     // scales + biases: 128 rows x an aligned pair of groups
+  static constexpr int SC = 4096;                     // scales + biases: 2 x 128 rows x 8 groups (or a pair by cp.async)
   static constexpr int NMMA = BK / 16;
-  static constexpr int CP = 32;                       // cp.async arrivals per step
+  static constexpr int CP = 32;                       // cp.async arrivals per step (when not by TMA)
 };
 template <>
 struct Tr<Fmt::Gptq, 4> {
@@ -189,11 +199,25 @@ __device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h,
   constexpr int BK = T::BK;
   const int kh = k * BK + h * (BK / 2);    // first k of this thread's half step
   if constexpr (F == Fmt::Affine) {
-    int idx = (kh >> a.gs_log2) - (((k * BK) >> a.gs_log2) & ~1);   // group within the staged pair
-    idx = idx < 1 ? idx : 1;
-    const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW);
-    const float sf = bf16_val(sc[r * 2 + idx]);
-    const float bfv = bf16_val(sc[(kTileN + r) * 2 + idx]);
+    float sf, bfv;
+    if (a.sc_tma) {
+      // the row's 8 scales (16 bytes, one conflict-free load) of the aligned
+      // block of 8 groups that holds this half step's group
+      const int g8 = (kh >> a.gs_log2) & 7;
+      const uint4 *box = reinterpret_cast<const uint4 *>(R + T::RAW);
+      const uint4 vs = box[a.sc_swap ? kTileN + r : r], vb = box[a.sc_swap ? r : kTileN + r];
+      const int wsel = g8 >> 1;
+      const uint32_t ws = wsel == 0 ? vs.x : wsel == 1 ? vs.y : wsel == 2 ? vs.z : vs.w;
+      const uint32_t wb = wsel == 0 ? vb.x : wsel == 1 ? vb.y : wsel == 2 ? vb.z : vb.w;
+      sf = __uint_as_float((g8 & 1) ? (ws & 0xffff0000u) : (ws << 16));
+      bfv = __uint_as_float((g8 & 1) ? (wb & 0xffff0000u) : (wb << 16));
+    } else {
+      int idx = (kh >> a.gs_log2) - (((k * BK) >> a.gs_log2) & ~1);   // group within the staged pair
+      idx = idx < 1 ? idx : 1;
+      const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW);
+      sf = bf16_val(sc[r * 2 + idx]);
+      bfv = bf16_val(sc[(kTileN + r) * 2 + idx]);
+    }
     if constexpr (BITS == 4) {
       const uint4 raw = *reinterpret_cast<const uint4 *>(R + (r * 8 + h * 4) * 4);
       const __nv_bfloat162 s2b = __floats2bfloat162_rn(sf, sf), b2b = __floats2bfloat162_rn(bfv, bfv);
@@ -248,7 +272,8 @@ __device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h,
 
 template <Fmt F, int BITS, int BT, int PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_tc2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Args a) {
+    k_tc2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+          const __grid_constant__ CUtensorMap tm_sb, const Args a) {
   using T = Tr<F, BITS>;
   using P = Plan2<F, BITS, BT, PAIR>;
   constexpr int BK = T::BK;
@@ -285,11 +310,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; s++) { mbar_init(&xfull[s], 1); mbar_init(&xempty[s], 1); }
     for (int s = 0; s < SA; s++) { mbar_init(&afull[s], kDqWarps * PAIR); mbar_init(&aempty[s], 1); }
-    for (int s = 0; s < SR; s++) { mbar_init(&rfull[s], 1 + T::CP); mbar_init(&rempty[s], kDqWarps); }
+    for (int s = 0; s < SR; s++) {
+      mbar_init(&rfull[s], 1 + (F == Fmt::Affine && a.sc_tma ? 0 : T::CP));
+      mbar_init(&rempty[s], kDqWarps);
+    }
     for (int b = 0; b < 2; b++) { mbar_init(&accfull[b], 1); mbar_init(&accempty[b], 4 * PAIR); }
     *abort_flag = 0;
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
+    if (F == Fmt::Affine && a.sc_tma) tma_prefetch_desc(&tm_sb);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -345,13 +374,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*abort_flag || !mbar_wait(&rempty[s], ((it / SR) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
         unsigned char *st = ringR + s * P::RB;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&rfull[s], T::RAW);
+          const bool sct = F == Fmt::Affine && a.sc_tma;
+          mbar_arrive_expect_tx(&rfull[s], T::RAW + (sct ? 4096 : 0));
           if constexpr (F == Fmt::Gptq) tma_load_2d(st, &tm_w, n0, k * (BK / 8), &rfull[s]);
           else if constexpr (F == Fmt::I8) tma_load_2d(st, &tm_w, k * (BK / 8), n0, &rfull[s]);
           else tma_load_2d(st, &tm_w, k * (BK * BITS / 32), n0, &rfull[s]);
+          if (sct) tma_load_3d_sb(st + T::RAW, &tm_sb, ((k * BK) >> a.gs_log2) & ~7, n0, &rfull[s]);
         }
         unsigned char *sc = st + T::RAW;
         if constexpr (F == Fmt::Affine) {
+          if (!a.sc_tma) {
           const int G = a.K / a.gs;
           const int gp = ((k * BK) >> a.gs_log2) & ~1;
           for (int e = lane; e < 2 * kTileN; e += 32) {   // (array, row) -> 4 bytes: groups gp, gp+1
@@ -361,6 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             cp_async_4(sc + e * 4, src, okc ? 4u : 0u);
           }
           cp_async_arrive_noinc(&rfull[s]);
+          }
         } else if constexpr (F == Fmt::Gptq) {
           const int G = a.K / a.gs;
           const int gp = (k * BK) >> a.gs_log2;
@@ -532,8 +565,8 @@ gwb_status map2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64
 }
 
 template <Fmt F, int BITS, int BT, int PAIR>
-gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw, Args a,
-                   cudaStream_t st) {
+gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
+                   const CUtensorMap &tsb, Args a, cudaStream_t st) {
   using P = Plan2<F, BITS, BT, PAIR>;
   CUtensorMap tx;
   gwb_status s = map2d(&tx, xdt, xptr, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * xelem, 128u / xelem,
@@ -561,7 +594,7 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = PAIR == 2 ? 1 : 0;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tw, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tx, tw, tsb, a);
   if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "persistent tensor-core GEMM: %s", cudaGetErrorString(e));
   return GWB_OK;
 }
@@ -570,9 +603,9 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
 // half the activation bytes per SM); else 128 x 128 tiles on single CTAs.
 template <Fmt F, int BITS>
 gwb_status dispatch2(int64_t M, const void *x, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
-                     const Args &a, cudaStream_t st) {
-  if (M <= 128) return run_tc2<F, BITS, 128, 1>(x, xdt, xelem, tw, a, st);
-  return run_tc2<F, BITS, 256, 2>(x, xdt, xelem, tw, a, st);
+                     const CUtensorMap &tsb, const Args &a, cudaStream_t st) {
+  if (M <= 128) return run_tc2<F, BITS, 128, 1>(x, xdt, xelem, tw, tsb, a, st);
+  return run_tc2<F, BITS, 256, 2>(x, xdt, xelem, tw, tsb, a, st);
 }
 
 }  // namespace
@@ -586,14 +619,33 @@ gwb_status launch_tc2_affine(const uint16_t *x, int64_t M, const uint32_t *wq, c
   a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
   a.gs_log2 = gs == 32 ? 5 : (gs == 64 ? 6 : 7);
   a.scales = scales; a.biases = biases; a.y = y;
-  CUtensorMap tw;
+  CUtensorMap tw, tsb;
   const uint64_t words = (uint64_t)K * bits / 32;
   gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, (uint64_t)N, words * 4,
                        (uint32_t)(64 * bits / 32), (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (s != GWB_OK) return s;
-  if (bits == 4) return dispatch2<Fmt::Affine, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, a, st);
-  if (bits == 8) return dispatch2<Fmt::Affine, 8>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, a, st);
-  return dispatch2<Fmt::Affine, 2>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, a, st);
+  // Scales and biases by TMA: one 3-D box [2 arrays][128 rows][8 groups] per K
+  // step over both arrays (the third dimension steps from the lower array to
+  // the higher one); needs 16-byte scale rows.  Else 4-byte cp.async copies.
+  const int64_t G = K / gs;
+  const uintptr_t ps = (uintptr_t)scales, pb = (uintptr_t)biases;
+  const uint64_t diff = ps > pb ? ps - pb : pb - ps;
+  a.sc_tma = 0;
+  a.sc_swap = pb < ps ? 1 : 0;
+  tsb = tw;
+  if (G % 8 == 0 && diff != 0 && diff % 16 == 0 && diff < (1ull << 39)) {
+    const cuuint64_t dims[3] = {(cuuint64_t)G, (cuuint64_t)N, 2};
+    const cuuint64_t strides[2] = {(cuuint64_t)G * 2, diff};
+    const cuuint32_t box[3] = {8, (cuuint32_t)kTileN, 2};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (encode_fn()(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, (void *)(a.sc_swap ? pb : ps), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+      a.sc_tma = 1;
+  }
+  if (bits == 4) return dispatch2<Fmt::Affine, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, tsb, a, st);
+  if (bits == 8) return dispatch2<Fmt::Affine, 8>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, tsb, a, st);
+  return dispatch2<Fmt::Affine, 2>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, tsb, a, st);
 }
 
 gwb_status launch_tc2_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
@@ -608,7 +660,7 @@ gwb_status launch_tc2_gptq(const uint16_t *x, int64_t M, const int32_t *qweight,
   gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, (uint64_t)N, (uint64_t)(K / 8), (uint64_t)N * 4,
                        (uint32_t)kTileN, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (s != GWB_OK) return s;
-  return dispatch2<Fmt::Gptq, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, tw, a, st);
+  return dispatch2<Fmt::Gptq, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, tw, tw, a, st);
 }
 
 gwb_status launch_tc2_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
@@ -620,7 +672,7 @@ gwb_status launch_tc2_i8i4(const int8_t *qx, const float *sx, int64_t M, const u
   gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, (uint64_t)(K / 8), (uint64_t)N, (uint64_t)(K / 8) * 4,
                        16u, (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (s != GWB_OK) return s;
-  return dispatch2<Fmt::I8, 4>(M, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, a, st);
+  return dispatch2<Fmt::I8, 4>(M, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
 }
 
 gwb_status read_and_clear_device_error_tc2(cudaStream_t st, unsigned int *flag) {
