@@ -39,7 +39,10 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "dequant.cuh"
 #include "internal.h"
@@ -100,6 +103,24 @@ __device__ __forceinline__ void tma_load_3d_sb(void *dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(0), "r"(smem_u32(bar))
       : "memory");
 }
+// Stream-K handshake on a global word: publish (release) the epoch once this
+// CTA's partial is stored; wait (acquire, bounded) until a peer published it.
+__device__ __forceinline__ void flag_publish(uint32_t *f, uint32_t epoch) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(epoch) : "memory");
+}
+__device__ __forceinline__ bool flag_wait(const uint32_t *f, uint32_t epoch) {
+  const unsigned long long t0 = clock64();
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    if (v == epoch) return true;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(&g_device_error, 1u);
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
 // Arrive once on the barrier at this offset in both CTAs of the pair when the
 // pair's MMAs issued so far complete.
 __device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
@@ -142,6 +163,37 @@ struct Args {
   const float *sx, *sw;     // i8: per-token / per-channel scales
   uint16_t *y;              // bf16 (affine, i8) or fp16 (gptq) [M, N]
   int32_t *acc;             // i8: optional int32 [M, N]
+  // stream-K: partial tiles through a workspace (null: whole tiles per unit)
+  uint32_t *ws;             // [CTAs][BT tokens][128 rows] fp32 (i8: s32) partial accumulators
+  uint32_t *flags;          // [CTAs] epoch at which the CTA's partial is complete
+  uint32_t epoch;           // this launch's epoch (never 0)
+};
+
+// A unit's contiguous share of the flattened (tile, K step) iteration space,
+// walked as segments of one tile each.  With a workspace the shares are equal
+// (stream-K: a tile may be split between units); without one they are whole
+// tiles.
+struct SegWalk {
+  int64_t L, Le;
+  int nk;
+  __device__ SegWalk(const Args &a, int nk_, int unit, int units) : nk(nk_) {
+    const int64_t W = (int64_t)a.T * nk_;
+    if (a.ws) {
+      L = (int64_t)unit * W / units;
+      Le = (int64_t)(unit + 1) * W / units;
+    } else {
+      L = (int64_t)unit * a.T / units * nk_;
+      Le = (int64_t)(unit + 1) * a.T / units * nk_;
+    }
+  }
+  __device__ bool next(int &t, int &k0, int &k1) {
+    if (L >= Le) return false;
+    t = (int)(L / nk);
+    k0 = (int)(L - (int64_t)t * nk);
+    k1 = (Le - L) < (int64_t)(nk - k0) ? k0 + (int)(Le - L) : nk;
+    L += k1 - k0;
+    return true;
+  }
 };
 
 template <Fmt F, int BITS>
@@ -343,11 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ X producer
     if (lane == 0) {
-      int it = 0;
+      int it = 0, t, k0, k1;
       bool ok = true;
-      for (int t = unit; t < a.T && ok; t += units) {
+      SegWalk sw(a, nk, unit, units);
+      while (ok && sw.next(t, k0, k1)) {
         const int mx = (t / a.Nt) * BT + rank * XT;    // first token of this CTA's half
-        for (int k = 0; k < nk; k++, it++) {
+        for (int k = k0; k < k1; k++, it++) {
           const int s = it % SX;
           if (*abort_flag || !mbar_wait(&xempty[s], ((it / SX) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
           if constexpr (PAIR == 2) {
@@ -365,11 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ R producer
-    int it = 0;
+    int it = 0, t, k0, k1;
     bool ok = true;
-    for (int t = unit; t < a.T && ok; t += units) {
+    SegWalk sw(a, nk, unit, units);
+    while (ok && sw.next(t, k0, k1)) {
       const int n0 = (t % a.Nt) * kTileN * PAIR + rank * kTileN;
-      for (int k = 0; k < nk; k++, it++) {
+      for (int k = k0; k < k1; k++, it++) {
         const int s = it % SR;
         if (*abort_flag || !mbar_wait(&rempty[s], ((it / SR) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
         unsigned char *st = ringR + s * P::RB;
@@ -416,14 +470,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (the leader's)
     if (lane == 0 && leader) {
-      int xi = 0, tc = 0;
+      int xi = 0, tc = 0, t, k0, k1;
       bool ok = true;
-      for (int t = unit; t < a.T && ok; t += units, tc++) {
+      SegWalk sw(a, nk, unit, units);
+      for (; ok && sw.next(t, k0, k1); tc++) {
         const int buf = tc & 1;
         if (*abort_flag || !mbar_wait(&accempty[buf], ((tc >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(buf * BT);
-        for (int k = 0; k < nk; k++, xi++) {
+        for (int k = k0; k < k1; k++, xi++) {
           const int sx = xi % SX, sa = xi % SA;
           if (*abort_flag || !mbar_wait(&afull[sa], (xi / SA) & 1) || !mbar_wait(&xfull[sx], (xi / SX) & 1)) {
             *abort_flag = 1;
@@ -436,11 +491,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < T::NMMA; kk++) {
             const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
             if constexpr (PAIR == 2) {
-              if constexpr (F == Fmt::I8) umma_i8_pair(d, ad, bd, IDESC, (k | kk) != 0);
-              else umma_f16_pair(d, ad, bd, IDESC, (k | kk) != 0);
+              if constexpr (F == Fmt::I8) umma_i8_pair(d, ad, bd, IDESC, (k - k0) | kk);
+              else umma_f16_pair(d, ad, bd, IDESC, (k - k0) | kk);
             } else {
-              if constexpr (F == Fmt::I8) umma_i8(d, ad, bd, IDESC, (k | kk) != 0);
-              else umma_f16(d, ad, bd, IDESC, (k | kk) != 0);
+              if constexpr (F == Fmt::I8) umma_i8(d, ad, bd, IDESC, (k - k0) | kk);
+              else umma_f16(d, ad, bd, IDESC, (k - k0) | kk);
             }
           }
           if constexpr (PAIR == 2) {
@@ -463,10 +518,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ dequantizers
     const int d = threadIdx.x - kFirstDq * 32;
     const int r = d & (kTileN - 1), h = d >> 7;   // tile row, half of the K step
-    int it = 0;
+    int it = 0, t, k0, k1;
     bool ok = true;
-    for (int t = unit; t < a.T && ok; t += units) {
-      for (int k = 0; k < nk; k++, it++) {
+    SegWalk sw(a, nk, unit, units);
+    while (ok && sw.next(t, k0, k1)) {
+      for (int k = k0; k < k1; k++, it++) {
         const int sr = it % SR, sa = it % SA;
         if (*abort_flag || !mbar_wait(&rfull[sr], (it / SR) & 1) || !mbar_wait(&aempty[sa], ((it / SA) & 1) ^ 1)) {
           *abort_flag = 1;
@@ -485,23 +541,82 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Per segment: a whole tile is written out; a segment that starts inside
+    // its tile (this unit's first) is stored as a partial for the unit that
+    // holds the tile's head; the head segment (this unit's last) adds the
+    // later units' partials, in unit order, and writes the tile.
     const int q = warp & 3;                        // TMEM lanes 32q .. 32q + 31 (this warp's quarter)
-    int tc = 0;
-    for (int t = unit; t < a.T; t += units, tc++) {
+    const int lrow = 32 * q + lane;                // row within the CTA's 128
+    const bool lead_thread = threadIdx.x == kFirstEpi * 32;
+    int tc = 0, t, k0, k1;
+    SegWalk sw(a, nk, unit, units);
+    for (; sw.next(t, k0, k1); tc++) {
       const int buf = tc & 1;
       const int n0 = (t % a.Nt) * kTileN * PAIR + rank * kTileN, m0 = (t / a.Nt) * BT;
       if (*abort_flag || !mbar_wait(&accfull[buf], (tc >> 1) & 1)) { *abort_flag = 1; break; }
       tc_fence_after();
-      const int row = n0 + 32 * q + lane;
+      const bool contrib = k0 > 0;                  // store a partial
+      const bool head = k0 == 0 && k1 < nk;         // finish a split tile
+      int vfirst = 0, vlast = -1;                   // contributing units of a split tile
+      if (head) {
+        const int64_t W = (int64_t)a.T * nk, tile_end = (int64_t)(t + 1) * nk;
+        vfirst = unit + 1;
+        vlast = unit;
+        while (vlast + 1 < units && (int64_t)(vlast + 1) * W / units < tile_end) vlast++;
+        if (lead_thread) {
+          for (int v = vfirst; v <= vlast; v++) {
+            const uint32_t *f = a.flags + v * PAIR + rank;
+            if (!flag_wait(f, a.epoch)) { *abort_flag = 1; break; }
+          }
+        }
+        named_bar_sync(1, 128);
+      }
+      const int row = n0 + lrow;
       float swn = 0.f;
       if constexpr (F == Fmt::I8) swn = row < a.N ? a.sw[row] : 0.f;
-      for (int ch = 0; ch < BT / 16; ch++) {
-        uint32_t v[16];
-        tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BT + ch * 16), v);
-        tmem_ld_wait();
+      // two 16-token chunks at a time: the partial loads of both are in flight
+      // together with the TMEM loads
+      for (int ch = 0; ch < BT / 16; ch += 2) {
+        uint32_t v[32], pv[32];
+        if (!contrib) {
+#pragma unroll
+          for (int j = 0; j < 32; j++) pv[j] = 0u;
+          for (int vv = vfirst; vv <= vlast; vv++) {
+            const uint32_t *src = a.ws + ((size_t)(vv * PAIR + rank) * BT + ch * 16) * kTileN + lrow;
+            uint32_t w[32];
+#pragma unroll
+            for (int j = 0; j < 32; j++) w[j] = __ldcg(src + j * kTileN);
+#pragma unroll
+            for (int j = 0; j < 32; j++) {
+              if constexpr (F == Fmt::I8) pv[j] = (uint32_t)((int)pv[j] + (int)w[j]);
+              else pv[j] = __float_as_uint(__uint_as_float(pv[j]) + __uint_as_float(w[j]));
+            }
+          }
+        }
+        {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BT + ch * 16), v0);
+          tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BT + ch * 16 + 16), v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; j++) { v[j] = v0[j]; v[16 + j] = v1[j]; }
+        }
+        if (contrib) {
+          uint32_t *dst = a.ws + ((size_t)blockIdx.x * BT + ch * 16) * kTileN + lrow;
+#pragma unroll
+          for (int j = 0; j < 32; j++) dst[j * kTileN] = v[j];
+          continue;
+        }
+        if (vlast >= vfirst) {
+#pragma unroll
+          for (int j = 0; j < 32; j++) {
+            if constexpr (F == Fmt::I8) v[j] = (uint32_t)((int)v[j] + (int)pv[j]);
+            else v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(pv[j]));
+          }
+        }
         if (row < a.N) {
 #pragma unroll
-          for (int j = 0; j < 16; j++) {
+          for (int j = 0; j < 32; j++) {
             const int m = m0 + ch * 16 + j;
             if (m < a.M) {
               const int64_t o = (int64_t)m * a.N + row;
@@ -523,6 +638,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         if constexpr (PAIR == 2) mbar_arrive_remote(lead_accempty + buf * 8);
         else mbar_arrive(&accempty[buf]);
+      }
+      if (contrib) {   // publish the partial once all four warps stored theirs
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (lead_thread) flag_publish(a.flags + blockIdx.x, a.epoch);
       }
     }
   }
@@ -564,6 +684,52 @@ gwb_status map2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64
   return GWB_OK;
 }
 
+// Stream-K workspace, owned by the library: one per (device, stream), so that
+// GEMMs on different streams never share partial slots; allocated (and its
+// flags zeroed) on the first call that needs it, outside stream capture, and
+// kept until the process exits.  Each launch takes a fresh epoch, so the flags
+// never need clearing again.
+struct Workspace {
+  uint32_t *base = nullptr;
+  size_t partial_bytes = 0;
+  int nflags = 0;
+};
+std::mutex g_ws_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+std::atomic<uint32_t> g_epoch{0};
+
+bool stream_workspace(cudaStream_t st, size_t partial_bytes, int nflags, uint32_t **ws, uint32_t **flags) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  Workspace &w = g_ws[std::make_pair(dev, st)];
+  if (w.base == nullptr || w.partial_bytes < partial_bytes || w.nflags < nflags) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return false;
+    if (w.base) {
+      if (cudaStreamSynchronize(st) != cudaSuccess) return false;
+      cudaFree(w.base);
+      w = Workspace{};
+    }
+    const size_t fbytes = ((size_t)nflags * 4 + 255) / 256 * 256;
+    void *p = nullptr;
+    if (cudaMalloc(&p, partial_bytes + fbytes) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return false;
+    }
+    if (cudaMemsetAsync(static_cast<unsigned char *>(p) + partial_bytes, 0, fbytes, st) != cudaSuccess) {
+      cudaFree(p);
+      return false;
+    }
+    w.base = static_cast<uint32_t *>(p);
+    w.partial_bytes = partial_bytes;
+    w.nflags = nflags;
+  }
+  *ws = w.base;
+  *flags = w.base + w.partial_bytes / 4;
+  return true;
+}
+
 template <Fmt F, int BITS, int BT, int PAIR>
 gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
                    const CUtensorMap &tsb, Args a, cudaStream_t st) {
@@ -582,8 +748,26 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
   });
   if (attr_err != cudaSuccess) return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
   const int units = kSMs / PAIR;
+  const int nk = (a.K + Tr<F, BITS>::BK - 1) / Tr<F, BITS>::BK;
+  // Stream-K when whole tiles would leave part of the last wave idle and every
+  // unit gets a few K steps; else whole tiles per unit.
+  int grid_units = a.T < units ? a.T : units;
+  a.ws = nullptr;
+  a.flags = nullptr;
+  a.epoch = 0;
+  if (a.T % units != 0 && (int64_t)a.T * nk >= 4LL * units) {
+    uint32_t *ws = nullptr, *fl = nullptr;
+    if (stream_workspace(st, (size_t)kSMs * BT * kTileN * 4, kSMs, &ws, &fl)) {
+      a.ws = ws;
+      a.flags = fl;
+      uint32_t e = g_epoch.fetch_add(1) + 1;
+      if (e == 0) e = g_epoch.fetch_add(1) + 1;
+      a.epoch = e;
+      grid_units = units;
+    }
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(PAIR * (a.T < units ? a.T : units)));
+  cfg.gridDim = dim3((unsigned)(PAIR * grid_units));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = P::SMEM;
   cfg.stream = st;

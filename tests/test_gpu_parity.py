@@ -257,6 +257,17 @@ def test_w4a8_k_tail():
     W4A8(136, 96).check(24)   # K = 96 < one 128-wide K step
 
 
+@pytest.mark.parametrize("bits,M", [(4, 512), (4, 300), (8, 512)])
+def test_qmm_affine_stream_k_split_tiles(bits, M):
+    # 8 x 2 tiles of 256 x 256 and 32 K steps over 74 CTA pairs: every tile is
+    # split between four or five pairs and finished from their partials
+    Affine(2048, 2048, bits, 64, seed=11).check_qmm(M, outlier_frac=0.01, label=f"stream-K b{bits} M={M}")
+
+
+def test_w4a8_stream_k_split_tiles():
+    W4A8(2048, 2048).check(512)
+
+
 # --------------------------------------------------------------------------- full sizes
 def test_full_single_affine_linear_512():
     a = Affine(512, 512, 4, 64)
