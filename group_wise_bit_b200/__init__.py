@@ -28,6 +28,7 @@ SIGNATURES = {
     "gwb_qpack_affine": [_P, _I64, _I64, _INT, _INT, _P, _P, _P, _P],
     "gwb_dequant_affine": [_P, _P, _P, _I64, _I64, _INT, _INT, _P, _P],
     "gwb_qmm_affine": [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P],
+    "gwb_qmm_affine_noalloc": [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P],
     "gwb_gptq_dequant": [_P, _P, _P, _P, _I64, _I64, _INT, _P, _P],
     "gwb_gptq_qmm": [_P, _I64, _P, _P, _P, _P, _I64, _I64, _INT, _P, _P],
     "gwb_quant_per_token_i8": [_P, _I64, _I64, _P, _P, _P],
@@ -143,6 +144,21 @@ def qmm_affine(x, wq, scales, biases, bits, group_size, y=None):
     y = _out(y, "y", (M, N), torch.bfloat16, x.device)
     _call("gwb_qmm_affine", _ptr(x), M, _ptr(wq), _ptr(scales), _ptr(biases), N, K, bits, group_size, _ptr(y),
           _stream())
+    return y
+
+
+def qmm_affine_noalloc(x, wq, scales, biases, bits, group_size, y=None):
+    """As qmm_affine for M > 128, with the GEMM's scratch in the library's fixed
+    device array instead of device memory it allocates (see gwb.h)."""
+    _dev(x, "x", (torch.bfloat16,))
+    M, K = x.shape
+    N = wq.shape[0]
+    _dev(wq, "wq", _WORDS, (N, K * bits // 32))
+    _dev(scales, "scales", (torch.bfloat16,), (N, K // group_size))
+    _dev(biases, "biases", (torch.bfloat16,), (N, K // group_size))
+    y = _out(y, "y", (M, N), torch.bfloat16, x.device)
+    _call("gwb_qmm_affine_noalloc", _ptr(x), M, _ptr(wq), _ptr(scales), _ptr(biases), N, K, bits, group_size,
+          _ptr(y), _stream())
     return y
 
 

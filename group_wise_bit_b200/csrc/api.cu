@@ -148,6 +148,26 @@ gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, cons
   return gwb::launch_tc_affine(x, M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
 }
 
+gwb_status gwb_qmm_affine_noalloc(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
+                                  const uint16_t *biases, int64_t N, int64_t K, int bits, int group_size,
+                                  uint16_t *y, void *stream) {
+  GWB_TRY(check_layout(N, K, bits, group_size));
+  if (M < 0) return fail(GWB_ERR_INVALID_ARG, "negative M=%lld", (long long)M);
+  if (M >= kMaxDim) return fail(GWB_ERR_SHAPE, "M must be below 2^31");
+  if (M <= 128)
+    return fail(GWB_ERR_SHAPE, "qmm_affine_noalloc runs the prefill GEMM: M must exceed 128 (M=%lld)", (long long)M);
+  if (N == 0) return GWB_OK;
+  if (K == 0) return fail(GWB_ERR_SHAPE, "qmm_affine_noalloc needs K > 0");
+  GWB_TRY(need(y, "y"));
+  GWB_TRY(need(x, "x"));
+  GWB_TRY(need(wq, "wq"));
+  GWB_TRY(need(scales, "scales"));
+  GWB_TRY(need(biases, "biases"));
+  if (bits == 2 && K % 64 != 0)
+    return fail(GWB_ERR_UNSUPPORTED, "bits=2 needs K %% 64 == 0 on the tensor-core path (K=%lld)", (long long)K);
+  return gwb::launch_tc2_affine_noalloc(x, M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
+}
+
 gwb_status gwb_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
                             const int32_t *g_idx, int64_t K, int64_t N, int group_size, uint16_t *w_out,
                             void *stream) {

@@ -77,5 +77,10 @@ gwb_status launch_tc2_gptq(const uint16_t *x, int64_t M, const int32_t *qweight,
 gwb_status launch_tc2_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
                            int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 gwb_status read_and_clear_device_error_tc2(cudaStream_t st, unsigned int *flag);
+// The persistent GEMM with its stream-K scratch in a fixed device array (no
+// allocation); M must exceed 128.
+gwb_status launch_tc2_affine_noalloc(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
+                                     const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
+                                     cudaStream_t st);
 
 }  // namespace gwb

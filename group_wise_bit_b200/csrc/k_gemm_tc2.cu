@@ -730,9 +730,12 @@ bool stream_workspace(cudaStream_t st, size_t partial_bytes, int nflags, uint32_
   return true;
 }
 
+// fixed_ws: stream-K scratch supplied by the caller of this function (partials
+// then flags, room for max_units units) instead of the stream workspace.
 template <Fmt F, int BITS, int BT, int PAIR>
 gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
-                   const CUtensorMap &tsb, Args a, cudaStream_t st) {
+                   const CUtensorMap &tsb, Args a, cudaStream_t st, uint32_t *fixed_ws = nullptr,
+                   int max_units = 0) {
   using P = Plan2<F, BITS, BT, PAIR>;
   CUtensorMap tx;
   gwb_status s = map2d(&tx, xdt, xptr, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * xelem, 128u / xelem,
@@ -747,7 +750,8 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
   });
   if (attr_err != cudaSuccess) return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err));
-  const int units = kSMs / PAIR;
+  int units = kSMs / PAIR;
+  if (max_units > 0 && max_units < units) units = max_units;
   const int nk = (a.K + Tr<F, BITS>::BK - 1) / Tr<F, BITS>::BK;
   // Stream-K when whole tiles would leave part of the last wave idle and every
   // unit gets a few K steps; else whole tiles per unit.
@@ -757,7 +761,15 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
   a.epoch = 0;
   if (a.T % units != 0 && (int64_t)a.T * nk >= 4LL * units) {
     uint32_t *ws = nullptr, *fl = nullptr;
-    if (stream_workspace(st, (size_t)kSMs * BT * kTileN * 4, kSMs, &ws, &fl)) {
+    bool have_ws = false;
+    if (fixed_ws) {
+      ws = fixed_ws;
+      fl = fixed_ws + (size_t)units * PAIR * BT * kTileN;
+      have_ws = cudaMemsetAsync(fl, 0, (size_t)units * PAIR * 4, st) == cudaSuccess;
+    } else {
+      have_ws = stream_workspace(st, (size_t)kSMs * BT * kTileN * 4, kSMs, &ws, &fl);
+    }
+    if (have_ws) {
       a.ws = ws;
       a.flags = fl;
       uint32_t e = g_epoch.fetch_add(1) + 1;
@@ -787,9 +799,46 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
 // half the activation bytes per SM); else 128 x 128 tiles on single CTAs.
 template <Fmt F, int BITS>
 gwb_status dispatch2(int64_t M, const void *x, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
-                     const CUtensorMap &tsb, const Args &a, cudaStream_t st) {
-  if (M <= 128) return run_tc2<F, BITS, 128, 1>(x, xdt, xelem, tw, tsb, a, st);
-  return run_tc2<F, BITS, 256, 2>(x, xdt, xelem, tw, tsb, a, st);
+                     const CUtensorMap &tsb, const Args &a, cudaStream_t st, uint32_t *fixed_ws = nullptr,
+                     int max_units = 0) {
+  if (M <= 128) return run_tc2<F, BITS, 128, 1>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
+  return run_tc2<F, BITS, 256, 2>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
+}
+
+// ---------------------------------------------------------------- scratch without allocation
+// Some callers cannot allocate device memory: code running under an allocator
+// that owns all of the GPU's memory (a framework's caching pool, a serving
+// runtime that reserves memory up front), or code that must not call
+// cudaMalloc / cudaFree at all, since both may synchronize the device.  For
+// them the prefill GEMM can run with its stream-K scratch in this fixed array:
+// the partial tiles of at most kScratchPairs CTA pairs (8 MiB) and their flags.
+// It lives in every GPU that loads the library until the process exits.
+constexpr int kScratchPairs = 32;
+constexpr size_t kScratchPartialWords = (size_t)kScratchPairs * 2 * 256 * kTileN;
+constexpr size_t kScratchFlagWords = 64;
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kScratchPartialWords + kScratchFlagWords];
+
+// Device address of the array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+std::mutex g_scratch_mu;
+std::map<int, uint32_t *> g_scratch_addr;
+
+gwb_status noalloc_scratch(uint32_t **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  auto it = g_scratch_addr.find(dev);
+  if (it == g_scratch_addr.end()) {
+    uint32_t *p = nullptr;
+    e = cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(GWB_ERR_CUDA, "cudaGetSymbolAddress of the GEMM scratch: %s", cudaGetErrorString(e));
+    it = g_scratch_addr.emplace(dev, p).first;
+  }
+  *out = it->second;
+  return GWB_OK;
 }
 
 }  // namespace
@@ -830,6 +879,40 @@ gwb_status launch_tc2_affine(const uint16_t *x, int64_t M, const uint32_t *wq, c
   if (bits == 4) return dispatch2<Fmt::Affine, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, tsb, a, st);
   if (bits == 8) return dispatch2<Fmt::Affine, 8>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, tsb, a, st);
   return dispatch2<Fmt::Affine, 2>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, tsb, a, st);
+}
+
+gwb_status launch_tc2_affine_noalloc(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
+                                     const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
+                                     cudaStream_t st) {
+  if (M <= 128)
+    return fail(GWB_ERR_SHAPE, "qmm_affine_noalloc runs the prefill GEMM: M must exceed 128 (M=%lld)", (long long)M);
+  if ((K / gs) % 2 != 0 || (((uintptr_t)scales | (uintptr_t)biases) & 3) != 0)
+    return fail(GWB_ERR_UNSUPPORTED, "qmm_affine_noalloc needs an even number of groups per row (K/gs=%lld)",
+                (long long)(K / gs));
+  // the scratch holds one 256-token x 128-row fp32 partial per CTA of at most
+  // kScratchPairs pairs, plus their flags
+  const size_t need = (size_t)kScratchPairs * 2 * 256 * kTileN + (size_t)kScratchPairs * 2;
+  if (need > kScratchPartialWords + kScratchFlagWords)
+    return fail(GWB_ERR_SHAPE, "qmm_affine_noalloc: %zu scratch words needed, %zu available", need,
+                kScratchPartialWords + kScratchFlagWords);
+  uint32_t *scratch = nullptr;
+  gwb_status s = noalloc_scratch(&scratch);
+  if (s != GWB_OK) return s;
+  Args a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
+  a.gs_log2 = gs == 32 ? 5 : (gs == 64 ? 6 : 7);
+  a.scales = scales; a.biases = biases; a.y = y;
+  a.sc_tma = 0;
+  CUtensorMap tw;
+  const uint64_t words = (uint64_t)K * bits / 32;
+  s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, (uint64_t)N, words * 4, (uint32_t)(64 * bits / 32),
+            (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (s != GWB_OK) return s;
+  if (bits == 4)
+    return dispatch2<Fmt::Affine, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, tw, a, st, scratch, kScratchPairs);
+  if (bits == 8)
+    return dispatch2<Fmt::Affine, 8>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, tw, a, st, scratch, kScratchPairs);
+  return dispatch2<Fmt::Affine, 2>(M, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tw, tw, a, st, scratch, kScratchPairs);
 }
 
 gwb_status launch_tc2_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,

@@ -7,6 +7,13 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
  *    never allocates, frees or retains them.  Tensors are dense and row-major
  *    with the shapes stated per call; no strides are taken.
+ *  - The one device buffer the library owns is the prefill GEMM's stream-K
+ *    workspace (partial tiles, about 19 MB): one per (device, stream),
+ *    allocated by the first qmm_affine / gptq_qmm / gemm_i8i4 call with more
+ *    than 128 tokens on that stream, and kept until the process exits.  A call
+ *    made while its stream is being captured into a CUDA graph never
+ *    allocates; it runs without the workspace (whole tiles per CTA pair).
+ *    gwb_qmm_affine_noalloc is the entry point that allocates nothing.
  *  - bf16 and fp16 values are passed as their raw 16-bit patterns (uint16_t).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
  *    validates its arguments synchronously, on the host, before launching
@@ -112,6 +119,34 @@ gwb_status gwb_dequant_affine(const uint32_t *wq, const uint16_t *scales, const 
 gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
                           const uint16_t *biases, int64_t N, int64_t K, int bits, int group_size,
                           uint16_t *y, void *stream);
+
+/* qmm_affine_noalloc -- gwb_qmm_affine's prefill GEMM for callers that cannot
+ * allocate device memory.  Such callers exist: code running under an allocator
+ * that owns all of the GPU's memory (a framework's caching pool, a serving
+ * runtime that reserves memory up front), and code that must not call cudaMalloc
+ * or cudaFree at all (both may synchronize the whole device).  The pages
+ * describe no counterpart of this entry point; it is a property of this library.
+ * Same arguments, layouts and result as gwb_qmm_affine, for M > 128 only
+ * (GWB_ERR_SHAPE otherwise: smaller M needs no scratch, call gwb_qmm_affine).
+ * The GEMM's stream-K scratch (partial tiles and their flags) is a file-scope
+ * device array of the library, 8 MiB + 256 bytes, which holds the partials of
+ * at most 32 CTA pairs, so the GEMM runs on at most 32 pairs (64 of the 148
+ * SMs) and every problem size fits; a size whose scratch would not fit is
+ * rejected with GWB_ERR_SHAPE and a message.  Every GPU that loads the library
+ * holds the array until the process exits.
+ *  - The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *    routine.  The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls share the one array, which keeps the last call's contents; each
+ *    call clears the flags it needs before its kernel runs.  Calls that overlap
+ *    on the GPU (concurrent streams, or several devices' threads racing on one
+ *    device) race on the array and give wrong results: serialize them.
+ * Also GWB_ERR_UNSUPPORTED when K/group_size is odd or scales/biases are not
+ * 4-byte aligned. */
+gwb_status gwb_qmm_affine_noalloc(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
+                                  const uint16_t *biases, int64_t N, int64_t K, int bits, int group_size,
+                                  uint16_t *y, void *stream);
 
 /* ------------------------------------------------------------------ GPTQ */
 
