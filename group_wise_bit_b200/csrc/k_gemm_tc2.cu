@@ -121,6 +121,23 @@ __device__ __forceinline__ bool flag_wait(const uint32_t *f, uint32_t epoch) {
     __nanosleep(64);
   }
 }
+// Same, with A read from tensor memory (each CTA's TMEM holds its 128 rows).
+__device__ __forceinline__ void umma_f16_ts_pair(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                                 uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_i8_ts_pair(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                                uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
 // Arrive once on the barrier at this offset in both CTAs of the pair when the
 // pair's MMAs issued so far complete.
 __device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
@@ -148,6 +165,7 @@ constexpr int kFirstDq = 3, kFirstEpi = 11;
 constexpr int kTileN = 128;      // output features per tile (tensor-core M)
 constexpr int kMaxSmem = 232448;
 constexpr int kSMs = 148;
+constexpr bool kAInTmem = true;   // pairs keep the dequantized A operand in tensor memory
 
 enum class Fmt { Affine, Gptq, I8 };
 
@@ -227,26 +245,37 @@ struct Tr<Fmt::I8, 4> {
 // 6 dequantized slots (the dequantizers then run well ahead of the tensor core)
 // next to 4 activation slots; a single CTA keeps 3 A slots and fits as many
 // activation slots as it can.  The packed-weight ring takes what is left, up to 8.
-template <Fmt F, int BITS, int BT, int PAIR>
+// With ATM the dequantized A stages live in tensor memory (8 slots of 32
+// columns next to one 256-column accumulator) and take no shared memory.
+template <Fmt F, int BITS, int BT, int PAIR, bool ATM>
 struct Plan2 {
   static constexpr int XB = BT / PAIR * 128;
   static constexpr int AB = kTileN * 128;
   static constexpr int RB = (Tr<F, BITS>::RAW + Tr<F, BITS>::SC + 127) / 128 * 128;
-  static constexpr int SA = PAIR == 2 ? 6 : 3;
+  static constexpr int SA = ATM ? 8 : (PAIR == 2 ? 6 : 3);
+  static constexpr int A_SMEM = ATM ? 0 : SA * AB;
+  // ATM: a bf16 staging tile [BT tokens][128 rows] for the epilogue, so that it
+  // frees the single accumulator before writing the output
+  static constexpr int EPI = ATM ? BT * kTileN * 2 : 0;
   static constexpr int BUDGET = kMaxSmem - 1024 - 1024 - 1024;   // alignment, barriers, static
-  static constexpr int SXF = (BUDGET - SA * AB - 4 * RB) / XB > 6 ? 6 : (BUDGET - SA * AB - 4 * RB) / XB;
-  static constexpr int SX = PAIR == 2 && SXF > 4 ? 4 : SXF;
-  static constexpr int SR0 = (BUDGET - SA * AB - SX * XB) / RB;
+  static constexpr int SXF = (BUDGET - A_SMEM - EPI - 4 * RB) / XB > 6 ? 6 : (BUDGET - A_SMEM - EPI - 4 * RB) / XB;
+  static constexpr int SX = PAIR == 2 && !ATM && SXF > 4 ? 4 : SXF;
+  static constexpr int SR0 = (BUDGET - A_SMEM - EPI - SX * XB) / RB;
   static constexpr int SR = SR0 > 8 ? 8 : SR0;
-  static constexpr int SMEM = SX * XB + SA * AB + SR * RB + 1024 + 1024;
+  static constexpr int SMEM = SX * XB + A_SMEM + EPI + SR * RB + 1024 + 1024;
   static_assert(SX >= 2 && SR >= 4, "shared memory too small");
 };
 
-// Dequantizes K step `k` of the tile at feature n0 (rows r, half h of the step)
-// from the R stage into the A stage.
+__device__ __forceinline__ void put4(uint32_t (&o)[16], int j, uint4 v) {
+  o[4 * j] = v.x; o[4 * j + 1] = v.y; o[4 * j + 2] = v.z; o[4 * j + 3] = v.w;
+}
+
+// Dequantizes K step `k` (row r, half h of the step) from the R stage into the
+// 16 words of A the thread owns: o[4j .. 4j+3] = 16-byte chunk 4h + j of row r
+// (k = 8 (4h + j) .. +7 for 16-bit operands, 16 (4h + j) .. +15 for int8).
 template <Fmt F, int BITS>
-__device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h, const unsigned char *R,
-                                             unsigned char *A) {
+__device__ __forceinline__ void dequant_words(const Args &a, int k, int r, int h, const unsigned char *R,
+                                              uint32_t (&o)[16]) {
   using T = Tr<F, BITS>;
   constexpr int BK = T::BK;
   const int kh = k * BK + h * (BK / 2);    // first k of this thread's half step
@@ -275,24 +304,24 @@ __device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h,
       const __nv_bfloat162 s2b = __floats2bfloat162_rn(sf, sf), b2b = __floats2bfloat162_rn(bfv, bfv);
       const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-      for (int j = 0; j < 4; j++) *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + j)) = dq_affine4(wv[j], s2b, b2b);
+      for (int j = 0; j < 4; j++) put4(o, j, dq_affine4(wv[j], s2b, b2b));
     } else if constexpr (BITS == 2) {
       const uint2 raw = *reinterpret_cast<const uint2 *>(R + (r * 4 + h * 2) * 4);
       const __nv_bfloat162 s2q = __floats2bfloat162_rn(sf, sf * 0.25f), b2b = __floats2bfloat162_rn(bfv, bfv);
       uint4 c0, c1;
       dq_affine2(raw.x, s2q, b2b, c0, c1);
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 0)) = c0;
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 1)) = c1;
+      put4(o, 0, c0);
+      put4(o, 1, c1);
       dq_affine2(raw.y, s2q, b2b, c0, c1);
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 2)) = c0;
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 3)) = c1;
+      put4(o, 2, c0);
+      put4(o, 3, c1);
     } else {
       const uint4 *rp = reinterpret_cast<const uint4 *>(R + (r * 16 + h * 8) * 4);
       const uint4 ra = rp[0], rb = rp[1];
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 0)) = dq_affine8(ra.x, ra.y, sf, bfv);
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 1)) = dq_affine8(ra.z, ra.w, sf, bfv);
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 2)) = dq_affine8(rb.x, rb.y, sf, bfv);
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + 3)) = dq_affine8(rb.z, rb.w, sf, bfv);
+      put4(o, 0, dq_affine8(ra.x, ra.y, sf, bfv));
+      put4(o, 1, dq_affine8(ra.z, ra.w, sf, bfv));
+      put4(o, 2, dq_affine8(rb.x, rb.y, sf, bfv));
+      put4(o, 3, dq_affine8(rb.z, rb.w, sf, bfv));
     }
   } else if constexpr (F == Fmt::Gptq) {
     int idx = (kh >> a.gs_log2) - ((k * BK) >> a.gs_log2);
@@ -308,7 +337,7 @@ __device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h,
 #pragma unroll
     for (int j = 0; j < 4; j++) {
       const int kq = 4 * h + j;                  // k-octet within the step = chunk index
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, kq)) = dq_gptq(Rw[kq * kTileN + r], z2, s2);
+      put4(o, j, dq_gptq(Rw[kq * kTileN + r], z2, s2));
     }
   } else {
     const uint4 *rp = reinterpret_cast<const uint4 *>(R + (r * 16 + h * 8) * 4);
@@ -317,21 +346,33 @@ __device__ __forceinline__ void dequant_step(const Args &a, int k, int r, int h,
 #pragma unroll
     for (int j = 0; j < 4; j++) {
       const uint2 lo = dq_i4(wv[2 * j]), hi = dq_i4(wv[2 * j + 1]);
-      *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + j)) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+      put4(o, j, make_uint4(lo.x, lo.y, hi.x, hi.y));
     }
   }
 }
 
-template <Fmt F, int BITS, int BT, int PAIR>
+// The thread's 16 words of A into the 128-byte-swizzled shared-memory A stage.
+__device__ __forceinline__ void store_a_smem(unsigned char *A, int r, int h, const uint32_t (&o)[16]) {
+#pragma unroll
+  for (int j = 0; j < 4; j++)
+    *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + j)) = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+}
+
+template <Fmt F, int BITS, int BT, int PAIR, bool ATM>
 __global__ void __launch_bounds__(kThreads, 1)
     k_tc2(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
           const __grid_constant__ CUtensorMap tm_sb, const Args a) {
   using T = Tr<F, BITS>;
-  using P = Plan2<F, BITS, BT, PAIR>;
+  using P = Plan2<F, BITS, BT, PAIR, ATM>;
   constexpr int BK = T::BK;
   constexpr int SX = P::SX, SA = P::SA, SR = P::SR;
   constexpr int XT = BT / PAIR;                        // tokens of this CTA's activation slot
-  constexpr uint32_t NCOLS = 2 * BT;                  // two accumulators of BT fp32 / s32 columns
+  // TMEM: two accumulators of BT fp32 / s32 columns, or (ATM) one accumulator
+  // and SA A slots of 32 columns (64 bf16 or 128 int8 k per row)
+  constexpr uint32_t NCOLS = ATM ? 512u : 2u * BT;
+  constexpr int NACC = ATM ? 1 : 2;
+  constexpr uint32_t ACOL = BT;                        // first A slot column (ATM)
+  static_assert(!ATM || (PAIR == 2 && BT == 256), "A in tensor memory is laid out for 256-token pairs");
   constexpr uint32_t IDESC = (F == Fmt::I8) ? make_idesc(2, 1, kTileN * PAIR, BT)
                              : (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN * PAIR, BT)
                                                 : make_idesc(1, 1, kTileN * PAIR, BT);
@@ -340,8 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char *base = align_smem_1024(smem_raw);
   unsigned char *ringX = base;
   unsigned char *ringA = ringX + SX * P::XB;
-  unsigned char *ringR = ringA + SA * P::AB;
-  uint64_t *xfull = reinterpret_cast<uint64_t *>(ringR + SR * P::RB);
+  unsigned char *ringR = ringA + P::A_SMEM;
+  uint16_t *stage = reinterpret_cast<uint16_t *>(ringR + SR * P::RB);   // ATM epilogue staging
+  uint64_t *xfull = reinterpret_cast<uint64_t *>(ringR + SR * P::RB + P::EPI);
   uint64_t *xempty = xfull + SX;
   uint64_t *afull = xempty + SX;
   uint64_t *aempty = afull + SA;
@@ -474,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       SegWalk sw(a, nk, unit, units);
       for (; ok && sw.next(t, k0, k1); tc++) {
-        const int buf = tc & 1;
-        if (*abort_flag || !mbar_wait(&accempty[buf], ((tc >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
+        const int buf = tc % NACC, use = tc / NACC;
+        if (*abort_flag || !mbar_wait(&accempty[buf], (use & 1) ^ 1)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(buf * BT);
         for (int k = k0; k < k1; k++, xi++) {
@@ -490,7 +532,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < T::NMMA; kk++) {
             const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
-            if constexpr (PAIR == 2) {
+            if constexpr (ATM) {
+              const uint32_t at = tmem + ACOL + (uint32_t)(32 * sa + 8 * kk);
+              if constexpr (F == Fmt::I8) umma_i8_ts_pair(d, at, bd, IDESC, (k - k0) | kk);
+              else umma_f16_ts_pair(d, at, bd, IDESC, (k - k0) | kk);
+              (void)ad;
+            } else if constexpr (PAIR == 2) {
               if constexpr (F == Fmt::I8) umma_i8_pair(d, ad, bd, IDESC, (k - k0) | kk);
               else umma_f16_pair(d, ad, bd, IDESC, (k - k0) | kk);
             } else {
@@ -517,7 +564,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < kFirstEpi) {
     // ------------------------------------------------------------ dequantizers
     const int d = threadIdx.x - kFirstDq * 32;
-    const int r = d & (kTileN - 1), h = d >> 7;   // tile row, half of the K step
+    // tile row and half of the K step; with A in TMEM a warp owns the row
+    // quarter its warp index may address (32 * (warp % 4) ..)
+    const int r = ATM ? 32 * (warp & 3) + lane : (d & (kTileN - 1));
+    const int h = ATM ? (warp - kFirstDq) >> 2 : (d >> 7);
     int it = 0, t, k0, k1;
     bool ok = true;
     SegWalk sw(a, nk, unit, units);
@@ -529,8 +579,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        dequant_step<F, BITS>(a, k, r, h, ringR + sr * P::RB, ringA + sa * P::AB);
-        fence_proxy_async_smem();
+        {
+          uint32_t o[16];
+          dequant_words<F, BITS>(a, k, r, h, ringR + sr * P::RB, o);
+          if constexpr (ATM) {
+            tmem_st<16>(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + ACOL + (uint32_t)(32 * sa + 16 * h), o);
+            tmem_st_wait();
+            tc_fence_before();
+          } else {
+            store_a_smem(ringA + sa * P::AB, r, h, o);
+          }
+        }
+        if constexpr (!ATM) fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           if constexpr (PAIR == 2) mbar_arrive_remote(lead_afull + sa * 8);
@@ -551,9 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int tc = 0, t, k0, k1;
     SegWalk sw(a, nk, unit, units);
     for (; sw.next(t, k0, k1); tc++) {
-      const int buf = tc & 1;
+      const int buf = tc % NACC, use = tc / NACC;
       const int n0 = (t % a.Nt) * kTileN * PAIR + rank * kTileN, m0 = (t / a.Nt) * BT;
-      if (*abort_flag || !mbar_wait(&accfull[buf], (tc >> 1) & 1)) { *abort_flag = 1; break; }
+      if (*abort_flag || !mbar_wait(&accfull[buf], use & 1)) { *abort_flag = 1; break; }
       tc_fence_after();
       const bool contrib = k0 > 0;                  // store a partial
       const bool head = k0 == 0 && k1 < nk;         // finish a split tile
@@ -574,6 +634,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = n0 + lrow;
       float swn = 0.f;
       if constexpr (F == Fmt::I8) swn = row < a.N ? a.sw[row] : 0.f;
+      if constexpr (ATM && F != Fmt::I8) {
+        if (!contrib && !head) {
+          // whole tile: TMEM -> bf16 / fp16 staging, free the accumulator, then
+          // write the tile row by row of tokens with 16-byte stores
+          for (int ch = 0; ch < BT / 16; ch += 2) {
+            uint32_t v0[16], v1[16];
+            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ch * 16), v0);
+            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ch * 16 + 16), v1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; j++) {
+              const float f = __uint_as_float(j < 16 ? v0[j] : v1[j - 16]);
+              stage[(ch * 16 + j) * kTileN + lrow] = F == Fmt::Gptq ? __half_as_ushort(__float2half_rn(f))
+                                                                    : __bfloat16_as_ushort(__float2bfloat16_rn(f));
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (PAIR == 2) mbar_arrive_remote(lead_accempty + buf * 8);
+            else mbar_arrive(&accempty[buf]);
+          }
+          named_bar_sync(1, 128);
+          const bool vec = (a.N % 8) == 0;
+          const int tid = threadIdx.x - kFirstEpi * 32;
+          for (int e = tid; e < BT * (kTileN / 8); e += 128) {
+            const int tok = e / (kTileN / 8), c8 = (e % (kTileN / 8)) * 8;
+            const int m = m0 + tok, n = n0 + c8;
+            if (m >= a.M || n >= a.N) continue;
+            const uint16_t *src = stage + tok * kTileN + c8;
+            if (vec && n + 8 <= a.N) {
+              *reinterpret_cast<uint4 *>(a.y + (int64_t)m * a.N + n) = *reinterpret_cast<const uint4 *>(src);
+            } else {
+              for (int i = 0; i < 8 && n + i < a.N; i++) a.y[(int64_t)m * a.N + n + i] = src[i];
+            }
+          }
+          named_bar_sync(1, 128);   // the staging tile is free for the next segment
+          continue;
+        }
+      }
       // two 16-token chunks at a time: the partial loads of both are in flight
       // together with the TMEM loads
       for (int ch = 0; ch < BT / 16; ch += 2) {
@@ -732,18 +832,18 @@ bool stream_workspace(cudaStream_t st, size_t partial_bytes, int nflags, uint32_
 
 // fixed_ws: stream-K scratch supplied by the caller of this function (partials
 // then flags, room for max_units units) instead of the stream workspace.
-template <Fmt F, int BITS, int BT, int PAIR>
+template <Fmt F, int BITS, int BT, int PAIR, bool ATM>
 gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
                    const CUtensorMap &tsb, Args a, cudaStream_t st, uint32_t *fixed_ws = nullptr,
                    int max_units = 0) {
-  using P = Plan2<F, BITS, BT, PAIR>;
+  using P = Plan2<F, BITS, BT, PAIR, ATM>;
   CUtensorMap tx;
   gwb_status s = map2d(&tx, xdt, xptr, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * xelem, 128u / xelem,
                        (uint32_t)(BT / PAIR), CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != GWB_OK) return s;
   a.Nt = (a.N + kTileN * PAIR - 1) / (kTileN * PAIR);
   a.T = a.Nt * ((a.M + BT - 1) / BT);
-  auto kern = k_tc2<F, BITS, BT, PAIR>;
+  auto kern = k_tc2<F, BITS, BT, PAIR, ATM>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -801,8 +901,8 @@ template <Fmt F, int BITS>
 gwb_status dispatch2(int64_t M, const void *x, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
                      const CUtensorMap &tsb, const Args &a, cudaStream_t st, uint32_t *fixed_ws = nullptr,
                      int max_units = 0) {
-  if (M <= 128) return run_tc2<F, BITS, 128, 1>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
-  return run_tc2<F, BITS, 256, 2>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
+  if (M <= 128) return run_tc2<F, BITS, 128, 1, false>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
+  return run_tc2<F, BITS, 256, 2, kAInTmem>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
 }
 
 // ---------------------------------------------------------------- scratch without allocation
