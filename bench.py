@@ -263,6 +263,7 @@ def run_gpu(args, world, rank, local):
     e2e_value = world * STEP_BYTES * args.steps / (e_ms * 1e-3) / 1e9
 
     prefill = run_prefill(gwb, dev, stream, bf16_peak, peak_kind) if not args.no_prefill else None
+    w4a8 = run_w4a8(gwb, dev, stream) if not args.no_prefill else None
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -284,10 +285,64 @@ def run_gpu(args, world, rank, local):
     }
     if prefill:
         out["prefill_m2048"] = prefill
+    if w4a8:
+        out["w4a8_m4096"] = w4a8
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def int8_peak_tops(dev, stream, reps=5):
+    """Dense int8 tensor throughput of this GPU, measured here: torch._int_mm on
+    8192^3 (2 * 8192^3 ops per call), best of `reps` launches."""
+    a = torch.randint(-64, 64, (8192, 8192), dtype=torch.int8, device=dev)
+    b = torch.randint(-64, 64, (8192, 8192), dtype=torch.int8, device=dev)
+    best = float("inf")
+    with torch.cuda.stream(stream):
+        torch._int_mm(a, b)
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            torch._int_mm(a, b)
+            e1.record(stream)
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+    return 2.0 * 8192 ** 3 / (best * 1e-3) / 1e12
+
+
+def run_w4a8(gwb, dev, stream, reps=5):
+    """W4A8 GEMM (int8 x int4 -> int32, bf16 out) at N x K = 14336 x 4096, M = 4096,
+    each launch timed alone with an L2 flush before it; ops = 2 M N K."""
+    N, K, M = 14336, 4096, 4096
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(91)
+    w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+    wq, sw = gwb.qpack_sym_i4(w)
+    del w
+    x = synth.activations(M, K, seed=1).to(dev)
+    qx, sx = gwb.quant_per_token_i8(x)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ts = []
+    with torch.cuda.stream(stream):
+        for r in range(reps + 2):
+            flush.fill_(r)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            gwb.gemm_i8i4(qx, sx, wq, sw, y=y)
+            b.record(stream)
+            b.synchronize()
+            if r >= 2:
+                ts.append(a.elapsed_time(b))
+    ms = statistics.median(ts)
+    tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+    peak = int8_peak_tops(dev, stream)
+    return {"value": round(tops, 1), "unit": "TOP/s", "N": N, "K": K, "M": M, "us": round(ms * 1e3, 1),
+            "roofline": {"kernel": "k_tc2<I8,4,256,pair,A in TMEM> (kind::i8)", "bound": "tensor",
+                         "achieved": round(tops, 1), "peak": round(peak, 1), "unit": "TOP/s",
+                         "frac": round(tops / peak, 4),
+                         "peak_source": "measured in this run: torch._int_mm 8192^3 int8, best of 5"}}
 
 
 def run_prefill(gwb, dev, stream, bf16_peak, peak_kind, reps=5):
@@ -321,9 +376,10 @@ def run_prefill(gwb, dev, stream, bf16_peak, peak_kind, reps=5):
     tf = total_flop / (total_ms * 1e-3) / 1e12
     return {"value": round(tf, 1), "unit": "TFLOP/s", "M": M_PREFILL, "bits": 4, "group_size": GS,
             "l2": "256 MB buffer written before every timed launch",
-            "roofline": {"kernel": "k_tc<Affine,4,256>", "bound": "tensor", "achieved": round(tf, 1),
+            "roofline": {"kernel": "k_tc2<Affine,4,256,pair,A in TMEM> (persistent, stream-K)", "bound": "tensor",
+                         "achieved": round(tf, 1),
                          "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(tf / bf16_peak, 4),
-                         "peak_source": peak_kind, "traffic": traffic_for("k_tc_affine4_m2048")},
+                         "peak_source": peak_kind, "traffic": traffic_for("k_tc2_affine4_m2048")},
             "shapes": per}
 
 
