@@ -286,30 +286,74 @@ __global__ void __launch_bounds__(kThreads, 2)
   };
   // issue-side position (strip, stage) of this warp, advanced without divisions
   int is_strip = sb + ub(warp) / NCS, is_st = ub(warp) % NCS;
+  // ---- activations of the K-slice, staged per item = (group, token, quad lane c):
+  // the item's NCH runs of CPW values at k = group start + (wi * 4 + c) * CPW.
+  // A thread loads its first item into registers before the ring fill below
+  // (so the load latency hides behind the TMA issue) and keeps it for pass B.
+  const int items = GR * MP * 4;
+  auto item_src = [&](int idx, int &t, int &c, int &g) -> const uint16_t * {
+    c = idx & 3;
+    t = (idx >> 2) % MP;
+    g = (idx >> 2) / MP;
+    const int kg = k0 + g * GS;
+    return (idx < items && t < a.M && kg < a.K) ? a.x + (int64_t)t * a.K + kg : nullptr;
+  };
+  auto load_item = [&](const uint16_t *src, int c, uint32_t (&raw)[C::NCH][C::CPW / 2]) {
+#pragma unroll
+    for (int wi = 0; wi < C::NCH; wi++) {
+#pragma unroll
+      for (int q = 0; q < C::CPW / 2; q++) raw[wi][q] = 0u;
+      if (src) {
+        const uint16_t *p = src + k_in_group<BITS>(wi, c, 0);
+        if constexpr (C::CPW == 4) {
+          const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p));
+          raw[wi][0] = v.x; raw[wi][1] = v.y;
+        } else {
+#pragma unroll
+          for (int q = 0; q < C::CPW / 8; q++) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p) + q);
+            raw[wi][4 * q] = v.x; raw[wi][4 * q + 1] = v.y; raw[wi][4 * q + 2] = v.z; raw[wi][4 * q + 3] = v.w;
+          }
+        }
+      }
+    }
+  };
+  uint32_t raw0[C::NCH][C::CPW / 2];
+  int t0i, c0i, g0i;
+  const uint16_t *src0 = item_src(threadIdx.x, t0i, c0i, g0i);
+  load_item(src0, c0i, raw0);
+
   for (int i = 0; i < (units < D ? units : D); i++) {
     if (lane == 0) issue(is_strip, is_st, warp * D + i);
     if (++is_st == NCS) { is_st = 0; ++is_strip; }
   }
 
-  // ---- activations of the K-slice.  Pass A: |x| max per token (per warp).
+  // Pass A: |x| max per token (per warp), over every item
   {
     float m[MP];
 #pragma unroll
     for (int t = 0; t < MP; t++) m[t] = 0.0f;
-    const int vpt = KR / 8;
-    for (int idx = threadIdx.x; idx < a.M * vpt; idx += kThreads) {
-      const int t = idx / vpt, k = k0 + 8 * (idx % vpt);
-      if (k < a.K) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.x + (int64_t)t * a.K + k));
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-        float mx = 0.0f;
+    for (int b0 = 0; b0 < items; b0 += kThreads) {
+      int t, c, g;
+      uint32_t rawb[C::NCH][C::CPW / 2];
+      const uint16_t *src = item_src(b0 + threadIdx.x, t, c, g);
+      if (b0 == 0) {
 #pragma unroll
-        for (int q = 0; q < 4; q++)
-          mx = fmaxf(mx, fmaxf(fabsf(bf16_val(w4[q] & 0xffffu)), fabsf(bf16_val(w4[q] >> 16))));
+        for (int wi = 0; wi < C::NCH; wi++)
 #pragma unroll
-        for (int tt = 0; tt < MP; tt++)
-          if (tt == t) m[tt] = fmaxf(m[tt], mx);
+          for (int q = 0; q < C::CPW / 2; q++) rawb[wi][q] = raw0[wi][q];
+      } else {
+        load_item(src, c, rawb);
       }
+      float mx = 0.0f;
+#pragma unroll
+      for (int wi = 0; wi < C::NCH; wi++)
+#pragma unroll
+        for (int q = 0; q < C::CPW / 2; q++)
+          mx = fmaxf(mx, fmaxf(fabsf(bf16_val(rawb[wi][q] & 0xffffu)), fabsf(bf16_val(rawb[wi][q] >> 16))));
+#pragma unroll
+      for (int tt = 0; tt < MP; tt++)
+        if (tt == t) m[tt] = fmaxf(m[tt], mx);
     }
 #pragma unroll
     for (int t = 0; t < MP; t++) {
@@ -330,44 +374,36 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int e = 140 - be;                                       // 14 - (be - 126)
     return e > 120 ? 120 : (e < -120 ? -120 : e);
   };
-  // Pass B: one thread per (group, token, quad lane c): the B fragments of the
-  // lane's codes, and (combined over c in order) the group's activation sum X
-  // and magic sum XN, written straight into the accumulator start quads (XNF)
-  // and the split-bf16 B operand of the bias MMAs (XF).
+  // Pass B: one thread per item: the B fragments of the lane's codes, and
+  // (combined over c in order) the group's activation sum X and magic sum XN,
+  // written straight into the accumulator start quads (XNF) and the
+  // split-bf16 B operand of the bias MMAs (XF).
   {
-    const int total = GR * MP * 4;
+    const int total = items;
     for (int b0 = 0; b0 < total; b0 += kThreads) {
       const int idx = b0 + threadIdx.x;
       const bool valid = idx < total;
-      const int c = idx & 3, t = (idx >> 2) % MP, g = (idx >> 2) / MP;
-      const int kg = k0 + g * GS;                    // first k of the group
-      const bool live = valid && t < a.M && kg < a.K;
+      int t, c, g;
+      const uint16_t *src = item_src(idx, t, c, g);
+      const bool live = src != nullptr;
       const float sc = pow2f(live ? token_exp(t) : 0);
+      uint32_t rawb[C::NCH][C::CPW / 2];
+      if (b0 == 0) {
+#pragma unroll
+        for (int wi = 0; wi < C::NCH; wi++)
+#pragma unroll
+          for (int q = 0; q < C::CPW / 2; q++) rawb[wi][q] = raw0[wi][q];
+      } else {
+        load_item(src, c, rawb);
+      }
       float sx = 0.0f, sn = 0.0f;
       uint32_t pr[C::NREG];
 #pragma unroll
       for (int wi = 0; wi < C::NCH; wi++) {
         uint16_t h[C::CPW];
-        const int kw = kg + k_in_group<BITS>(wi, c, 0);
-        uint32_t raw[C::CPW / 2];
-#pragma unroll
-        for (int q = 0; q < C::CPW / 2; q++) raw[q] = 0u;
-        if (live) {
-          const uint16_t *src = a.x + (int64_t)t * a.K + kw;
-          if constexpr (C::CPW == 4) {
-            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src));
-            raw[0] = v.x; raw[1] = v.y;
-          } else {
-#pragma unroll
-            for (int q = 0; q < C::CPW / 8; q++) {
-              const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src) + q);
-              raw[4 * q] = v.x; raw[4 * q + 1] = v.y; raw[4 * q + 2] = v.z; raw[4 * q + 3] = v.w;
-            }
-          }
-        }
 #pragma unroll
         for (int p = 0; p < C::CPW; p++) {
-          const uint32_t bits = (p & 1) ? (raw[p >> 1] >> 16) : (raw[p >> 1] & 0xffffu);
+          const uint32_t bits = (p & 1) ? (rawb[wi][p >> 1] >> 16) : (rawb[wi][p >> 1] & 0xffffu);
           h[p] = __half_as_ushort(__float2half_rn(bf16_val(bits) * sc));
           sx += __half2float(__ushort_as_half(h[p]));
         }
