@@ -31,6 +31,8 @@ SIGNATURES = {
     "gwb_qmm_affine_noalloc": [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P],
     "gwb_gptq_dequant": [_P, _P, _P, _P, _I64, _I64, _INT, _P, _P],
     "gwb_gptq_qmm": [_P, _I64, _P, _P, _P, _P, _I64, _I64, _INT, _P, _P],
+    "gwb_awq_dequant": [_P, _P, _P, _I64, _I64, _INT, _P, _P],
+    "gwb_awq_qmm": [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _P, _P],
     "gwb_quant_per_token_i8": [_P, _I64, _I64, _P, _P, _P],
     "gwb_qpack_sym_i4": [_P, _I64, _I64, _P, _P, _P],
     "gwb_gemm_i8i4": [_P, _P, _I64, _P, _P, _I64, _I64, _P, _P, _P],
@@ -192,6 +194,26 @@ def gptq_qmm(x, qweight, scales, qzeros, g_idx, group_size, y=None):
     y = _out(y, "y", (M, N), torch.float16, x.device)
     _call("gwb_gptq_qmm", _ptr(x), M, _ptr(qweight), _ptr(scales), _ptr(qzeros), _ptr(g_idx), K, N, group_size,
           _ptr(y), _stream())
+    return y
+
+
+# ------------------------------------------------------------------ AWQ
+def awq_dequant(qweight, scales, qzeros, group_size, out=None):
+    """-> fp16 [N, K]: the GPTQ layout with the stored zero used as is (no "+1", no g_idx)."""
+    K, N = _gptq_check(qweight, scales, qzeros, None, group_size)
+    out = _out(out, "out", (N, K), torch.float16, qweight.device)
+    _call("gwb_awq_dequant", _ptr(qweight), _ptr(scales), _ptr(qzeros), K, N, group_size, _ptr(out), _stream())
+    return out
+
+
+def awq_qmm(x, qweight, scales, qzeros, group_size, y=None):
+    """y fp16 [M, N] = x fp16 [M, K] . W^T with W as awq_dequant defines it."""
+    K, N = _gptq_check(qweight, scales, qzeros, None, group_size)
+    _dev(x, "x", (torch.float16,), (x.shape[0], K))
+    M = x.shape[0]
+    y = _out(y, "y", (M, N), torch.float16, x.device)
+    _call("gwb_awq_qmm", _ptr(x), M, _ptr(qweight), _ptr(scales), _ptr(qzeros), K, N, group_size, _ptr(y),
+          _stream())
     return y
 
 

@@ -168,9 +168,13 @@ gwb_status gwb_qmm_affine_noalloc(const uint16_t *x, int64_t M, const uint32_t *
   return gwb::launch_tc2_affine_noalloc(x, M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
 }
 
-gwb_status gwb_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
-                            const int32_t *g_idx, int64_t K, int64_t N, int group_size, uint16_t *w_out,
-                            void *stream) {
+namespace {
+
+// The GPTQ layout's dequant and qmm; zadd is added to each stored zero nibble
+// (1: GPTQ's "+1" convention, 0: AWQ's stored zero as is).
+gwb_status gptq_dequant_impl(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
+                             const int32_t *g_idx, int64_t K, int64_t N, int group_size, uint16_t *w_out,
+                             void *stream, int zadd) {
   GWB_TRY(check_gptq(K, N, group_size));
   if (N == 0 || K == 0) return GWB_OK;
   GWB_TRY(need(qweight, "qweight"));
@@ -178,13 +182,13 @@ gwb_status gwb_gptq_dequant(const int32_t *qweight, const uint16_t *scales, cons
   GWB_TRY(need(qzeros, "qzeros"));
   GWB_TRY(need(w_out, "w_out"));
   if (g_idx && !aligned16(g_idx)) return fail(GWB_ERR_ALIGN, "g_idx is not 16-byte aligned");
-  gwb::launch_gptq_dequant(qweight, scales, qzeros, g_idx, K, N, group_size, w_out, as_stream(stream));
-  return gwb::check_launch("gptq_dequant");
+  gwb::launch_gptq_dequant(qweight, scales, qzeros, g_idx, K, N, group_size, w_out, as_stream(stream), zadd);
+  return gwb::check_launch(zadd ? "gptq_dequant" : "awq_dequant");
 }
 
-gwb_status gwb_gptq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
-                        const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int group_size,
-                        uint16_t *y, void *stream) {
+gwb_status gptq_qmm_impl(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
+                         const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int group_size,
+                         uint16_t *y, void *stream, int zadd) {
   GWB_TRY(check_gptq(K, N, group_size));
   if (M < 0) return fail(GWB_ERR_INVALID_ARG, "negative M=%lld", (long long)M);
   if (M >= kMaxDim) return fail(GWB_ERR_SHAPE, "M must be below 2^31");
@@ -197,13 +201,38 @@ gwb_status gwb_gptq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, co
   GWB_TRY(need(qzeros, "qzeros"));
   if (g_idx && !aligned16(g_idx)) return fail(GWB_ERR_ALIGN, "g_idx is not 16-byte aligned");
   if (M <= 8)
-    return gwb::launch_gemv_gptq(x, (int)M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream));
+    return gwb::launch_gemv_gptq(x, (int)M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream),
+                                 zadd);
   if (M >= 128) {
     const gwb_status s =
-        gwb::launch_tc2_gptq(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream));
+        gwb::launch_tc2_gptq(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream), zadd);
     if (s != GWB_ERR_UNSUPPORTED) return s;
   }
-  return gwb::launch_tc_gptq(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream));
+  return gwb::launch_tc_gptq(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream), zadd);
+}
+
+}  // namespace
+
+gwb_status gwb_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
+                            const int32_t *g_idx, int64_t K, int64_t N, int group_size, uint16_t *w_out,
+                            void *stream) {
+  return gptq_dequant_impl(qweight, scales, qzeros, g_idx, K, N, group_size, w_out, stream, 1);
+}
+
+gwb_status gwb_gptq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
+                        const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int group_size,
+                        uint16_t *y, void *stream) {
+  return gptq_qmm_impl(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, stream, 1);
+}
+
+gwb_status gwb_awq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros, int64_t K,
+                           int64_t N, int group_size, uint16_t *w_out, void *stream) {
+  return gptq_dequant_impl(qweight, scales, qzeros, nullptr, K, N, group_size, w_out, stream, 0);
+}
+
+gwb_status gwb_awq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
+                       const int32_t *qzeros, int64_t K, int64_t N, int group_size, uint16_t *y, void *stream) {
+  return gptq_qmm_impl(x, M, qweight, scales, qzeros, nullptr, K, N, group_size, y, stream, 0);
 }
 
 gwb_status gwb_quant_per_token_i8(const uint16_t *x, int64_t M, int64_t K, int8_t *qx, float *sx, void *stream) {

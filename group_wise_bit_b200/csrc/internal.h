@@ -20,8 +20,10 @@ void launch_qpack_affine(const float *w, int64_t N, int64_t K, int bits, int gs,
                          uint16_t *scales, uint16_t *biases, cudaStream_t st);
 void launch_dequant_affine(const uint32_t *wq, const uint16_t *scales, const uint16_t *biases, int64_t N,
                            int64_t K, int bits, int gs, uint16_t *w_out, cudaStream_t st);
+// zadd: added to each stored zero nibble (1: GPTQ's "+1" convention, 0: AWQ's).
 void launch_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
-                         const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *w_out, cudaStream_t st);
+                         const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *w_out, cudaStream_t st,
+                         int zadd = 1);
 void launch_quant_per_token_i8(const uint16_t *x, int64_t M, int64_t K, int8_t *qx, float *sx,
                                cudaStream_t st);
 void launch_qpack_sym_i4(const float *w, int64_t N, int64_t K, uint32_t *wq, float *sw, cudaStream_t st);
@@ -54,7 +56,7 @@ gwb_status launch_gemv_tmem(const uint16_t *x, int M, const uint32_t *wq, const 
 gwb_status read_and_clear_device_error_tmem(cudaStream_t st, unsigned int *flag);
 gwb_status launch_gemv_gptq(const uint16_t *x, int M, const int32_t *qweight, const uint16_t *scales,
                             const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
-                            uint16_t *y, cudaStream_t st);
+                            uint16_t *y, cudaStream_t st, int zadd = 1);
 
 // ------------------------------------------------------------ tensor-core GEMM regime
 gwb_status launch_tc_affine(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
@@ -62,7 +64,7 @@ gwb_status launch_tc_affine(const uint16_t *x, int64_t M, const uint32_t *wq, co
                             cudaStream_t st);
 gwb_status launch_tc_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
                           const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
-                          uint16_t *y, cudaStream_t st);
+                          uint16_t *y, cudaStream_t st, int zadd = 1);
 gwb_status launch_tc_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
                           int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 gwb_status read_and_clear_device_error(cudaStream_t st, unsigned int *flag);
@@ -73,7 +75,7 @@ gwb_status launch_tc2_affine(const uint16_t *x, int64_t M, const uint32_t *wq, c
                              cudaStream_t st);
 gwb_status launch_tc2_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
                            const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *y,
-                           cudaStream_t st);
+                           cudaStream_t st, int zadd = 1);
 gwb_status launch_tc2_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
                            int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 gwb_status read_and_clear_device_error_tc2(cudaStream_t st, unsigned int *flag);

@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(256) k_gptq_dequant(const int32_t *__restrict_
                                                       const uint16_t *__restrict__ scales,
                                                       const int32_t *__restrict__ qzeros,
                                                       const int32_t *__restrict__ g_idx, int64_t K, int64_t N,
-                                                      int gs, uint16_t *__restrict__ out) {
+                                                      int gs, int zadd, uint16_t *__restrict__ out) {
   const int64_t total = (K / 8) * N;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (int64_t)gridDim.x * blockDim.x) {
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(256) k_gptq_dequant(const int32_t *__restrict_
       const int64_t g = g_idx ? (int64_t)g_idx[k] : k / gs;
       const float s = __half2float(__ushort_as_half(scales[g * N + o]));
       const uint32_t zw = static_cast<uint32_t>(qzeros[g * (N / 8) + o / 8]);
-      const int zero = (int)((zw >> ((o % 8) * 4)) & 0xFu) + 1;
+      const int zero = (int)((zw >> ((o % 8) * 4)) & 0xFu) + zadd;
       const int q = (int)((word >> (j * 4)) & 0xFu);
       const uint16_t h = __half_as_ushort(__float2half_rn(__fmul_rn(s, (float)(q - zero))));
       if (j & 1) packed[j / 2] |= (uint32_t)h << 16;
@@ -307,8 +307,9 @@ void launch_dequant_affine(const uint32_t *wq, const uint16_t *scales, const uin
 }
 
 void launch_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
-                         const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *w_out, cudaStream_t st) {
-  k_gptq_dequant<<<grid_for((K / 8) * N, 256), 256, 0, st>>>(qweight, scales, qzeros, g_idx, K, N, gs, w_out);
+                         const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *w_out, cudaStream_t st,
+                         int zadd) {
+  k_gptq_dequant<<<grid_for((K / 8) * N, 256), 256, 0, st>>>(qweight, scales, qzeros, g_idx, K, N, gs, zadd, w_out);
 }
 
 void launch_quant_per_token_i8(const uint16_t *x, int64_t M, int64_t K, int8_t *qx, float *sx,

@@ -53,6 +53,7 @@ struct TcArgs {
   uint16_t *y;              // bf16 (affine, i8) or fp16 (gptq) [M, N]
   int32_t *acc;             // i8: optional int32 [M, N]
   int staged_scales;        // 1: the producer copies each stage's scales (and zeros) into shared memory
+  int zadd;                 // gptq: added to the stored zero (1: GPTQ's convention, 0: AWQ's)
 };
 
 template <Fmt F, int BITS>
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           g = g < G ? g : G - 1;
           const uint32_t sv = __ldg(args.scales + (int64_t)g * args.N + nc);
           const uint32_t zw = (uint32_t)__ldg(args.qzeros + (int64_t)g * (args.N / 8) + nc / 8);
-          const uint32_t zv = 0x6400u | (((zw >> ((nc % 8) * 4)) & 0xFu) + 1u);
+          const uint32_t zv = 0x6400u | (((zw >> ((nc % 8) * 4)) & 0xFu) + (uint32_t)args.zadd);
 #pragma unroll
           for (int p = 0; p < 4; p++) { s2[p] = sv | (sv << 16); z2[p] = zv | (zv << 16); }
         }
@@ -258,7 +259,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW_BYTES);
           const uint32_t *zc = reinterpret_cast<const uint32_t *>(R + T::RAW_BYTES + 512);
           const uint32_t sv = sc[idx * kTileN + r];
-          const uint32_t zv = 0x6400u | (((zc[idx * 16 + r / 8] >> ((r % 8) * 4)) & 0xFu) + 1u);
+          const uint32_t zv = 0x6400u | (((zc[idx * 16 + r / 8] >> ((r % 8) * 4)) & 0xFu) + (uint32_t)args.zadd);
 #pragma unroll
           for (int p = 0; p < 4; p++) { s2[p] = sv | (sv << 16); z2[p] = zv | (zv << 16); }
         }
@@ -303,7 +304,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int g = k < args.K ? __ldg(args.g_idx + k) : 0;
                 sv[e] = __ldg(args.scales + (int64_t)g * args.N + nc);
                 const uint32_t zw = (uint32_t)__ldg(args.qzeros + (int64_t)g * (args.N / 8) + nc / 8);
-                zv[e] = 0x6400u | (((zw >> ((nc % 8) * 4)) & 0xFu) + 1u);
+                zv[e] = 0x6400u | (((zw >> ((nc % 8) * 4)) & 0xFu) + (uint32_t)args.zadd);
               }
               s2[p] = sv[0] | (sv[1] << 16);
               z2[p] = zv[0] | (zv[1] << 16);
@@ -461,10 +462,11 @@ gwb_status launch_tc_affine(const uint16_t *x, int64_t M, const uint32_t *wq, co
 
 gwb_status launch_tc_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
                           const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
-                          uint16_t *y, cudaStream_t st) {
+                          uint16_t *y, cudaStream_t st, int zadd) {
   TcArgs a{};
   a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
   a.scales = scales; a.qzeros = qzeros; a.g_idx = g_idx; a.y = y;
+  a.zadd = zadd;
   // 16-byte scale copies and 4-byte qzeros copies need those alignments.
   a.staged_scales = (g_idx == nullptr && ((uintptr_t)scales & 15) == 0 && ((uintptr_t)qzeros & 3) == 0) ? 1 : 0;
   CUtensorMap tw;

@@ -174,6 +174,7 @@ struct Args {
   int gs_log2;              // group size = 1 << gs_log2
   int sc_tma;               // affine: scales + biases arrive by TMA as [2 arrays][128 rows][8 groups]
   int sc_swap;              //   ... with the biases first (they sit below the scales in memory)
+  int zadd;                 // gptq: added to the stored zero (1: GPTQ's convention, 0: AWQ's)
   int Nt, T;                // feature tiles, tiles
   const uint16_t *scales;   // affine: bf16 [N, K/gs];   gptq: fp16 [K/gs, N]
   const uint16_t *biases;   // affine: bf16 [N, K/gs]
@@ -329,7 +330,7 @@ __device__ __forceinline__ void dequant_words(const Args &a, int k, int r, int h
     const uint16_t *sc = reinterpret_cast<const uint16_t *>(R + T::RAW);
     const uint32_t *zc = reinterpret_cast<const uint32_t *>(R + T::RAW + 512);
     const uint32_t sv = sc[idx * kTileN + r];
-    const uint32_t zv = 0x6400u | (((zc[idx * 16 + r / 8] >> ((r % 8) * 4)) & 0xFu) + 1u);
+    const uint32_t zv = 0x6400u | (((zc[idx * 16 + r / 8] >> ((r % 8) * 4)) & 0xFu) + (uint32_t)a.zadd);
     uint32_t s2[4], z2[4];
 #pragma unroll
     for (int p = 0; p < 4; p++) { s2[p] = sv | (sv << 16); z2[p] = zv | (zv << 16); }
@@ -1017,12 +1018,13 @@ gwb_status launch_tc2_affine_noalloc(const uint16_t *x, int64_t M, const uint32_
 
 gwb_status launch_tc2_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
                            const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *y,
-                           cudaStream_t st) {
+                           cudaStream_t st, int zadd) {
   if (g_idx != nullptr || ((uintptr_t)scales & 15) != 0 || ((uintptr_t)qzeros & 3) != 0) return GWB_ERR_UNSUPPORTED;
   Args a{};
   a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = gs;
   a.gs_log2 = gs == 32 ? 5 : (gs == 64 ? 6 : 7);
   a.scales = scales; a.qzeros = qzeros; a.y = y;
+  a.zadd = zadd;
   CUtensorMap tw;
   gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, qweight, (uint64_t)N, (uint64_t)(K / 8), (uint64_t)N * 4,
                        (uint32_t)kTileN, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);

@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     k_gemv_gptq(const uint16_t *__restrict__ x, int M, const int32_t *__restrict__ qweight,
                 const uint16_t *__restrict__ scales, const int32_t *__restrict__ qzeros,
                 const int32_t *__restrict__ g_idx, int N, int K, int gs, uint16_t *__restrict__ y, int RS,
-                int KR) {
+                int KR, int zadd) {
   constexpr int UNIT = 32, NMMA = 2, U = 4;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ float s_inv[8];
@@ -380,8 +380,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const __half sBh = __ushort_as_half(__ldg(scales + (int64_t)gq * N + nB));
         const uint32_t zwA = (uint32_t)__ldg(qzeros + (int64_t)gq * NZ + nA / 8);
         const uint32_t zwB = (uint32_t)__ldg(qzeros + (int64_t)gq * NZ + nB / 8);
-        const uint32_t zA = 0x6400u | (((zwA >> ((nA % 8) * 4)) & 0xFu) + 1u);
-        const uint32_t zB = 0x6400u | (((zwB >> ((nB % 8) * 4)) & 0xFu) + 1u);
+        const uint32_t zA = 0x6400u | (((zwA >> ((nA % 8) * 4)) & 0xFu) + (uint32_t)zadd);
+        const uint32_t zB = 0x6400u | (((zwB >> ((nB % 8) * 4)) & 0xFu) + (uint32_t)zadd);
         const __half2 zA2 = __halves2half2(__ushort_as_half(zA), __ushort_as_half(zA));
         const __half2 zB2 = __halves2half2(__ushort_as_half(zB), __ushort_as_half(zB));
         const __half2 sA2 = __halves2half2(sAh, sAh), sB2 = __halves2half2(sBh, sBh);
@@ -399,10 +399,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int glo = GT[kbase + i], ghi = GT[kbase + i + 4];
           const uint16_t sAl = __ldg(scales + (int64_t)glo * N + nA), sAh = __ldg(scales + (int64_t)ghi * N + nA);
           const uint16_t sBl = __ldg(scales + (int64_t)glo * N + nB), sBh = __ldg(scales + (int64_t)ghi * N + nB);
-          const uint32_t zAl = 0x6400u | ((((uint32_t)__ldg(qzeros + (int64_t)glo * NZ + nA / 8) >> ((nA % 8) * 4)) & 0xFu) + 1u);
-          const uint32_t zAh = 0x6400u | ((((uint32_t)__ldg(qzeros + (int64_t)ghi * NZ + nA / 8) >> ((nA % 8) * 4)) & 0xFu) + 1u);
-          const uint32_t zBl = 0x6400u | ((((uint32_t)__ldg(qzeros + (int64_t)glo * NZ + nB / 8) >> ((nB % 8) * 4)) & 0xFu) + 1u);
-          const uint32_t zBh = 0x6400u | ((((uint32_t)__ldg(qzeros + (int64_t)ghi * NZ + nB / 8) >> ((nB % 8) * 4)) & 0xFu) + 1u);
+          const uint32_t zAl = 0x6400u | ((((uint32_t)__ldg(qzeros + (int64_t)glo * NZ + nA / 8) >> ((nA % 8) * 4)) & 0xFu) + (uint32_t)zadd);
+          const uint32_t zAh = 0x6400u | ((((uint32_t)__ldg(qzeros + (int64_t)ghi * NZ + nA / 8) >> ((nA % 8) * 4)) & 0xFu) + (uint32_t)zadd);
+          const uint32_t zBl = 0x6400u | ((((uint32_t)__ldg(qzeros + (int64_t)glo * NZ + nB / 8) >> ((nB % 8) * 4)) & 0xFu) + (uint32_t)zadd);
+          const uint32_t zBh = 0x6400u | ((((uint32_t)__ldg(qzeros + (int64_t)ghi * NZ + nB / 8) >> ((nB % 8) * 4)) & 0xFu) + (uint32_t)zadd);
           const uint32_t zA2 = zAl | (zAh << 16), zB2 = zBl | (zBh << 16);
           const uint32_t sA2 = (uint32_t)sAl | ((uint32_t)sAh << 16), sB2 = (uint32_t)sBl | ((uint32_t)sBh << 16);
           __half2 qa = *reinterpret_cast<__half2 *>(&ra[i]), qb = *reinterpret_cast<__half2 *>(&rb[i]);
@@ -492,13 +492,13 @@ gwb_status run_affine(const uint16_t *x, int M, const uint32_t *wq, const uint16
 
 template <int MP, bool GIDX>
 gwb_status run_gptq(const uint16_t *x, int M, const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
-                    const int32_t *g_idx, int64_t N, int64_t K, int gs, uint16_t *y, cudaStream_t st) {
+                    const int32_t *g_idx, int64_t N, int64_t K, int gs, uint16_t *y, cudaStream_t st, int zadd) {
   const size_t per_k = 2 * MP + (GIDX ? 4 : 0);
   const size_t fixed = (kWarps * 128 + 8 * 16 * 8) * sizeof(float) + 64;
   GemvGeom g = plan(N, K, 32, MP, per_k, fixed);
   dim3 grid((unsigned)((N + 16 * g.RS - 1) / (16 * g.RS)), (unsigned)g.S);
   return launch_cluster(k_gemv_gptq<MP, GIDX>, grid, g.smem, g.S, st, x, M, qweight, scales, qzeros, g_idx, (int)N,
-                        (int)K, gs, y, g.RS, g.KR);
+                        (int)K, gs, y, g.RS, g.KR, zadd);
 }
 
 int pad_tokens(int M) { return M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8)); }
@@ -524,12 +524,12 @@ gwb_status launch_gemv_affine(const uint16_t *x, int M, const uint32_t *wq, cons
 
 gwb_status launch_gemv_gptq(const uint16_t *x, int M, const int32_t *qweight, const uint16_t *scales,
                             const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
-                            uint16_t *y, cudaStream_t st) {
+                            uint16_t *y, cudaStream_t st, int zadd) {
   const int MP = pad_tokens(M);
 #define GWB_GG(P)                                                                                   \
   if (MP == P) {                                                                                     \
-    if (g_idx) return run_gptq<P, true>(x, M, qweight, scales, qzeros, g_idx, N, K, gs, y, st);     \
-    return run_gptq<P, false>(x, M, qweight, scales, qzeros, g_idx, N, K, gs, y, st);               \
+    if (g_idx) return run_gptq<P, true>(x, M, qweight, scales, qzeros, g_idx, N, K, gs, y, st, zadd); \
+    return run_gptq<P, false>(x, M, qweight, scales, qzeros, g_idx, N, K, gs, y, st, zadd);         \
   }
   GWB_GG(1) GWB_GG(2) GWB_GG(4) GWB_GG(8)
 #undef GWB_GG

@@ -173,6 +173,17 @@ gwb_status gwb_gptq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, co
                         const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N,
                         int group_size, uint16_t *y, void *stream);
 
+/* awq_dequant / awq_qmm -- the same layout and shapes as gwb_gptq_dequant /
+ * gwb_gptq_qmm, with the zero taken as stored: zero = (qzeros[g, o/8] >> ((o%8)*4)) & 0xF,
+ * no "+1", and no g_idx (g = i / group_size).
+ * Source: GPTQ page (section 1, after the dequant recipe): auto-gptq stores
+ * zero - 1 and re-adds 1, AWQ does not; the AWQ reader has identical shapes.
+ * Only that difference is stated, so only it is implemented. */
+gwb_status gwb_awq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros, int64_t K,
+                           int64_t N, int group_size, uint16_t *w_out, void *stream);
+gwb_status gwb_awq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
+                       const int32_t *qzeros, int64_t K, int64_t N, int group_size, uint16_t *y, void *stream);
+
 /* ------------------------------------------------------------------ W4A8 */
 
 /* quant_per_token_i8 -- dynamic symmetric per-token int8 (qMax = 127), fp32:

@@ -59,6 +59,9 @@ def _load():
             "orc_gptq_dequant_f64": (None, [_P, _P, _P, _P, _I64, _I64, _INT, _P]),
             "orc_gptq_dequant_f16": (None, [_P, _P, _P, _P, _I64, _I64, _INT, _P]),
             "orc_gptq_qmm": (None, [_P, _I64, _P, _I64, _P, _P, _P, _P, _I64, _I64, _INT, _P]),
+            "orc_awq_dequant_f64": (None, [_P, _P, _P, _I64, _I64, _INT, _P]),
+            "orc_awq_dequant_f16": (None, [_P, _P, _P, _I64, _I64, _INT, _P]),
+            "orc_awq_qmm": (None, [_P, _I64, _P, _I64, _P, _P, _P, _I64, _I64, _INT, _P]),
             "orc_quant_per_token_i8": (None, [_P, _I64, _I64, _P, _P]),
             "orc_qpack_sym_i4": (None, [_P, _I64, _I64, _P, _P, _P]),
             "orc_gemm_i8i4": (_INT, [_P, _P, _I64, _P, _I64, _P, _P, _I64, _I64, _P, _P]),
@@ -193,6 +196,31 @@ def gptq_qmm(x_f16, qweight, scales, qzeros, g_idx, K, N, gs, rows=None):
     gi = None if g_idx is None else _c(g_idx, np.int32)
     y = np.empty((nr, N), np.float64)
     _load().orc_gptq_qmm(_p(x), M, _p(r), nr, _p(qw), _p(sc), _p(qz), _p(gi), K, N, gs, _p(y))
+    return y
+
+
+# ----------------------------------------------------------------- AWQ
+def awq_dequant_f64(qweight, scales, qzeros, K, N, gs):
+    qw, sc, qz = _c(qweight, np.int32), _c(scales, np.uint16), _c(qzeros, np.int32)
+    out = np.empty((N, K), np.float64)
+    _load().orc_awq_dequant_f64(_p(qw), _p(sc), _p(qz), K, N, gs, _p(out))
+    return out
+
+
+def awq_dequant_f16(qweight, scales, qzeros, K, N, gs):
+    qw, sc, qz = _c(qweight, np.int32), _c(scales, np.uint16), _c(qzeros, np.int32)
+    out = np.empty((N, K), np.uint16)
+    _load().orc_awq_dequant_f16(_p(qw), _p(sc), _p(qz), K, N, gs, _p(out))
+    return out
+
+
+def awq_qmm(x_f16, qweight, scales, qzeros, K, N, gs, rows=None):
+    x = _c(x_f16, np.uint16)
+    M = x.shape[0]
+    r, nr = _rows(rows, M)
+    qw, sc, qz = _c(qweight, np.int32), _c(scales, np.uint16), _c(qzeros, np.int32)
+    y = np.empty((nr, N), np.float64)
+    _load().orc_awq_qmm(_p(x), M, _p(r), nr, _p(qw), _p(sc), _p(qz), K, N, gs, _p(y))
     return y
 
 

@@ -27,6 +27,11 @@
  *   [GPTQ]  TinyGPT "Quantization Expansion", section 1 "GPTQReader", "Format"
  *           and the dequant recipe (qweight packed along IN, qzeros packed
  *           along OUT, zero = stored + 1, g = g_idx[i]).
+ *   [AWQZ]  TinyGPT "Quantization Expansion", section 1 "GPTQReader", the note
+ *           after the dequant recipe: the "+1" on the stored zero belongs to
+ *           GPTQ only; AWQ uses the stored zero as is.  The same note names
+ *           the AWQ reader as a sibling of identical shapes, and its g_idx
+ *           remark says plain AWQ has no g_idx.
  *   [QAT]   TinyGPT "Quantization Expansion", section 4 "QAT", "Fake-quant +
  *           STE": per-row symmetric scale = max|W|/qMax, clip(round(W/scale)),
  *           qMax = 2^(bits-1) - 1.
@@ -312,6 +317,58 @@ void orc_gptq_qmm(const uint16_t *x, int64_t M, const int64_t *rows, int64_t nro
             for (int64_t i = 0; i < K; i++)
                 acc += orc_f16_to_f64(x[m * K + i]) *
                        gptq_weight(qweight, scales, qzeros, g_idx, K, N, gs, o, i);
+            y[r * N + o] = acc;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* AWQ zero convention [AWQZ]: the GPTQ tensors and shapes, no g_idx, and    */
+/* the stored zero nibble taken as the zero itself.                          */
+/* ------------------------------------------------------------------------ */
+
+/* W[o, i] = scales[i/gs, o] * (int4 - zero),
+ *   int4 = (qweight[i/8, o] >> ((i%8)*4)) & 0xF,
+ *   zero = (qzeros[i/gs, o/8] >> ((o%8)*4)) & 0xF                         */
+static double awq_weight(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
+                         int64_t N, int gs, int64_t o, int64_t i)
+{
+    int64_t g = i / gs;
+    int int4 = (int)(((uint32_t)qweight[(i / 8) * N + o] >> ((i % 8) * 4)) & 0xFu);
+    int zero = (int)(((uint32_t)qzeros[g * (N / 8) + o / 8] >> ((o % 8) * 4)) & 0xFu);
+    return orc_f16_to_f64(scales[g * N + o]) * (double)(int4 - zero);
+}
+
+void orc_awq_dequant_f64(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
+                         int64_t K, int64_t N, int gs, double *w /* [N,K] */)
+{
+    for (int64_t o = 0; o < N; o++)
+        for (int64_t i = 0; i < K; i++)
+            w[o * K + i] = awq_weight(qweight, scales, qzeros, N, gs, o, i);
+}
+
+/* One rounding to binary16 of the exact fp64 product (11-bit scale times an
+ * integer in [-15, 15]). */
+void orc_awq_dequant_f16(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
+                         int64_t K, int64_t N, int gs, uint16_t *w /* [N,K] */)
+{
+    for (int64_t o = 0; o < N; o++)
+        for (int64_t i = 0; i < K; i++)
+            w[o * K + i] = orc_f64_to_f16(awq_weight(qweight, scales, qzeros, N, gs, o, i));
+}
+
+/* y[r, o] = sum_i x[rows[r], i] * W[o, i], x fp16 [M, K], fp64 accumulation. */
+void orc_awq_qmm(const uint16_t *x, int64_t M, const int64_t *rows, int64_t nrows,
+                 const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
+                 int64_t K, int64_t N, int gs, double *y)
+{
+    (void)M;
+    for (int64_t r = 0; r < nrows; r++) {
+        int64_t m = rows ? rows[r] : r;
+        for (int64_t o = 0; o < N; o++) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < K; i++)
+                acc += orc_f16_to_f64(x[m * K + i]) * awq_weight(qweight, scales, qzeros, N, gs, o, i);
             y[r * N + o] = acc;
         }
     }

@@ -221,6 +221,59 @@ def test_gptq_qmm_small(permuted, M):
     Gptq(384, 264, 128 if M % 2 else 64, permuted, seed=M).check_qmm(M)
 
 
+# --------------------------------------------------------------------------- AWQ zero convention
+class Awq:
+    """The GPTQ tensors without g_idx, the stored zero used as is."""
+
+    def __init__(self, K, N, gs, seed=0):
+        self.K, self.N, self.gs = K, N, gs
+        qw, sc, qz, _ = synth.gptq_quartet(K, N, gs, seed=seed)
+        self.h = (qw.numpy(), synth.bits16(sc), qz.numpy())
+        self.d = (qw.to(DEV), sc.to(DEV), qz.to(DEV))
+
+    def check_dequant(self):
+        w = gwb.awq_dequant(*self.d, self.gs)
+        ref = oracle.awq_dequant_f16(*self.h, self.K, self.N, self.gs)
+        assert np.array_equal(_np16(w), ref)
+        return float(w.float().abs().max())
+
+    def check_qmm(self, M, seed=1):
+        max_w = self.check_dequant()
+        x = synth.activations(M, self.K, seed=seed, dtype=torch.float16)
+        y = gwb.awq_qmm(x.to(DEV), *self.d, self.gs)
+        rows = _rows(M, self.N, self.K, budget=1e8)
+        y_ref = oracle.awq_qmm(synth.bits16(x), *self.h, self.K, self.N, self.gs, rows=rows)
+        yg = y.float().cpu().numpy()
+        if rows is not None:
+            yg = yg[rows]
+        return check_float(yg, y_ref, self.K, max_w, float(x.float().abs().max()), f"awq M={M}")
+
+
+@pytest.mark.parametrize("gs", [32, 128])
+def test_awq_dequant_bit_exact(gs):
+    Awq(512, 200, gs, seed=gs).check_dequant()
+
+
+@pytest.mark.parametrize("M", [1, 4, 8, 32, 150, 300])
+def test_awq_qmm_small(M):
+    Awq(384, 264, 128 if M % 2 else 64, seed=M).check_qmm(M)
+
+
+def test_awq_equals_gptq_with_stored_zero_minus_one():
+    """Both entry points on the same codes: AWQ with stored zeros z in 1..15 gives the same
+    fp16 weights and outputs as GPTQ with stored zeros z - 1."""
+    K, N, gs = 512, 192, 64
+    qw, sc, qz, _ = synth.gptq_quartet(K, N, gs, seed=9)
+    nib = [((qz.to(torch.int64) >> (4 * j)) & 0xF).clamp(min=1) for j in range(8)]
+    pack = lambda d: sum((v - d) << (4 * j) for j, v in enumerate(nib)).to(torch.uint32).view(torch.int32)
+    qz_awq, qz_gptq = pack(0).to(DEV), pack(1).to(DEV)
+    qw, sc = qw.to(DEV), sc.to(DEV)
+    assert torch.equal(gwb.awq_dequant(qw, sc, qz_awq, gs), gwb.gptq_dequant(qw, sc, qz_gptq, None, gs))
+    for M in (1, 200):
+        x = synth.activations(M, K, seed=M, dtype=torch.float16).to(DEV)
+        assert torch.equal(gwb.awq_qmm(x, qw, sc, qz_awq, gs), gwb.gptq_qmm(x, qw, sc, qz_gptq, None, gs))
+
+
 # --------------------------------------------------------------------------- W4A8
 class W4A8:
     def __init__(self, N, K, seed=0):
@@ -310,6 +363,12 @@ def test_full_gptq(permuted):
     g = Gptq(4096, 11008, 128, permuted)
     for M in (1, 32, 1024):
         g.check_qmm(M)
+
+
+def test_full_awq():
+    a = Awq(4096, 11008, 128)
+    for M in (1, 32, 1024):
+        a.check_qmm(M)
 
 
 @pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096), (4096, 14336)])

@@ -293,6 +293,63 @@ def test_gptq_qmm_against_numpy_and_permutation_invariance():
     assert np.allclose(y2, y, rtol=1e-12, atol=1e-12)
 
 
+# --------------------------------------------------------------------- AWQ zero convention
+def test_awq_worked_example_without_plus_one():
+    """The GPTQ smoke-test inputs read with the AWQ convention: the page says AWQ does not
+    re-add the 1, so the printed row [-1, ..., 14] moves up by exactly one to [0, ..., 15]."""
+    rows = {r[0]: r[1:] for r in _golden_lines("gptq_worked_example.txt")}
+    K, gs = int(rows["in_features"][0]), int(rows["group_size"][0])
+    N = 8
+    expected = np.array([float(v) for v in rows["row0"]]) + 1.0
+    qweight = np.zeros((K // 8, N), np.int64)
+    qweight[0, 0] = 0x76543210
+    qweight[1, 0] = 0xFEDCBA98
+    qweight = qweight.astype(np.uint32).view(np.int32)
+    qzeros = np.zeros((K // gs, N // 8), np.int32)   # stored zero 0 -> zero 0
+    scales = _f16(np.ones((K // gs, N)))
+    assert np.array_equal(oracle.awq_dequant_f64(qweight, scales, qzeros, K, N, gs)[0], expected)
+    W16 = oracle.awq_dequant_f16(qweight, scales, qzeros, K, N, gs)
+    assert np.array_equal(np.array([oracle.f16_to_f64(h) for h in W16[0]]), expected)
+
+
+def test_awq_zero_nibble_closed_form():
+    """qzeros packed along OUT, zero taken as stored: W[o, i] = s_g * (i - z_o) for codes
+    0..7, with a different scale per group (pins the group index i // gs and the nibble
+    index o % 8 of word o // 8)."""
+    K, N, gs = 16, 16, 8
+    qweight = np.full((2, N), 0x76543210, np.int64).astype(np.uint32).view(np.int32)  # codes i % 8
+    z = np.array([3, 0, 15, 7, 1, 2, 9, 4, 5, 6, 8, 10, 11, 12, 13, 14])
+    words = [sum(int(z[8 * w + j]) << (4 * j) for j in range(8)) for w in range(2)]
+    qzeros = np.array([words, words], np.int64).astype(np.uint32).view(np.int32)
+    scales = _f16(np.array([[0.5] * N, [-2.0] * N]))
+    W = oracle.awq_dequant_f64(qweight, scales, qzeros, K, N, gs)
+    i = np.arange(K)
+    for o in range(N):
+        assert np.array_equal(W[o], np.where(i < 8, 0.5, -2.0) * (i % 8 - z[o]))
+
+
+def test_awq_equals_gptq_with_stored_zero_minus_one():
+    """The one stated difference: AWQ with stored zero z is GPTQ with stored zero z - 1
+    (z >= 1, no g_idx), for every weight and for the matmul."""
+    rng = np.random.default_rng(31)
+    K, N, gs = 128, 24, 32
+    qweight = rng.integers(0, 2**32, size=(K // 8, N), dtype=np.uint64).astype(np.uint32).view(np.int32)
+    z = rng.integers(1, 16, size=(K // gs, N))
+    pack = lambda zz: sum(zz.reshape(K // gs, N // 8, 8)[:, :, j].astype(np.int64) << (4 * j) for j in range(8))
+    qz_awq = pack(z).astype(np.uint32).view(np.int32)
+    qz_gptq = pack(z - 1).astype(np.uint32).view(np.int32)
+    scales = _f16(rng.standard_normal((K // gs, N)) * 0.01).reshape(K // gs, N)
+    Wa = oracle.awq_dequant_f64(qweight, scales, qz_awq, K, N, gs)
+    assert np.array_equal(Wa, oracle.gptq_dequant_f64(qweight, scales, qz_gptq, None, K, N, gs))
+    assert np.array_equal(oracle.awq_dequant_f16(qweight, scales, qz_awq, K, N, gs),
+                          oracle.gptq_dequant_f16(qweight, scales, qz_gptq, None, K, N, gs))
+    x = _f16((rng.integers(-8, 9, size=(3, K)) * 0.125).astype(np.float32)).reshape(3, K)
+    ya = oracle.awq_qmm(x, qweight, scales, qz_awq, K, N, gs)
+    assert np.array_equal(ya, oracle.gptq_qmm(x, qweight, scales, qz_gptq, None, K, N, gs))
+    xf = np.array([[oracle.f16_to_f64(h) for h in row] for row in x])
+    assert np.allclose(ya, xf @ Wa.T, rtol=1e-13, atol=1e-13)
+
+
 # --------------------------------------------------------------------- W4A8
 def test_quant_per_token_i8_properties():
     """Per token: sx = amax/127 (fp32), the argmax hits +-127, codes are the nearest grid
