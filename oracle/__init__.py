@@ -65,6 +65,8 @@ def _load():
             "orc_quant_per_token_i8": (None, [_P, _I64, _I64, _P, _P]),
             "orc_qpack_sym_i4": (None, [_P, _I64, _I64, _P, _P, _P]),
             "orc_gemm_i8i4": (_INT, [_P, _P, _I64, _P, _I64, _P, _P, _I64, _I64, _P, _P]),
+            "orc_qpack_sym_i8": (None, [_P, _I64, _I64, _P, _P]),
+            "orc_gemm_i8i8": (_INT, [_P, _P, _I64, _P, _I64, _P, _P, _I64, _I64, _P, _P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -254,4 +256,27 @@ def gemm_i8i4(qx, sx, wq, sw, N, K, rows=None):
     acc = np.empty((nr, N), np.int64)
     y = np.empty((nr, N), np.float64)
     ovf = _load().orc_gemm_i8i4(_p(qx), _p(sx), M, _p(r), nr, _p(wq), _p(sw), N, K, _p(acc), _p(y))
+    return acc, y, bool(ovf)
+
+
+# ----------------------------------------------------------------- W8A8
+def qpack_sym_i8(w):
+    """Returns (wq int8 [N, K], sw float32 [N])."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    wq = np.empty((N, K), np.int8)
+    sw = np.empty((N,), np.float32)
+    _load().orc_qpack_sym_i8(_p(w), N, K, _p(wq), _p(sw))
+    return wq, sw
+
+
+def gemm_i8i8(qx, sx, wq, sw, N, K, rows=None):
+    """Returns (acc int64 [R, N], y fp64 [R, N], overflow flag)."""
+    qx, sx = _c(qx, np.int8), _c(sx, np.float32)
+    wq, sw = _c(wq, np.int8), _c(sw, np.float32)
+    M = qx.shape[0]
+    r, nr = _rows(rows, M)
+    acc = np.empty((nr, N), np.int64)
+    y = np.empty((nr, N), np.float64)
+    ovf = _load().orc_gemm_i8i8(_p(qx), _p(sx), M, _p(r), nr, _p(wq), _p(sw), N, K, _p(acc), _p(y))
     return acc, y, bool(ovf)

@@ -38,6 +38,10 @@
  *   [W4A8]  executorch PR #24467 "mlx::int8_int4_gemm": dynamic symmetric
  *           per-token int8 activations x symmetric per-channel int4 weights,
  *           INT32 accumulation.
+ *   [W8A8]  executorch PR #17234, Parakeet README "Quantization Configs":
+ *           8da8w = 8-bit dynamic activations x 8-bit weights; the weights
+ *           take the per-row symmetric quantizer of [QAT] with bits = 8
+ *           (qMax = 127, clip to [-qMax, +qMax]).
  *   [LIN]   executorch PR #17234 DecomposeLinearPass and mlx_int8.rs gemm doc:
  *           linear(x, W) = x . W^T with W stored [out, in].
  */
@@ -455,6 +459,57 @@ int orc_gemm_i8i4(const int8_t *qx, const float *sx, int64_t M, const int64_t *r
             int64_t a = 0;
             for (int64_t k = 0; k < K; k++)
                 a += (int64_t)qx[m * K + k] * (int64_t)sym_i4_code(wq, K, n, k);
+            if (a > INT32_MAX || a < INT32_MIN) overflow = 1;
+            if (acc) acc[r * N + n] = a;
+            if (y) y[r * N + n] = (double)a * (double)sx[m] * (double)sw[n];
+        }
+    }
+    return overflow;
+}
+
+/* ------------------------------------------------------------------------ */
+/* W8A8 [W8A8]: per-token int8 activations (orc_quant_per_token_i8) x       */
+/* per-output-channel symmetric int8 weights, INT32 accumulation.           */
+/* ------------------------------------------------------------------------ */
+
+/* [QAT] with bits = 8: sw = max_k |w[n,k]| / 127, q = clip(round_half_even(w / sw),
+ * -127, 127), fp32 arithmetic; sw == 0 gives q = 0.  wq int8 [N, K]. */
+void orc_qpack_sym_i8(const float *w, int64_t N, int64_t K, int8_t *wq, float *sw)
+{
+    for (int64_t n = 0; n < N; n++) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; k++) {
+            float v = fabsf(w[n * K + k]);
+            if (v > amax) amax = v;
+        }
+        float s = amax / 127.0f;
+        sw[n] = s;
+        for (int64_t k = 0; k < K; k++) {
+            int q = 0;
+            if (s != 0.0f) {
+                float r = rintf(w[n * K + k] / s);
+                if (r < -127.0f) r = -127.0f;
+                if (r > 127.0f) r = 127.0f;
+                q = (int)r;
+            }
+            wq[n * K + k] = (int8_t)q;
+        }
+    }
+}
+
+/* acc[r, n] = sum_k qx[rows[r], k] * wq[n, k] in int64;  y = acc * sx[m] * sw[n]
+ * in fp64.  Returns 0, or 1 when some accumulator does not fit in int32. */
+int orc_gemm_i8i8(const int8_t *qx, const float *sx, int64_t M, const int64_t *rows, int64_t nrows,
+                  const int8_t *wq, const float *sw, int64_t N, int64_t K, int64_t *acc, double *y)
+{
+    int overflow = 0;
+    (void)M;
+    for (int64_t r = 0; r < nrows; r++) {
+        int64_t m = rows ? rows[r] : r;
+        for (int64_t n = 0; n < N; n++) {
+            int64_t a = 0;
+            for (int64_t k = 0; k < K; k++)
+                a += (int64_t)qx[m * K + k] * (int64_t)wq[n * K + k];
             if (a > INT32_MAX || a < INT32_MIN) overflow = 1;
             if (acc) acc[r * N + n] = a;
             if (y) y[r * N + n] = (double)a * (double)sx[m] * (double)sw[n];

@@ -431,3 +431,57 @@ def test_symmetric_quant_error_bounds():
     xf = x.float().numpy()
     q = qx.astype(np.float64)
     assert np.all(np.abs(q * sx[:, None] - xf) <= sx[:, None] * (0.5 + np.abs(q) * 2.0 ** -23))
+
+
+# --------------------------------------------------------------------- W8A8
+def test_qpack_sym_i8_hand_values():
+    """Per-row symmetric int8 with qMax = 127 (QAT section, bits = 8): a row whose max is 127
+    has sw = 1, so codes are the row itself rounded half to even (63.5 -> 64, 0.5 -> 0,
+    -2.5 -> -2, 1.5 -> 2); a constant -1 row maps to -127; a zero row gives sw = 0, codes 0;
+    clipping is to [-127, 127] (never -128)."""
+    w = np.zeros((3, 16), np.float32)
+    w[0, :8] = [127, -127, 63.5, 0.5, -2.5, 1.5, -0.25, 100.49]
+    w[1, :] = -1.0
+    wq, sw = oracle.qpack_sym_i8(w)
+    assert sw.tolist() == [1.0, np.float32(np.float32(1.0) / np.float32(127.0)), 0.0]
+    assert wq[0, :8].tolist() == [127, -127, 64, 0, -2, 2, 0, 100]
+    assert np.all(wq[0, 8:] == 0) and np.all(wq[1] == -127) and np.all(wq[2] == 0)
+
+
+def test_qpack_sym_i8_nearest_grid_point():
+    """Every code is the nearest point of sw*[-127..127] (so the reconstruction error is at
+    most half a step, the page's 1/qMax bound), the row max maps to +-127, and negating the
+    row negates the codes."""
+    W = synth.weights(16, 384, seed=13).numpy()
+    wq, sw = oracle.qpack_sym_i8(W)
+    grid = np.arange(-127, 128, dtype=np.float64)
+    for n in range(16):
+        assert sw[n] == np.float32(np.float32(np.abs(W[n]).max()) / np.float32(127.0))
+        assert abs(int(wq[n, np.argmax(np.abs(W[n]))])) == 127
+        dist = np.abs(W[n].astype(np.float64)[:, None] - grid[None, :] * float(sw[n]))
+        chosen = dist[np.arange(384), wq[n].astype(np.int64) + 127]
+        # the decision is taken on the fp32 quotient w/sw, off by up to 127 * 2^-24 steps
+        assert np.all(chosen <= dist.min(axis=1) + 2.0 ** -16 * float(sw[n]))
+    wn, sn = oracle.qpack_sym_i8(-W)
+    assert np.array_equal(wn, -wq) and np.array_equal(sn, sw)
+
+
+def test_gemm_i8i8_integer_product_and_overflow_flag():
+    """acc equals numpy's int64 product of the int8 codes (pins the K pairing and the [N, K]
+    weight orientation: a transposed operand fails for N != M); y = acc*sx*sw; the flag
+    reports int32 overflow."""
+    rng = np.random.default_rng(4)
+    M, N, K = 5, 7, 96
+    qx = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+    wq = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    sx = rng.random(M).astype(np.float32)
+    sw = rng.random(N).astype(np.float32)
+    acc, y, ovf = oracle.gemm_i8i8(qx, sx, wq, sw, N, K)
+    ref = qx.astype(np.int64) @ wq.astype(np.int64).T
+    assert np.array_equal(acc, ref) and not ovf
+    assert np.allclose(y, ref * sx.astype(np.float64)[:, None] * sw.astype(np.float64)[None, :],
+                       rtol=1e-15, atol=0)
+    Kb = 1 << 18          # 127 * 127 * 2^18 > 2^31 - 1
+    acc2, _, ovf2 = oracle.gemm_i8i8(np.full((1, Kb), 127, np.int8), np.ones(1, np.float32),
+                                     np.full((1, Kb), -127, np.int8), np.ones(1, np.float32), 1, Kb)
+    assert ovf2 and acc2[0, 0] == -127 * 127 * Kb
