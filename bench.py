@@ -263,7 +263,12 @@ def run_gpu(args, world, rank, local):
     e2e_value = world * STEP_BYTES * args.steps / (e_ms * 1e-3) / 1e9
 
     prefill = run_prefill(gwb, dev, stream, bf16_peak, peak_kind) if not args.no_prefill else None
-    w4a8 = run_w4a8(gwb, dev, stream) if not args.no_prefill else None
+    int8 = {}
+    if not args.no_prefill:
+        i8peak = int8_peak_tops(dev, stream)
+        int8["w4a8_m4096"] = run_int8(gwb, dev, stream, "w4a8", 14336, 4096, 4096, i8peak, hbm_peak)
+        int8["w8a8_m4096"] = run_int8(gwb, dev, stream, "w8a8", 14336, 4096, 4096, i8peak, hbm_peak)
+        int8["w8a8_m1"] = run_int8(gwb, dev, stream, "w8a8", 14336, 4096, 1, i8peak, hbm_peak)
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -285,8 +290,7 @@ def run_gpu(args, world, rank, local):
     }
     if prefill:
         out["prefill_m2048"] = prefill
-    if w4a8:
-        out["w4a8_m4096"] = w4a8
+    out.update(int8)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
     if rank == 0:
@@ -311,38 +315,61 @@ def int8_peak_tops(dev, stream, reps=5):
     return 2.0 * 8192 ** 3 / (best * 1e-3) / 1e12
 
 
-def run_w4a8(gwb, dev, stream, reps=5):
-    """W4A8 GEMM (int8 x int4 -> int32, bf16 out) at N x K = 14336 x 4096, M = 4096,
-    each launch timed alone with an L2 flush before it; ops = 2 M N K."""
-    N, K, M = 14336, 4096, 4096
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+def int8_operands(gwb, dev, fmt, N, K, M, seed=91):
+    """Quantized weights (fmt 'w4a8': int4 codes, 'w8a8': int8) and per-token int8 activations."""
     g = torch.Generator(device=dev)
-    g.manual_seed(91)
+    g.manual_seed(seed)
     w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
-    wq, sw = gwb.qpack_sym_i4(w)
+    wq, sw = gwb.qpack_sym_i4(w) if fmt == "w4a8" else gwb.qpack_sym_i8(w)
     del w
     x = synth.activations(M, K, seed=1).to(dev)
     qx, sx = gwb.quant_per_token_i8(x)
+    return wq, sw, qx, sx
+
+
+def int8_gemm(gwb, fmt):
+    return gwb.gemm_i8i4 if fmt == "w4a8" else gwb.gemm_i8i8
+
+
+def run_int8(gwb, dev, stream, fmt, N, K, M, int8_peak, hbm_peak, reps=5):
+    """int8-activation GEMM (fmt 'w4a8' or 'w8a8', int32 accumulation, bf16 out) on an N x K
+    weight at M tokens, each launch timed alone with an L2 flush before it.  M = 1 is
+    HBM-bound (bytes = weights + scales + activations + output); larger M is tensor-bound
+    (ops = 2 M N K)."""
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    wq, sw, qx, sx = int8_operands(gwb, dev, fmt, N, K, M)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    gemm = int8_gemm(gwb, fmt)
     ts = []
     with torch.cuda.stream(stream):
         for r in range(reps + 2):
             flush.fill_(r)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            gwb.gemm_i8i4(qx, sx, wq, sw, y=y)
+            gemm(qx, sx, wq, sw, y=y)
             b.record(stream)
             b.synchronize()
             if r >= 2:
                 ts.append(a.elapsed_time(b))
     ms = statistics.median(ts)
-    tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
-    peak = int8_peak_tops(dev, stream)
-    return {"value": round(tops, 1), "unit": "TOP/s", "N": N, "K": K, "M": M, "us": round(ms * 1e3, 1),
-            "roofline": {"kernel": "k_tc2<I8,4,256,pair,A in TMEM> (kind::i8)", "bound": "tensor",
-                         "achieved": round(tops, 1), "peak": round(peak, 1), "unit": "TOP/s",
-                         "frac": round(tops / peak, 4),
-                         "peak_source": "measured in this run: torch._int_mm 8192^3 int8, best of 5"}}
+    kern = "k_tc2<I8,4,256,pair,A in TMEM> (kind::i8)" if fmt == "w4a8" else \
+        "k_tc2<W8,8,%s> (kind::i8, both operands by TMA)" % ("256,pair" if M > 128 else "128" if M > 32 else "32")
+    out = {"N": N, "K": K, "M": M, "us": round(ms * 1e3, 1)}
+    if M <= 8:
+        wbytes = N * K // (2 if fmt == "w4a8" else 1)
+        nbytes = wbytes + N * 4 + M * K + M * 4 + M * N * 2
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out.update({"value": round(gbs, 1), "unit": "GB/s",
+                    "roofline": {"kernel": kern, "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak,
+                                 "unit": "GB/s", "frac": round(gbs / hbm_peak, 4), "bytes_per_launch": nbytes,
+                                 "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}})
+    else:
+        tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        out.update({"value": round(tops, 1), "unit": "TOP/s",
+                    "roofline": {"kernel": kern, "bound": "tensor", "achieved": round(tops, 1),
+                                 "peak": round(int8_peak, 1), "unit": "TOP/s", "frac": round(tops / int8_peak, 4),
+                                 "peak_source": "measured in this run: torch._int_mm 8192^3 int8, best of 5"}})
+    return out
 
 
 def run_prefill(gwb, dev, stream, bf16_peak, peak_kind, reps=5):
@@ -447,30 +474,43 @@ def run_reference(args, world, rank):
 
 
 def run_layer(args):
-    """One layer only (for profiling): qmm_affine on an N x K weight at M tokens, replayed in a
-    CUDA graph of 20 launches that alternate between two weight sets (> L2)."""
+    """One layer only (for profiling): qmm_affine (or, with --fmt, the int8-activation GEMM) on an
+    N x K weight at M tokens, replayed in a CUDA graph of 20 launches that alternate between two
+    weight sets (> L2)."""
     import group_wise_bit_b200 as gwb
     N, K, bits, M = (list(map(int, args.layer.split(","))) + [1])[:4]
     dev = torch.device("cuda", 0)
-    sets = []
-    for s in range(2):
-        g = torch.Generator(device=dev)
-        g.manual_seed(s)
-        w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
-        sets.append(gwb.qpack_affine(w, bits, GS))
-        del w
-    x = synth.activations(M, K, seed=1).to(dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if args.fmt == "affine":
+        sets = []
+        for s in range(2):
+            g = torch.Generator(device=dev)
+            g.manual_seed(s)
+            w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+            sets.append(gwb.qpack_affine(w, bits, GS))
+            del w
+        x = synth.activations(M, K, seed=1).to(dev)
+
+        def launch(i):
+            wq, sc, bi = sets[i % 2]
+            gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+    else:
+        sets = [int8_operands(gwb, dev, args.fmt, N, K, M, seed=s) for s in range(2)]
+        gemm = int8_gemm(gwb, args.fmt)
+        bits = 4 if args.fmt == "w4a8" else 8
+
+        def launch(i):
+            wq, sw, qx, sx = sets[i % 2]
+            gemm(qx, sx, wq, sw, y=y)
     st = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(st):
-        for wq, sc, bi in sets:
-            gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+        for i in range(2):
+            launch(i)
         torch.cuda.synchronize()
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=st):
             for i in range(20):
-                wq, sc, bi = sets[i % 2]
-                gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+                launch(i)
         for _ in range(args.warmup):
             gr.replay()
         torch.cuda.synchronize()
@@ -481,12 +521,16 @@ def run_layer(args):
         b.record(st)
     torch.cuda.synchronize()
     us = a.elapsed_time(b) * 1e3 / (20 * args.steps)
-    nbytes = gemv_bytes(N, K, bits, M=M) if M <= 8 else None
-    out = {"layer": {"N": N, "K": K, "bits": bits, "group_size": GS, "M": M}, "us_per_launch": round(us, 2)}
+    if args.fmt == "affine":
+        nbytes = gemv_bytes(N, K, bits, M=M) if M <= 8 else None
+    else:
+        nbytes = (N * K * bits // 8 + N * 4 + M * K + M * 4 + M * N * 2) if M <= 8 else None
+    out = {"layer": {"fmt": args.fmt, "N": N, "K": K, "bits": bits, "group_size": GS, "M": M},
+           "us_per_launch": round(us, 2)}
     if nbytes:
         out["GB/s"] = round(nbytes / us / 1e3, 1)
     else:
-        out["TFLOP/s"] = round(2.0 * M * N * K / us / 1e6, 1)
+        out["TFLOP/s" if args.fmt == "affine" else "TOP/s"] = round(2.0 * M * N * K / us / 1e6, 1)
     print(json.dumps(out), flush=True)
 
 
@@ -497,11 +541,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["gwb", "reference"], default="gwb")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--fmt", choices=["affine", "w4a8", "w8a8"], default="affine",
+                    help="--layer: weight format (affine: MLX group-wise, bits from --layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-frac", type=float, default=1 / 16)
     ap.add_argument("--layer", default=None,
-                    help="N,K,bits[,M]: time one qmm_affine layer (group size 64) instead of the sweep")
+                    help="N,K,bits[,M]: time one layer (qmm_affine at group size 64, or --fmt) instead of the sweep")
     args = ap.parse_args()
     if args.layer:
         run_layer(args)

@@ -36,6 +36,8 @@ SIGNATURES = {
     "gwb_quant_per_token_i8": [_P, _I64, _I64, _P, _P, _P],
     "gwb_qpack_sym_i4": [_P, _I64, _I64, _P, _P, _P],
     "gwb_gemm_i8i4": [_P, _P, _I64, _P, _P, _I64, _I64, _P, _P, _P],
+    "gwb_qpack_sym_i8": [_P, _I64, _I64, _P, _P, _P],
+    "gwb_gemm_i8i8": [_P, _P, _I64, _P, _P, _I64, _I64, _P, _P, _P],
     "gwb_check_device_error": [_P],
 }
 
@@ -251,6 +253,33 @@ def gemm_i8i4(qx, sx, wq, sw, want_y=True, want_acc=False, y=None, acc=None):
     if want_acc or acc is not None:
         acc = _out(acc, "acc", (M, N), torch.int32, qx.device)
     _call("gwb_gemm_i8i4", _ptr(qx), _ptr(sx), M, _ptr(wq), _ptr(sw), N, K, _ptr(y), _ptr(acc), _stream())
+    return y, acc
+
+
+# ------------------------------------------------------------------ W8A8
+def qpack_sym_i8(w, wq=None, sw=None):
+    """w fp32 [N, K] -> (wq int8 [N, K], sw fp32 [N])."""
+    _dev(w, "w", (torch.float32,))
+    N, K = w.shape
+    wq = _out(wq, "wq", (N, K), torch.int8, w.device)
+    sw = _out(sw, "sw", (N,), torch.float32, w.device)
+    _call("gwb_qpack_sym_i8", _ptr(w), N, K, _ptr(wq), _ptr(sw), _stream())
+    return wq, sw
+
+
+def gemm_i8i8(qx, sx, wq, sw, want_y=True, want_acc=False, y=None, acc=None):
+    """-> (y bf16 [M, N] or None, acc int32 [M, N] or None)."""
+    _dev(qx, "qx", (torch.int8,))
+    M, K = qx.shape
+    N = wq.shape[0]
+    _dev(sx, "sx", (torch.float32,), (M,))
+    _dev(wq, "wq", (torch.int8,), (N, K))
+    _dev(sw, "sw", (torch.float32,), (N,))
+    if want_y or y is not None:
+        y = _out(y, "y", (M, N), torch.bfloat16, qx.device)
+    if want_acc or acc is not None:
+        acc = _out(acc, "acc", (M, N), torch.int32, qx.device)
+    _call("gwb_gemm_i8i8", _ptr(qx), _ptr(sx), M, _ptr(wq), _ptr(sw), N, K, _ptr(y), _ptr(acc), _stream())
     return y, acc
 
 

@@ -287,4 +287,41 @@ gwb_status gwb_gemm_i8i4(const int8_t *qx, const float *sx, int64_t M, const uin
   return gwb::launch_tc_i8i4(qx, sx, M, wq, sw, N, K, y, acc, as_stream(stream));
 }
 
+gwb_status gwb_qpack_sym_i8(const float *w, int64_t N, int64_t K, int8_t *wq, float *sw, void *stream) {
+  if (N < 0 || K < 0) return fail(GWB_ERR_INVALID_ARG, "negative size (N=%lld, K=%lld)", (long long)N, (long long)K);
+  if (N >= kMaxDim || K >= kMaxDim) return fail(GWB_ERR_SHAPE, "N and K must be below 2^31");
+  if (K % 16 != 0) return fail(GWB_ERR_SHAPE, "K=%lld is not a multiple of 16", (long long)K);
+  if (N == 0) return GWB_OK;
+  GWB_TRY(need(sw, "sw"));
+  if (K > 0) {
+    GWB_TRY(need(w, "w"));
+    GWB_TRY(need(wq, "wq"));
+  }
+  gwb::launch_qpack_sym_i8(w, N, K, wq, sw, as_stream(stream));
+  return gwb::check_launch("qpack_sym_i8");
+}
+
+gwb_status gwb_gemm_i8i8(const int8_t *qx, const float *sx, int64_t M, const int8_t *wq, const float *sw,
+                         int64_t N, int64_t K, uint16_t *y, int32_t *acc, void *stream) {
+  if (M < 0 || N < 0 || K < 0)
+    return fail(GWB_ERR_INVALID_ARG, "negative size (M=%lld, N=%lld, K=%lld)", (long long)M, (long long)N,
+                (long long)K);
+  if (M >= kMaxDim || N >= kMaxDim) return fail(GWB_ERR_SHAPE, "M and N must be below 2^31");
+  if (K % 16 != 0) return fail(GWB_ERR_SHAPE, "K=%lld is not a multiple of 16", (long long)K);
+  if (K > 131072) return fail(GWB_ERR_SHAPE, "K=%lld exceeds 131072 (int32 accumulator bound)", (long long)K);
+  if (!y && !acc) return fail(GWB_ERR_INVALID_ARG, "at least one of y and acc must be non-NULL");
+  if (M == 0 || N == 0) return GWB_OK;
+  if (K == 0) {
+    if (y) GWB_TRY(zero_fill(y, (size_t)M * N * 2, stream));
+    if (acc) GWB_TRY(zero_fill(acc, (size_t)M * N * 4, stream));
+    return GWB_OK;
+  }
+  GWB_TRY(need(qx, "qx"));
+  GWB_TRY(need(sx, "sx"));
+  GWB_TRY(need(wq, "wq"));
+  GWB_TRY(need(sw, "sw"));
+  if (!aligned16(qx) || !aligned16(wq)) return fail(GWB_ERR_ALIGN, "qx and wq must be 16-byte aligned");
+  return gwb::launch_tc2_i8i8(qx, sx, M, wq, sw, N, K, y, acc, as_stream(stream));
+}
+
 }  // extern "C"

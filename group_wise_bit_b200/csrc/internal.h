@@ -26,6 +26,7 @@ void launch_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const i
                          int zadd = 1);
 void launch_quant_per_token_i8(const uint16_t *x, int64_t M, int64_t K, int8_t *qx, float *sx,
                                cudaStream_t st);
+void launch_qpack_sym_i8(const float *w, int64_t N, int64_t K, int8_t *wq, float *sw, cudaStream_t st);
 void launch_qpack_sym_i4(const float *w, int64_t N, int64_t K, uint32_t *wq, float *sw, cudaStream_t st);
 
 // ------------------------------------------------------------ GEMV regime (M <= 8)
@@ -76,6 +77,8 @@ gwb_status launch_tc2_affine(const uint16_t *x, int64_t M, const uint32_t *wq, c
 gwb_status launch_tc2_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
                            const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *y,
                            cudaStream_t st, int zadd = 1);
+gwb_status launch_tc2_i8i8(const int8_t *qx, const float *sx, int64_t M, const int8_t *wq, const float *sw,
+                           int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 gwb_status launch_tc2_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
                            int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 gwb_status read_and_clear_device_error_tc2(cudaStream_t st, unsigned int *flag);

@@ -280,6 +280,44 @@ int grid_for(int64_t work, int threads) {
   return (int)(b < 1 ? 1 : b);
 }
 
+
+// ----------------------------------------------------------------------------
+// qpack_sym_i8: one warp per output row; pass 1 reduces max|w|, pass 2 writes
+// sixteen int8 codes per 16-byte store (K % 16 == 0).
+__global__ void __launch_bounds__(256) k_qpack_sym_i8(const float *__restrict__ w, int64_t N, int64_t K,
+                                                      int8_t *__restrict__ wq, float *__restrict__ sw) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (n >= N) return;
+  const float *row = w + n * K;
+  float amax = 0.0f;
+  for (int64_t i = lane; i < K / 4; i += 32) {
+    const float4 t = reinterpret_cast<const float4 *>(row)[i];
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
+  }
+  for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, off));
+  const float s = __fdiv_rn(amax, 127.0f);
+  if (lane == 0) sw[n] = s;
+  for (int64_t ci = lane; ci < K / 16; ci += 32) {
+    const float4 *src = reinterpret_cast<const float4 *>(row + ci * 16);
+    uint32_t packed[4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; q4++) {
+      const float4 t = src[q4];
+      const float v[4] = {t.x, t.y, t.z, t.w};
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        int q = 0;
+        if (s != 0.0f) q = (int)fminf(fmaxf(rintf(__fdiv_rn(v[j], s)), -127.0f), 127.0f);
+        word |= ((uint32_t)q & 0xFFu) << (8 * j);
+      }
+      packed[q4] = word;
+    }
+    reinterpret_cast<uint4 *>(wq + n * K)[ci] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  }
+}
+
 }  // namespace
 
 void launch_qpack_affine(const float *w, int64_t N, int64_t K, int bits, int gs, uint32_t *wq,
@@ -315,6 +353,10 @@ void launch_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const i
 void launch_quant_per_token_i8(const uint16_t *x, int64_t M, int64_t K, int8_t *qx, float *sx,
                                cudaStream_t st) {
   k_quant_per_token_i8<<<(unsigned)M, 256, 0, st>>>(x, K, qx, sx);
+}
+
+void launch_qpack_sym_i8(const float *w, int64_t N, int64_t K, int8_t *wq, float *sw, cudaStream_t st) {
+  k_qpack_sym_i8<<<(unsigned)((N + 7) / 8), 256, 0, st>>>(w, N, K, wq, sw);
 }
 
 void launch_qpack_sym_i4(const float *w, int64_t N, int64_t K, uint32_t *wq, float *sw, cudaStream_t st) {

@@ -167,7 +167,10 @@ constexpr int kMaxSmem = 232448;
 constexpr int kSMs = 148;
 constexpr bool kAInTmem = true;   // pairs keep the dequantized A operand in tensor memory
 
-enum class Fmt { Affine, Gptq, I8 };
+// Affine / Gptq: 16-bit activations x dequantized weights; I8: int8
+// activations x int4 codes; W8: int8 activations x int8 weights, which need no
+// dequantization and go by TMA straight into the A stages.
+enum class Fmt { Affine, Gptq, I8, W8 };
 
 struct Args {
   int M, N, K, gs;
@@ -234,6 +237,14 @@ struct Tr<Fmt::Gptq, 4> {
   static constexpr int CP = 32;
 };
 template <>
+struct Tr<Fmt::W8, 8> {
+  static constexpr int BK = 128;
+  static constexpr int RAW = 0;
+  static constexpr int SC = 0;
+  static constexpr int NMMA = BK / 32;
+  static constexpr int CP = 0;
+};
+template <>
 struct Tr<Fmt::I8, 4> {
   static constexpr int BK = 128;                      // 128 int8 = 128 bytes per row
   static constexpr int RAW = kTileN * BK / 2;
@@ -248,23 +259,28 @@ struct Tr<Fmt::I8, 4> {
 // activation slots as it can.  The packed-weight ring takes what is left, up to 8.
 // With ATM the dequantized A stages live in tensor memory (8 slots of 32
 // columns next to one 256-column accumulator) and take no shared memory.
+// W8 has no packed-weight ring: activation and weight stages go in lockstep,
+// as many of each as fit (up to 8).
 template <Fmt F, int BITS, int BT, int PAIR, bool ATM>
 struct Plan2 {
+  static constexpr bool W8 = F == Fmt::W8;
   static constexpr int XB = BT / PAIR * 128;
   static constexpr int AB = kTileN * 128;
   static constexpr int RB = (Tr<F, BITS>::RAW + Tr<F, BITS>::SC + 127) / 128 * 128;
-  static constexpr int SA = ATM ? 8 : (PAIR == 2 ? 6 : 3);
-  static constexpr int A_SMEM = ATM ? 0 : SA * AB;
   // ATM: a bf16 staging tile [BT tokens][128 rows] for the epilogue, so that it
   // frees the single accumulator before writing the output
   static constexpr int EPI = ATM ? BT * kTileN * 2 : 0;
   static constexpr int BUDGET = kMaxSmem - 1024 - 1024 - 1024;   // alignment, barriers, static
+  static constexpr int SW8 = (BUDGET - EPI) / (XB + AB) > 8 ? 8 : (BUDGET - EPI) / (XB + AB);
+  static constexpr int SA = ATM ? 8 : W8 ? SW8 : (PAIR == 2 ? 6 : 3);
+  static constexpr int A_SMEM = ATM ? 0 : SA * AB;
   static constexpr int SXF = (BUDGET - A_SMEM - EPI - 4 * RB) / XB > 6 ? 6 : (BUDGET - A_SMEM - EPI - 4 * RB) / XB;
-  static constexpr int SX = PAIR == 2 && !ATM && SXF > 4 ? 4 : SXF;
-  static constexpr int SR0 = (BUDGET - A_SMEM - EPI - SX * XB) / RB;
-  static constexpr int SR = SR0 > 8 ? 8 : SR0;
+  static constexpr int SX = W8 ? SW8 : PAIR == 2 && !ATM && SXF > 4 ? 4 : SXF;
+  static constexpr int SR0 = RB ? (BUDGET - A_SMEM - EPI - SX * XB) / RB : 0;
+  static constexpr int SR = W8 ? 0 : SR0 > 8 ? 8 : SR0;
   static constexpr int SMEM = SX * XB + A_SMEM + EPI + SR * RB + 1024 + 1024;
-  static_assert(SX >= 2 && SR >= 4, "shared memory too small");
+  static_assert(SX >= 2 && (W8 || SR >= 4), "shared memory too small");
+  static_assert(!(W8 && ATM), "int8 weights are read from shared memory");
 };
 
 __device__ __forceinline__ void put4(uint32_t (&o)[16], int j, uint4 v) {
@@ -374,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NACC = ATM ? 1 : 2;
   constexpr uint32_t ACOL = BT;                        // first A slot column (ATM)
   static_assert(!ATM || (PAIR == 2 && BT == 256), "A in tensor memory is laid out for 256-token pairs");
-  constexpr uint32_t IDESC = (F == Fmt::I8) ? make_idesc(2, 1, kTileN * PAIR, BT)
+  constexpr bool kInt = F == Fmt::I8 || F == Fmt::W8;   // kind::i8, s32 accumulators
+  constexpr uint32_t IDESC = kInt ? make_idesc(2, 1, kTileN * PAIR, BT)
                              : (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN * PAIR, BT)
                                                 : make_idesc(1, 1, kTileN * PAIR, BT);
 
@@ -404,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; s++) { mbar_init(&xfull[s], 1); mbar_init(&xempty[s], 1); }
-    for (int s = 0; s < SA; s++) { mbar_init(&afull[s], kDqWarps * PAIR); mbar_init(&aempty[s], 1); }
+    for (int s = 0; s < SA; s++) { mbar_init(&afull[s], F == Fmt::W8 ? 1 : kDqWarps * PAIR); mbar_init(&aempty[s], 1); }
     for (int s = 0; s < SR; s++) {
       mbar_init(&rfull[s], 1 + (F == Fmt::Affine && a.sc_tma ? 0 : T::CP));
       mbar_init(&rempty[s], kDqWarps);
@@ -460,6 +477,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = it - SX < 0 ? 0 : it - SX; i < it; i++) mbar_wait(&xfull[i % SX], (i / SX) & 1);
     }
   } else if (warp == 2) {
+    if constexpr (F == Fmt::W8) {
+    // ------------------------------------------------------------ A producer (int8 weights)
+    // The weight tile [128 rows][128 k] lands in the A stage by one swizzled
+    // TMA copy; with a pair, both CTAs' copies complete on the leader's barrier.
+    if (lane == 0) {
+      int it = 0, t, k0, k1;
+      bool ok = true;
+      SegWalk sw(a, nk, unit, units);
+      while (ok && sw.next(t, k0, k1)) {
+        const int n0 = (t % a.Nt) * kTileN * PAIR + rank * kTileN;
+        for (int k = k0; k < k1; k++, it++) {
+          const int s = it % SA;
+          if (*abort_flag || !mbar_wait(&aempty[s], ((it / SA) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
+          if constexpr (PAIR == 2) {
+            if (leader) mbar_arrive_expect_tx(&afull[s], 2 * P::AB);
+            tma_load_2d_pair(ringA + s * P::AB, &tm_w, k * BK, n0, lead_afull + s * 8);
+          } else {
+            mbar_arrive_expect_tx(&afull[s], P::AB);
+            tma_load_2d(ringA + s * P::AB, &tm_w, k * BK, n0, &afull[s]);
+          }
+        }
+      }
+      if (leader)
+        for (int i = it - SA < 0 ? 0 : it - SA; i < it; i++) mbar_wait(&afull[i % SA], (i / SA) & 1);
+    }
+    } else {
     // ------------------------------------------------------------ R producer
     int it = 0, t, k0, k1;
     bool ok = true;
@@ -510,6 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0)
       for (int i = it - SR < 0 ? 0 : it - SR; i < it; i++) mbar_wait(&rfull[i % SR], (i / SR) & 1);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (the leader's)
     if (lane == 0 && leader) {
@@ -535,14 +579,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
             if constexpr (ATM) {
               const uint32_t at = tmem + ACOL + (uint32_t)(32 * sa + 8 * kk);
-              if constexpr (F == Fmt::I8) umma_i8_ts_pair(d, at, bd, IDESC, (k - k0) | kk);
+              if constexpr (kInt) umma_i8_ts_pair(d, at, bd, IDESC, (k - k0) | kk);
               else umma_f16_ts_pair(d, at, bd, IDESC, (k - k0) | kk);
               (void)ad;
             } else if constexpr (PAIR == 2) {
-              if constexpr (F == Fmt::I8) umma_i8_pair(d, ad, bd, IDESC, (k - k0) | kk);
+              if constexpr (kInt) umma_i8_pair(d, ad, bd, IDESC, (k - k0) | kk);
               else umma_f16_pair(d, ad, bd, IDESC, (k - k0) | kk);
             } else {
-              if constexpr (F == Fmt::I8) umma_i8(d, ad, bd, IDESC, (k - k0) | kk);
+              if constexpr (kInt) umma_i8(d, ad, bd, IDESC, (k - k0) | kk);
               else umma_f16(d, ad, bd, IDESC, (k - k0) | kk);
             }
           }
@@ -564,6 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kFirstEpi) {
     // ------------------------------------------------------------ dequantizers
+    if constexpr (F != Fmt::W8) {
     const int d = threadIdx.x - kFirstDq * 32;
     // tile row and half of the K step; with A in TMEM a warp owns the row
     // quarter its warp index may address (32 * (warp % 4) ..)
@@ -600,6 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     // Per segment: a whole tile is written out; a segment that starts inside
@@ -634,8 +680,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int row = n0 + lrow;
       float swn = 0.f;
-      if constexpr (F == Fmt::I8) swn = row < a.N ? a.sw[row] : 0.f;
-      if constexpr (ATM && F != Fmt::I8) {
+      if constexpr (kInt) swn = row < a.N ? a.sw[row] : 0.f;
+      if constexpr (ATM && !kInt) {
         if (!contrib && !head) {
           // whole tile: TMEM -> bf16 / fp16 staging, free the accumulator, then
           // write the tile row by row of tokens with 16-byte stores
@@ -689,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; j++) w[j] = __ldcg(src + j * kTileN);
 #pragma unroll
             for (int j = 0; j < 32; j++) {
-              if constexpr (F == Fmt::I8) pv[j] = (uint32_t)((int)pv[j] + (int)w[j]);
+              if constexpr (kInt) pv[j] = (uint32_t)((int)pv[j] + (int)w[j]);
               else pv[j] = __float_as_uint(__uint_as_float(pv[j]) + __uint_as_float(w[j]));
             }
           }
@@ -711,7 +757,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (vlast >= vfirst) {
 #pragma unroll
           for (int j = 0; j < 32; j++) {
-            if constexpr (F == Fmt::I8) v[j] = (uint32_t)((int)v[j] + (int)pv[j]);
+            if constexpr (kInt) v[j] = (uint32_t)((int)v[j] + (int)pv[j]);
             else v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(pv[j]));
           }
         }
@@ -721,8 +767,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int m = m0 + ch * 16 + j;
             if (m < a.M) {
               const int64_t o = (int64_t)m * a.N + row;
-              if constexpr (F == Fmt::I8) {
-                const int acc = static_cast<int>(v[j]) >> 4;   // the tensor core summed 16 * code
+              if constexpr (kInt) {
+                // I8: the tensor core summed 16 * code; W8: the codes themselves
+                const int acc = F == Fmt::I8 ? static_cast<int>(v[j]) >> 4 : static_cast<int>(v[j]);
                 if (a.acc) a.acc[o] = acc;
                 if (a.y) a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn((float)acc * (a.sx[m] * swn)));
               } else if constexpr (F == Fmt::Gptq) {
@@ -1042,6 +1089,21 @@ gwb_status launch_tc2_i8i4(const int8_t *qx, const float *sx, int64_t M, const u
                        16u, (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (s != GWB_OK) return s;
   return dispatch2<Fmt::I8, 4>(M, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
+}
+
+gwb_status launch_tc2_i8i8(const int8_t *qx, const float *sx, int64_t M, const int8_t *wq, const float *sw,
+                           int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st) {
+  Args a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = 0;
+  a.sx = sx; a.sw = sw; a.y = y; a.acc = acc;
+  CUtensorMap tw;
+  gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, (uint64_t)K, (uint64_t)N, (uint64_t)K, 128u,
+                       (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != GWB_OK) return s;
+  // a token tile no wider than the batch needs: 32 (decode), 128, or 256 on CTA pairs
+  if (M <= 32) return run_tc2<Fmt::W8, 8, 32, 1, false>(qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
+  if (M <= 128) return run_tc2<Fmt::W8, 8, 128, 1, false>(qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
+  return run_tc2<Fmt::W8, 8, 256, 2, false>(qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
 }
 
 gwb_status read_and_clear_device_error_tc2(cudaStream_t st, unsigned int *flag) {

@@ -216,6 +216,32 @@ gwb_status gwb_gemm_i8i4(const int8_t *qx, const float *sx, int64_t M, const uin
                          const float *sw, int64_t N, int64_t K, uint16_t *y, int32_t *acc,
                          void *stream);
 
+/* ------------------------------------------------------------------ W8A8 */
+
+/* qpack_sym_i8 -- symmetric per-output-channel int8 weights (qMax = 127):
+ *   sw[n] = max_k |w[n,k]| / 127;  wq[n,k] = clip(round_half_even(w / sw[n]), -127, 127)
+ * (0 when sw == 0), fp32 arithmetic.  Source: Parakeet export README of
+ * executorch PR #17234 ("Quantization Configs": 8da8w, 8-bit dynamic
+ * activations x 8-bit weights) with the per-row symmetric quantizer of QAT at
+ * bits = 8.
+ *   w fp32 [N, K] (finite), wq int8 [N, K], sw fp32 [N].  K % 16 == 0.  Bit-exact. */
+gwb_status gwb_qpack_sym_i8(const float *w, int64_t N, int64_t K, int8_t *wq, float *sw, void *stream);
+
+/* gemm_i8i8 -- int8 activations x int8 weights with int32 accumulation:
+ *   acc[m,n] = sum_k qx[m,k] * wq[n,k]                   (exact int32)
+ *   y[m,n]   = bf16_rne(fp32(acc[m,n]) * (sx[m] * sw[n]))
+ * Source: 8da8w (Parakeet export README, executorch PR #17234); scales as in
+ * gwb_gemm_i8i4.  qx, sx from gwb_quant_per_token_i8; wq, sw from
+ * gwb_qpack_sym_i8.
+ *   qx int8 [M, K], sx fp32 [M], wq int8 [N, K], sw fp32 [N]
+ *   y   bf16  [M, N] or NULL;  acc int32 [M, N] or NULL (at least one non-NULL)
+ * K % 16 == 0 (16-byte rows) and K <= 131072 (127 * 127 * K fits in int32);
+ * qx and wq 16-byte aligned (GWB_ERR_ALIGN otherwise).
+ * The int32 result is exact; y is a single rounding of its fp32 product. */
+gwb_status gwb_gemm_i8i8(const int8_t *qx, const float *sx, int64_t M, const int8_t *wq,
+                         const float *sw, int64_t N, int64_t K, uint16_t *y, int32_t *acc,
+                         void *stream);
+
 #ifdef __cplusplus
 }
 #endif

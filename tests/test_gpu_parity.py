@@ -310,6 +310,64 @@ def test_w4a8_k_tail():
     W4A8(136, 96).check(24)   # K = 96 < one 128-wide K step
 
 
+# --------------------------------------------------------------------------- W8A8
+class W8A8:
+    def __init__(self, N, K, seed=0):
+        self.N, self.K = N, K
+        w = synth.weights(N, K, seed=seed)
+        self.wq_o, self.sw_o = oracle.qpack_sym_i8(w.numpy())
+        self.wq, self.sw = gwb.qpack_sym_i8(w.to(DEV))
+        assert np.array_equal(self.wq.cpu().numpy(), self.wq_o) and np.array_equal(self.sw.cpu().numpy(), self.sw_o)
+
+    def check(self, M, seed=1):
+        x = synth.activations(M, self.K, seed=seed)
+        qx_o, sx_o = oracle.quant_per_token_i8(synth.bits16(x))
+        qx, sx = gwb.quant_per_token_i8(x.to(DEV))
+        assert np.array_equal(qx.cpu().numpy(), qx_o) and np.array_equal(sx.cpu().numpy(), sx_o)
+        y, acc = gwb.gemm_i8i8(qx, sx, self.wq, self.sw, want_y=True, want_acc=True)
+        rows = _rows(M, self.N, self.K)
+        acc_o, y_o, ovf = oracle.gemm_i8i8(qx_o, sx_o, self.wq_o, self.sw_o, self.N, self.K, rows=rows)
+        assert not ovf
+        a = acc.cpu().numpy().astype(np.int64)
+        yg = y.float().cpu().numpy()
+        if rows is not None:
+            a, yg = a[rows], yg[rows]
+        assert np.array_equal(a, acc_o), "int32 accumulators differ"
+        # y alone (no acc) must match the y written next to acc
+        y_only, none = gwb.gemm_i8i8(qx, sx, self.wq, self.sw, want_y=True, want_acc=False)
+        assert none is None and torch.equal(y_only, y)
+        max_w = float(np.max(np.abs(self.sw_o)) * 127)
+        return check_float(yg, y_o, self.K, max_w, float(x.float().abs().max()), f"w8a8 M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 8, 31, 32, 33, 100, 128, 129, 300])
+def test_w8a8_small(M):
+    W8A8(200, 384, seed=M).check(M)
+
+
+@pytest.mark.parametrize("N,K,M", [(136, 96, 24), (264, 144, 40), (72, 272, 200)])
+def test_w8a8_k_tail(N, K, M):
+    W8A8(N, K).check(M)    # K below or between 128-wide K steps
+
+
+@pytest.mark.parametrize("M", [1, 300, 512])
+def test_w8a8_stream_k_split_tiles(M):
+    # few tiles and 16 K steps each over 148 CTAs (74 pairs): tiles are split
+    W8A8(2048, 2048, seed=5).check(M)
+
+
+def test_w8a8_rejects_misaligned_and_bad_k():
+    buf = torch.zeros(4 * 256 + 16, dtype=torch.int8, device=DEV)
+    qx = buf[1:1 + 4 * 256].view(4, 256)
+    wq = torch.zeros(64, 256, dtype=torch.int8, device=DEV)
+    sx = torch.ones(4, device=DEV)
+    sw = torch.ones(64, device=DEV)
+    with pytest.raises(gwb.GwbError, match="ALIGN"):
+        gwb.gemm_i8i8(qx, sx, wq, sw)
+    with pytest.raises(gwb.GwbError, match="SHAPE"):
+        gwb.gemm_i8i8(torch.zeros(4, 72, dtype=torch.int8, device=DEV), sx, wq[:, :72].contiguous(), sw)
+
+
 @pytest.mark.parametrize("bits,M", [(4, 512), (4, 300), (8, 512)])
 def test_qmm_affine_stream_k_split_tiles(bits, M):
     # 8 x 2 tiles of 256 x 256 and 32 K steps over 74 CTA pairs: every tile is
@@ -369,6 +427,13 @@ def test_full_awq():
     a = Awq(4096, 11008, 128)
     for M in (1, 32, 1024):
         a.check_qmm(M)
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096), (4096, 14336)])
+def test_full_w8a8(N, K):
+    w = W8A8(N, K)
+    for M in (1, 64, 512, 4096):
+        w.check(M)
 
 
 @pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096), (4096, 14336)])
