@@ -681,18 +681,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = n0 + lrow;
       float swn = 0.f;
       if constexpr (kInt) swn = row < a.N ? a.sw[row] : 0.f;
-      if constexpr (ATM && !kInt) {
-        if (!contrib && !head) {
+      if constexpr (ATM) {
+        if (!contrib && !head && (!kInt || a.acc == nullptr)) {
           // whole tile: TMEM -> bf16 / fp16 staging, free the accumulator, then
           // write the tile row by row of tokens with 16-byte stores
           for (int ch = 0; ch < BT / 16; ch += 2) {
             uint32_t v0[16], v1[16];
+            float sxv[32];
+            if constexpr (kInt) {
+#pragma unroll
+              for (int j = 0; j < 32; j++) {
+                const int m = m0 + ch * 16 + j;
+                sxv[j] = m < a.M ? __ldg(a.sx + m) : 0.f;
+              }
+            }
             tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ch * 16), v0);
             tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ch * 16 + 16), v1);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; j++) {
-              const float f = __uint_as_float(j < 16 ? v0[j] : v1[j - 16]);
+              const uint32_t u = j < 16 ? v0[j] : v1[j - 16];
+              float f;
+              if constexpr (kInt) {
+                const int acc = F == Fmt::I8 ? static_cast<int>(u) >> 4 : static_cast<int>(u);
+                f = (float)acc * (sxv[j] * swn);
+              } else {
+                f = __uint_as_float(u);
+              }
               stage[(ch * 16 + j) * kTileN + lrow] = F == Fmt::Gptq ? __half_as_ushort(__float2half_rn(f))
                                                                     : __bfloat16_as_ushort(__float2bfloat16_rn(f));
             }
@@ -762,6 +777,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (row < a.N) {
+          // the chunk's token scales, loaded together before any store (the
+          // stores below could alias them as far as the compiler knows)
+          float sxv[32];
+          if constexpr (kInt) {
+#pragma unroll
+            for (int j = 0; j < 32; j++) {
+              const int m = m0 + ch * 16 + j;
+              sxv[j] = m < a.M ? __ldg(a.sx + m) : 0.f;
+            }
+          }
 #pragma unroll
           for (int j = 0; j < 32; j++) {
             const int m = m0 + ch * 16 + j;
@@ -771,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // I8: the tensor core summed 16 * code; W8: the codes themselves
                 const int acc = F == Fmt::I8 ? static_cast<int>(v[j]) >> 4 : static_cast<int>(v[j]);
                 if (a.acc) a.acc[o] = acc;
-                if (a.y) a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn((float)acc * (a.sx[m] * swn)));
+                if (a.y) a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn((float)acc * (sxv[j] * swn)));
               } else if constexpr (F == Fmt::Gptq) {
                 a.y[o] = __half_as_ushort(__float2half_rn(__uint_as_float(v[j])));
               } else {
