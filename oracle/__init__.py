@@ -66,6 +66,8 @@ def _load():
             "orc_qpack_sym_i4": (None, [_P, _I64, _I64, _P, _P, _P]),
             "orc_gemm_i8i4": (_INT, [_P, _P, _I64, _P, _I64, _P, _P, _I64, _I64, _P, _P]),
             "orc_qpack_sym_i8": (None, [_P, _I64, _I64, _P, _P]),
+            "orc_silu_mul": (None, [_P, _P, _I64, _P]),
+            "orc_qmv_silu_gate": (None, [_P, _P, _I64, _P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P]),
             "orc_gemm_i8i8": (_INT, [_P, _P, _I64, _P, _I64, _P, _P, _I64, _I64, _P, _P]),
         }
         for name, (res, args) in sig.items():
@@ -280,3 +282,31 @@ def gemm_i8i8(qx, sx, wq, sw, N, K, rows=None):
     y = np.empty((nr, N), np.float64)
     ovf = _load().orc_gemm_i8i8(_p(qx), _p(sx), M, _p(r), nr, _p(wq), _p(sw), N, K, _p(acc), _p(y))
     return acc, y, bool(ovf)
+
+
+# ----------------------------------------------------------------- fused decode products
+def silu_mul(gate_bf16, up_bf16):
+    """fp64 silu(gate) * up, elementwise, for bf16 bit patterns of equal shape."""
+    g, u = _c(gate_bf16, np.uint16), _c(up_bf16, np.uint16)
+    h = np.empty(g.shape, np.float64)
+    _load().orc_silu_mul(_p(g), _p(u), g.size, _p(h))
+    return h
+
+
+def qmv_silu_gate(gate_bf16, up_bf16, wq, scales, biases, N, K, bits, gs, resid_bf16=None, rows=None):
+    """fp64 y[len(rows) or M, N] = resid + (silu(gate) * up) . W^T (resid optional)."""
+    g, u = _c(gate_bf16, np.uint16), _c(up_bf16, np.uint16)
+    M = g.shape[0]
+    r, nr = _rows(rows, M)
+    wq, scales, biases = _c(wq, np.uint32), _c(scales, np.uint16), _c(biases, np.uint16)
+    res = None if resid_bf16 is None else _c(resid_bf16, np.uint16)
+    y = np.empty((nr, N), np.float64)
+    _load().orc_qmv_silu_gate(_p(g), _p(u), M, _p(r), nr, _p(wq), _p(scales), _p(biases), N, K, bits, gs,
+                              _p(res), _p(y))
+    return y
+
+
+def qmv_gate_up(x_bf16, gate_w, up_w, N, K, bits, gs, rows=None):
+    """(gate_y, up_y) = (x . W_gate^T, x . W_up^T) in fp64; gate_w, up_w = (wq, scales, biases)."""
+    return (qmm_affine(x_bf16, *gate_w, N, K, bits, gs, rows=rows),
+            qmm_affine(x_bf16, *up_w, N, K, bits, gs, rows=rows))

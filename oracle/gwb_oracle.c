@@ -32,6 +32,12 @@
  *           GPTQ only; AWQ uses the stored zero as is.  The same note names
  *           the AWQ reader as a sibling of identical shapes, and its g_idx
  *           remark says plain AWQ has no g_idx.
+ *   [FUSE]  metrale_gpu_runtime/mlx_int8.rs, doc comments of
+ *           MlxInt8Weight::gemv_silu_gate (y = W (silu(gate) * up), the product
+ *           never written to memory), MlxInt8Weight::gemv_silu_gate_resid
+ *           (y[n] = x_resid[n] + sum_k W[n,k] (silu(gate[k]) up[k])) and the
+ *           free function gemv_gate_up (gate_y = gate x, up_y = up x, x read
+ *           once); silu(g) = g * sigmoid(g) = g / (1 + exp(-g)).
  *   [QAT]   TinyGPT "Quantization Expansion", section 4 "QAT", "Fake-quant +
  *           STE": per-row symmetric scale = max|W|/qMax, clip(round(W/scale)),
  *           qMax = 2^(bits-1) - 1.
@@ -516,4 +522,45 @@ int orc_gemm_i8i8(const int8_t *qx, const float *sx, int64_t M, const int64_t *r
         }
     }
     return overflow;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Fused decode products [FUSE] on the MLX affine layout                    */
+/* ------------------------------------------------------------------------ */
+
+static double silu(double g) { return g / (1.0 + exp(-g)); }
+
+/* h[i] = silu(gate[i]) * up[i] in fp64, gate and up bf16 [n]. */
+void orc_silu_mul(const uint16_t *gate, const uint16_t *up, int64_t n, double *h)
+{
+    for (int64_t i = 0; i < n; i++)
+        h[i] = silu(orc_bf16_to_f64(gate[i])) * orc_bf16_to_f64(up[i]);
+}
+
+/* y[r, n] = (resid ? resid[m, n] : 0) + sum_k W[n, k] * silu(gate[m, k]) * up[m, k],
+ * m = rows[r]; gate, up bf16 [M, K], resid bf16 [M, N] or NULL; fp64
+ * throughout, W dequantized as orc_dequant_affine_f64 defines it. */
+void orc_qmv_silu_gate(const uint16_t *gate, const uint16_t *up, int64_t M, const int64_t *rows, int64_t nrows,
+                       const uint32_t *wq, const uint16_t *scales, const uint16_t *biases,
+                       int64_t N, int64_t K, int bits, int gs, const uint16_t *resid, double *y)
+{
+    int pw = per_word(bits);
+    int64_t words = K / pw;
+    int64_t G = K / gs;
+    uint32_t mask = (1u << bits) - 1u;
+    (void)M;
+    for (int64_t r = 0; r < nrows; r++) {
+        int64_t m = rows ? rows[r] : r;
+        for (int64_t n = 0; n < N; n++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                double h = silu(orc_bf16_to_f64(gate[m * K + k])) * orc_bf16_to_f64(up[m * K + k]);
+                uint32_t code = (wq[n * words + k / pw] >> ((k % pw) * bits)) & mask;
+                double sc = orc_bf16_to_f64(scales[n * G + k / gs]);
+                double b = orc_bf16_to_f64(biases[n * G + k / gs]);
+                acc += ((double)code * sc + b) * h;
+            }
+            y[r * N + n] = (resid ? orc_bf16_to_f64(resid[m * N + n]) : 0.0) + acc;
+        }
+    }
 }

@@ -485,3 +485,65 @@ def test_gemm_i8i8_integer_product_and_overflow_flag():
     acc2, _, ovf2 = oracle.gemm_i8i8(np.full((1, Kb), 127, np.int8), np.ones(1, np.float32),
                                      np.full((1, Kb), -127, np.int8), np.ones(1, np.float32), 1, Kb)
     assert ovf2 and acc2[0, 0] == -127 * 127 * Kb
+
+
+# --------------------------------------------------------------------- fused decode products
+def test_silu_mul_closed_forms():
+    """silu(g) = g * sigmoid(g): silu(0) = 0, silu(ln 3) = (3/4) ln 3, silu(-ln 3) = -(1/4) ln 3
+    (sigmoid(ln 3) = 3/4), silu(g) - silu(-g) = g for every g (sigmoid(g) + sigmoid(-g) = 1),
+    and the up factor multiplies (gate and up are not interchangeable)."""
+    ln3 = np.log(3.0)
+    g = np.array([0.0, ln3, -ln3, 2.0, -2.0, 0.5], np.float32)
+    gb = _bf16(g)
+    gv = np.array([oracle.bf16_to_f64(h) for h in gb])          # the bf16 values actually used
+    one = _bf16(np.ones_like(g))
+    h = oracle.silu_mul(gb, one)
+    assert h[0] == 0.0
+    assert np.isclose(h[1], gv[1] / (1 + 1 / np.exp(gv[1])), rtol=1e-15)
+    assert np.isclose(h[1], 0.75 * gv[1], rtol=2e-2)            # bf16(ln 3) is ln 3 to 2^-8
+    assert np.isclose(h[2], -0.25 * (-gv[2]), rtol=2e-2)
+    assert np.allclose(h[[1, 3]] - h[[2, 4]], gv[[1, 3]], rtol=1e-15, atol=0)
+    up = _bf16(np.full_like(g, -3.0))
+    assert np.allclose(oracle.silu_mul(gb, up), -3.0 * h, rtol=1e-15, atol=0)
+    # swapping gate and up changes the product: silu(2) * 1 != silu(1) * 2
+    a = oracle.silu_mul(_bf16(np.array([2.0], np.float32)), _bf16(np.array([1.0], np.float32)))
+    b = oracle.silu_mul(_bf16(np.array([1.0], np.float32)), _bf16(np.array([2.0], np.float32)))
+    assert abs(a[0] - b[0]) > 0.1
+
+
+def _identity_affine(n, bits, gs):
+    """Packed MLX weights of the n x n identity: code 1 on the diagonal, scale 1, bias 0."""
+    codes = np.eye(n, dtype=np.int32)
+    wq = oracle.pack_affine(codes, bits)
+    G = n // gs
+    return wq, _bf16(np.ones((n, G))).reshape(n, G), _bf16(np.zeros((n, G))).reshape(n, G)
+
+
+def test_qmv_silu_gate_identity_weight_and_residual():
+    """With W = I, y[t, n] = silu(gate[t, n]) * up[t, n] exactly (pins the elementwise product and
+    the [out, in] orientation); the residual adds resid[t, n] to every output."""
+    n, bits, gs = 64, 4, 32
+    wq, sc, bi = _identity_affine(n, bits, gs)
+    rng = np.random.default_rng(7)
+    gate = _bf16(rng.standard_normal((3, n)).astype(np.float32) * 2).reshape(3, n)
+    up = _bf16(rng.standard_normal((3, n)).astype(np.float32)).reshape(3, n)
+    y = oracle.qmv_silu_gate(gate, up, wq, sc, bi, n, n, bits, gs)
+    assert np.array_equal(y, oracle.silu_mul(gate, up))
+    res = _bf16(rng.standard_normal((3, n)).astype(np.float32)).reshape(3, n)
+    yr = oracle.qmv_silu_gate(gate, up, wq, sc, bi, n, n, bits, gs, resid_bf16=res)
+    rv = np.array([[oracle.bf16_to_f64(h) for h in row] for row in res])
+    assert np.allclose(yr - y, rv, rtol=0, atol=1e-12)
+
+
+def test_qmv_silu_gate_is_matmul_of_silu_product():
+    """A general weight: y = (silu(gate) * up) . W^T (numpy matmul on the oracle's dequantized W),
+    for two row samples."""
+    N, K, bits, gs = 24, 128, 8, 64
+    w = synth.weights(N, K, seed=17).numpy()
+    wq, sc, bi, _ = oracle.qpack_affine(w, bits, gs)
+    rng = np.random.default_rng(8)
+    gate = _bf16(rng.standard_normal((4, K)).astype(np.float32)).reshape(4, K)
+    up = _bf16(rng.standard_normal((4, K)).astype(np.float32)).reshape(4, K)
+    W = oracle.dequant_affine_f64(wq, sc, bi, N, K, bits, gs)
+    y = oracle.qmv_silu_gate(gate, up, wq, sc, bi, N, K, bits, gs, rows=[3, 1])
+    assert np.allclose(y, oracle.silu_mul(gate, up)[[3, 1]] @ W.T, rtol=1e-12, atol=1e-14)
