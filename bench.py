@@ -494,6 +494,28 @@ def run_layer(args):
         def launch(i):
             wq, sc, bi = sets[i % 2]
             gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+    elif args.fmt in ("gate_up", "silu_resid"):
+        sets = []
+        for s in range(2):
+            ws = []
+            for j in range(2 if args.fmt == "gate_up" else 1):
+                g = torch.Generator(device=dev)
+                g.manual_seed(10 * s + j)
+                w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+                ws.append(gwb.qpack_affine(w, bits, GS))
+                del w
+            sets.append(ws)
+        x = synth.activations(M, K, seed=1).to(dev)
+        x2 = synth.activations(M, K, seed=2).to(dev)
+        res = synth.activations(M, N, seed=3).to(dev)
+        y2 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+        def launch(i):
+            ws = sets[i % 2]
+            if args.fmt == "gate_up":
+                gwb.gemv_gate_up(x, ws[0], ws[1], bits, GS, y_gate=y, y_up=y2)
+            else:
+                gwb.gemv_silu_gate(x, x2, *ws[0], bits, GS, x_resid=res, y=y)
     else:
         sets = [int8_operands(gwb, dev, args.fmt, N, K, M, seed=s) for s in range(2)]
         gemm = int8_gemm(gwb, args.fmt)
@@ -523,6 +545,10 @@ def run_layer(args):
     us = a.elapsed_time(b) * 1e3 / (20 * args.steps)
     if args.fmt == "affine":
         nbytes = gemv_bytes(N, K, bits, M=M) if M <= 8 else None
+    elif args.fmt == "gate_up":
+        nbytes = 2 * gemv_bytes(N, K, bits, M=M) - 2 * M * K      # x is read once
+    elif args.fmt == "silu_resid":
+        nbytes = gemv_bytes(N, K, bits, M=M) + 2 * M * K + 2 * M * N   # up and the residual
     else:
         nbytes = (N * K * bits // 8 + N * 4 + M * K + M * 4 + M * N * 2) if M <= 8 else None
     out = {"layer": {"fmt": args.fmt, "N": N, "K": K, "bits": bits, "group_size": GS, "M": M},
@@ -541,7 +567,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["gwb", "reference"], default="gwb")
     ap.add_argument("--no-prefill", action="store_true")
-    ap.add_argument("--fmt", choices=["affine", "w4a8", "w8a8"], default="affine",
+    ap.add_argument("--fmt", choices=["affine", "w4a8", "w8a8", "gate_up", "silu_resid"], default="affine",
                     help="--layer: weight format (affine: MLX group-wise, bits from --layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

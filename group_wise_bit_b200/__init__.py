@@ -31,6 +31,9 @@ SIGNATURES = {
     "gwb_qmm_affine_noalloc": [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P],
     "gwb_gptq_dequant": [_P, _P, _P, _P, _I64, _I64, _INT, _P, _P],
     "gwb_gptq_qmm": [_P, _I64, _P, _P, _P, _P, _I64, _I64, _INT, _P, _P],
+    "gwb_gemv_gate_up": [_P, _I64, _P, _P, _P, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P, _P],
+    "gwb_gemv_silu_gate": [_P, _P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P],
+    "gwb_gemv_silu_gate_resid": [_P, _P, _I64, _P, _P, _P, _I64, _I64, _INT, _INT, _P, _P, _P],
     "gwb_awq_dequant": [_P, _P, _P, _I64, _I64, _INT, _P, _P],
     "gwb_awq_qmm": [_P, _I64, _P, _P, _P, _I64, _I64, _INT, _P, _P],
     "gwb_quant_per_token_i8": [_P, _I64, _I64, _P, _P, _P],
@@ -137,6 +140,15 @@ def dequant_affine(wq, scales, biases, K, bits, group_size, out=None):
     return out
 
 
+def _affine_check(wq, scales, biases, bits, group_size):
+    """(N, K) of a weight in the MLX affine layout, its three tensors checked."""
+    _dev(wq, "wq", _WORDS)
+    N, K = wq.shape[0], wq.shape[1] * 32 // bits
+    _dev(scales, "scales", (torch.bfloat16,), (N, K // group_size))
+    _dev(biases, "biases", (torch.bfloat16,), (N, K // group_size))
+    return N, K
+
+
 def qmm_affine(x, wq, scales, biases, bits, group_size, y=None):
     """y bf16 [M, N] = x bf16 [M, K] . W^T with W in the MLX affine layout."""
     _dev(x, "x", (torch.bfloat16,))
@@ -196,6 +208,40 @@ def gptq_qmm(x, qweight, scales, qzeros, g_idx, group_size, y=None):
     y = _out(y, "y", (M, N), torch.float16, x.device)
     _call("gwb_gptq_qmm", _ptr(x), M, _ptr(qweight), _ptr(scales), _ptr(qzeros), _ptr(g_idx), K, N, group_size,
           _ptr(y), _stream())
+    return y
+
+
+# ------------------------------------------------------------------ fused decode products
+def gemv_gate_up(x, gate_w, up_w, bits, group_size, y_gate=None, y_up=None):
+    """(x W_gate^T, x W_up^T) in one launch; gate_w / up_w = (wq, scales, biases) of one shape."""
+    wq, sc, bi = gate_w
+    wq2, sc2, bi2 = up_w
+    N, K = _affine_check(wq, sc, bi, bits, group_size)
+    if _affine_check(wq2, sc2, bi2, bits, group_size) != (N, K):
+        raise ValueError("gate and up weights differ in shape")
+    _dev(x, "x", (torch.bfloat16,), (x.shape[0], K))
+    M = x.shape[0]
+    y_gate = _out(y_gate, "y_gate", (M, N), torch.bfloat16, x.device)
+    y_up = _out(y_up, "y_up", (M, N), torch.bfloat16, x.device)
+    _call("gwb_gemv_gate_up", _ptr(x), M, _ptr(wq), _ptr(sc), _ptr(bi), _ptr(wq2), _ptr(sc2), _ptr(bi2), N, K,
+          bits, group_size, _ptr(y_gate), _ptr(y_up), _stream())
+    return y_gate, y_up
+
+
+def gemv_silu_gate(gate, up, wq, scales, biases, bits, group_size, x_resid=None, y=None):
+    """y = (x_resid +) (silu(gate) * up) W^T; gate, up bf16 [M, K], x_resid bf16 [M, N]."""
+    N, K = _affine_check(wq, scales, biases, bits, group_size)
+    _dev(gate, "gate", (torch.bfloat16,), (gate.shape[0], K))
+    M = gate.shape[0]
+    _dev(up, "up", (torch.bfloat16,), (M, K))
+    y = _out(y, "y", (M, N), torch.bfloat16, gate.device)
+    if x_resid is None:
+        _call("gwb_gemv_silu_gate", _ptr(gate), _ptr(up), M, _ptr(wq), _ptr(scales), _ptr(biases), N, K, bits,
+              group_size, _ptr(y), _stream())
+    else:
+        _dev(x_resid, "x_resid", (torch.bfloat16,), (M, N))
+        _call("gwb_gemv_silu_gate_resid", _ptr(gate), _ptr(up), M, _ptr(wq), _ptr(scales), _ptr(biases), N, K,
+              bits, group_size, _ptr(x_resid), _ptr(y), _stream())
     return y
 
 

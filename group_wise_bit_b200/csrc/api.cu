@@ -82,13 +82,15 @@ const char *gwb_last_error(void) { return gwb::g_msg; }
 const char *gwb_version(void) { return "group_wise_bit_b200 0.1 (sm_100a)"; }
 
 gwb_status gwb_check_device_error(void *stream) {
-  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0, flag5 = 0;
+  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0, flag5 = 0, flag6 = 0, flag7 = 0;
   GWB_TRY(gwb::read_and_clear_device_error(as_stream(stream), &flag));
   GWB_TRY(gwb::read_and_clear_device_error_stream(as_stream(stream), &flag2));
   GWB_TRY(gwb::read_and_clear_device_error_tmem(as_stream(stream), &flag3));
   GWB_TRY(gwb::read_and_clear_device_error_pipe(as_stream(stream), &flag4));
   GWB_TRY(gwb::read_and_clear_device_error_tc2(as_stream(stream), &flag5));
-  flag |= flag2 | flag3 | flag4 | flag5;
+  GWB_TRY(gwb::read_and_clear_device_error_gate_up(as_stream(stream), &flag6));
+  GWB_TRY(gwb::read_and_clear_device_error_silu(as_stream(stream), &flag7));
+  flag |= flag2 | flag3 | flag4 | flag5 | flag6 | flag7;
   if (flag) return fail(GWB_ERR_TIMEOUT, "a bounded device-side wait gave up (flag 0x%x)", flag);
   return GWB_OK;
 }
@@ -130,6 +132,7 @@ gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, cons
   GWB_TRY(need(wq, "wq"));
   GWB_TRY(need(scales, "scales"));
   GWB_TRY(need(biases, "biases"));
+  if (!aligned16(x)) return fail(GWB_ERR_ALIGN, "x is not 16-byte aligned");
   if (M <= 8 && gwb::gemv_affine_supported(bits, group_size)) {
     gwb_status s =
         gwb::launch_gemv_pipe(x, (int)M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
@@ -146,6 +149,90 @@ gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, cons
     if (s != GWB_ERR_UNSUPPORTED) return s;
   }
   return gwb::launch_tc_affine(x, M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
+}
+
+namespace {
+
+// Checks shared by the fused decode products: the affine layout, 1 <= M <= 8
+// tokens, and 16-byte aligned activation and output rows.
+gwb_status check_fused(int64_t M, int64_t N, int64_t K, int bits, int group_size) {
+  GWB_TRY(check_layout(N, K, bits, group_size));
+  if (M < 0) return fail(GWB_ERR_INVALID_ARG, "negative M=%lld", (long long)M);
+  if (M > 8) return fail(GWB_ERR_SHAPE, "fused decode products take at most 8 tokens (M=%lld)", (long long)M);
+  return GWB_OK;
+}
+
+gwb_status fused_unsupported(const char *what, int64_t K, int group_size) {
+  return fail(GWB_ERR_UNSUPPORTED, "%s needs K/group_size to be a multiple of 8 (K=%lld, group_size=%d)", what,
+              (long long)K, group_size);
+}
+
+}  // namespace
+
+gwb_status gwb_gemv_gate_up(const uint16_t *x, int64_t M, const uint32_t *wq_gate, const uint16_t *scales_gate,
+                            const uint16_t *biases_gate, const uint32_t *wq_up, const uint16_t *scales_up,
+                            const uint16_t *biases_up, int64_t N, int64_t K, int bits, int group_size,
+                            uint16_t *y_gate, uint16_t *y_up, void *stream) {
+  GWB_TRY(check_fused(M, N, K, bits, group_size));
+  if (M == 0 || N == 0) return GWB_OK;
+  GWB_TRY(need(y_gate, "y_gate"));
+  GWB_TRY(need(y_up, "y_up"));
+  if (K == 0) {
+    GWB_TRY(zero_fill(y_gate, (size_t)M * N * 2, stream));
+    return zero_fill(y_up, (size_t)M * N * 2, stream);
+  }
+  GWB_TRY(need(x, "x"));
+  GWB_TRY(need(wq_gate, "wq_gate"));
+  GWB_TRY(need(scales_gate, "scales_gate"));
+  GWB_TRY(need(biases_gate, "biases_gate"));
+  GWB_TRY(need(wq_up, "wq_up"));
+  GWB_TRY(need(scales_up, "scales_up"));
+  GWB_TRY(need(biases_up, "biases_up"));
+  if (!aligned16(x)) return fail(GWB_ERR_ALIGN, "x is not 16-byte aligned");
+  const gwb_status s = gwb::launch_gemv_gate_up(x, (int)M, wq_gate, scales_gate, biases_gate, wq_up, scales_up,
+                                                biases_up, N, K, bits, group_size, y_gate, y_up, as_stream(stream));
+  return s == GWB_ERR_UNSUPPORTED ? fused_unsupported("gemv_gate_up", K, group_size) : s;
+}
+
+namespace {
+
+gwb_status silu_gate_impl(const uint16_t *gate, const uint16_t *up, int64_t M, const uint32_t *wq,
+                          const uint16_t *scales, const uint16_t *biases, int64_t N, int64_t K, int bits,
+                          int group_size, const uint16_t *x_resid, uint16_t *y, void *stream, const char *what) {
+  GWB_TRY(check_fused(M, N, K, bits, group_size));
+  if (M == 0 || N == 0) return GWB_OK;
+  GWB_TRY(need(y, "y"));
+  if (K == 0) {
+    if (!x_resid) return zero_fill(y, (size_t)M * N * 2, stream);
+    const cudaError_t e = cudaMemcpyAsync(y, x_resid, (size_t)M * N * 2, cudaMemcpyDeviceToDevice, as_stream(stream));
+    return e == cudaSuccess ? GWB_OK : fail(GWB_ERR_CUDA, "cudaMemcpyAsync: %s", cudaGetErrorString(e));
+  }
+  GWB_TRY(need(gate, "gate"));
+  GWB_TRY(need(up, "up"));
+  GWB_TRY(need(wq, "wq"));
+  GWB_TRY(need(scales, "scales"));
+  GWB_TRY(need(biases, "biases"));
+  if (!aligned16(gate) || !aligned16(up)) return fail(GWB_ERR_ALIGN, "gate and up must be 16-byte aligned");
+  const gwb_status s = gwb::launch_gemv_silu_gate(gate, up, (int)M, wq, scales, biases, N, K, bits, group_size,
+                                                  x_resid, y, as_stream(stream));
+  return s == GWB_ERR_UNSUPPORTED ? fused_unsupported(what, K, group_size) : s;
+}
+
+}  // namespace
+
+gwb_status gwb_gemv_silu_gate(const uint16_t *gate, const uint16_t *up, int64_t M, const uint32_t *wq,
+                              const uint16_t *scales, const uint16_t *biases, int64_t N, int64_t K, int bits,
+                              int group_size, uint16_t *y, void *stream) {
+  return silu_gate_impl(gate, up, M, wq, scales, biases, N, K, bits, group_size, nullptr, y, stream,
+                        "gemv_silu_gate");
+}
+
+gwb_status gwb_gemv_silu_gate_resid(const uint16_t *gate, const uint16_t *up, int64_t M, const uint32_t *wq,
+                                    const uint16_t *scales, const uint16_t *biases, int64_t N, int64_t K, int bits,
+                                    int group_size, const uint16_t *x_resid, uint16_t *y, void *stream) {
+  if (M > 0 && N > 0) GWB_TRY(need(x_resid, "x_resid"));
+  return silu_gate_impl(gate, up, M, wq, scales, biases, N, K, bits, group_size, x_resid, y, stream,
+                        "gemv_silu_gate_resid");
 }
 
 gwb_status gwb_qmm_affine_noalloc(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,

@@ -49,6 +49,15 @@ gwb_status launch_gemv_pipe(const uint16_t *x, int M, const uint32_t *wq, const 
                             const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
                             cudaStream_t st);
 gwb_status read_and_clear_device_error_pipe(cudaStream_t st, unsigned int *flag);
+gwb_status read_and_clear_device_error_gate_up(cudaStream_t st, unsigned int *flag);
+gwb_status read_and_clear_device_error_silu(cudaStream_t st, unsigned int *flag);
+gwb_status launch_gemv_gate_up(const uint16_t *x, int M, const uint32_t *wq_gate, const uint16_t *sc_gate,
+                               const uint16_t *bi_gate, const uint32_t *wq_up, const uint16_t *sc_up,
+                               const uint16_t *bi_up, int64_t N, int64_t K, int bits, int gs, uint16_t *y_gate,
+                               uint16_t *y_up, cudaStream_t st);
+gwb_status launch_gemv_silu_gate(const uint16_t *gate, const uint16_t *up, int M, const uint32_t *wq,
+                                 const uint16_t *scales, const uint16_t *biases, int64_t N, int64_t K, int bits,
+                                 int gs, const uint16_t *resid, uint16_t *y, cudaStream_t st);
 // TMEM-operand tensor-core GEMV (the main decode kernel); GWB_ERR_UNSUPPORTED
 // (without a message) when the layout is outside what it covers.
 gwb_status launch_gemv_tmem(const uint16_t *x, int M, const uint32_t *wq, const uint16_t *scales,

@@ -173,6 +173,41 @@ gwb_status gwb_gptq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, co
                         const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N,
                         int group_size, uint16_t *y, void *stream);
 
+/* ------------------------------------------------------- fused decode products
+ * Source: metrale_gpu_runtime/mlx_int8.rs, the free function gemv_gate_up and
+ * MlxInt8Weight::gemv_silu_gate / gemv_silu_gate_resid (decode-time MLP fusion
+ * for MLX affine weights).  Every weight is in the layout of gwb_qmm_affine
+ * (wq u32 [N, K*bits/32], scales and biases bf16 [N, K/group_size]); vectors
+ * are bf16 rows of 1 <= M <= 8 tokens, 16-byte aligned.  K/group_size must be a
+ * multiple of 8 (GWB_ERR_UNSUPPORTED otherwise).  Float results: fp32
+ * accumulation, one rounding to bf16, within the tolerance of gwb_qmm_affine.
+ * M > 8 is GWB_ERR_SHAPE: these are single-token products.
+ *
+ * gemv_gate_up -- y_gate = x W_gate^T and y_up = x W_up^T in one launch; the
+ * two weights share N, K, bits and group_size.
+ *   x bf16 [M, K];  y_gate, y_up bf16 [M, N]. */
+gwb_status gwb_gemv_gate_up(const uint16_t *x, int64_t M, const uint32_t *wq_gate,
+                            const uint16_t *scales_gate, const uint16_t *biases_gate,
+                            const uint32_t *wq_up, const uint16_t *scales_up,
+                            const uint16_t *biases_up, int64_t N, int64_t K, int bits, int group_size,
+                            uint16_t *y_gate, uint16_t *y_up, void *stream);
+
+/* gemv_silu_gate -- y = (silu(gate) * up) W^T, silu(g) = g / (1 + exp(-g)); the
+ * product silu(gate) * up is formed in fp32 and never written to memory.
+ *   gate, up bf16 [M, K];  y bf16 [M, N]. */
+gwb_status gwb_gemv_silu_gate(const uint16_t *gate, const uint16_t *up, int64_t M, const uint32_t *wq,
+                              const uint16_t *scales, const uint16_t *biases, int64_t N, int64_t K,
+                              int bits, int group_size, uint16_t *y, void *stream);
+
+/* gemv_silu_gate_resid -- y = x_resid + (silu(gate) * up) W^T, the residual
+ * added to the fp32 sum before its rounding.  x_resid bf16 [M, N] (non-NULL;
+ * it may be y itself: each element is read before it is written). */
+gwb_status gwb_gemv_silu_gate_resid(const uint16_t *gate, const uint16_t *up, int64_t M,
+                                    const uint32_t *wq, const uint16_t *scales,
+                                    const uint16_t *biases, int64_t N, int64_t K, int bits,
+                                    int group_size, const uint16_t *x_resid, uint16_t *y,
+                                    void *stream);
+
 /* awq_dequant / awq_qmm -- the same layout and shapes as gwb_gptq_dequant /
  * gwb_gptq_qmm, with the zero taken as stored: zero = (qzeros[g, o/8] >> ((o%8)*4)) & 0xF,
  * no "+1", and no g_idx (g = i / group_size).

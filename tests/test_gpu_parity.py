@@ -221,6 +221,77 @@ def test_gptq_qmm_small(permuted, M):
     Gptq(384, 264, 128 if M % 2 else 64, permuted, seed=M).check_qmm(M)
 
 
+# --------------------------------------------------------------------------- fused decode products
+def _gate_up_case(N, K, bits, gs, M, seed):
+    g = Affine(N, K, bits, gs, seed=seed)
+    u = Affine(N, K, bits, gs, seed=seed + 1)
+    x = synth.activations(M, K, seed=seed + 2, outlier_frac=0.01)
+    yg, yu = gwb.gemv_gate_up(x.to(DEV), (g.wq, g.sc, g.bi), (u.wq, u.sc, u.bi), bits, gs)
+    rows = _rows(M, N, K)
+    rg, ru = oracle.qmv_gate_up(synth.bits16(x), (g.wq_o, g.sc_o, g.bi_o), (u.wq_o, u.sc_o, u.bi_o), N, K, bits, gs,
+                                rows=rows)
+    max_x = float(x.float().abs().max())
+    for y, ref, w, name in ((yg, rg, g, "gate"), (yu, ru, u, "up")):
+        yy = y.float().cpu().numpy()
+        if rows is not None:
+            yy = yy[rows]
+        check_float(yy, ref, K, w.max_w, max_x, f"gate_up {name} {N}x{K} b{bits} gs{gs} M={M}")
+
+
+@pytest.mark.parametrize("bits,gs", [(8, 64), (8, 32), (4, 64), (4, 128), (2, 64)])
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_gemv_gate_up(bits, gs, M):
+    _gate_up_case(200, 1024, bits, gs, M, seed=bits + M)      # ragged last strip of each weight
+
+
+@pytest.mark.parametrize("N,K", [(64, 8192), (48, 2048), (1000, 512)])
+def test_gemv_gate_up_split_layouts(N, K):
+    # few strips: K split over a cluster; many short strips: strips shared by warps
+    _gate_up_case(N, K, 8, 64, 2, seed=N)
+
+
+def _silu_case(N, K, bits, gs, M, seed, resid=False, alias=False):
+    a = Affine(N, K, bits, gs, seed=seed)
+    gate = (synth.activations(M, K, seed=seed + 1) * 4).to(torch.bfloat16)
+    up = synth.activations(M, K, seed=seed + 2, outlier_frac=0.01)
+    res = synth.activations(M, N, seed=seed + 3) if resid else None
+    dres = res.to(DEV) if resid else None
+    y = gwb.gemv_silu_gate(gate.to(DEV), up.to(DEV), a.wq, a.sc, a.bi, bits, gs, x_resid=dres,
+                           y=dres if alias else None)
+    rows = _rows(M, N, K)
+    ref = oracle.qmv_silu_gate(synth.bits16(gate), synth.bits16(up), a.wq_o, a.sc_o, a.bi_o, N, K, bits, gs,
+                               resid_bf16=synth.bits16(res) if resid else None, rows=rows)
+    yy = y.float().cpu().numpy()
+    if rows is not None:
+        yy = yy[rows]
+    max_x = float(np.abs(oracle.silu_mul(synth.bits16(gate), synth.bits16(up))).max())
+    return check_float(yy, ref, K, a.max_w, max_x, f"silu_gate {N}x{K} b{bits} gs{gs} M={M} resid={resid}")
+
+
+@pytest.mark.parametrize("bits,gs", [(8, 64), (4, 64), (4, 128), (2, 128)])
+@pytest.mark.parametrize("M", [1, 2, 5, 8])
+@pytest.mark.parametrize("resid", [False, True])
+def test_gemv_silu_gate(bits, gs, M, resid):
+    _silu_case(136, 2048, bits, gs, M, seed=bits * 7 + M, resid=resid)
+
+
+def test_gemv_silu_gate_resid_in_place():
+    _silu_case(256, 1024, 8, 64, 4, seed=3, resid=True, alias=True)   # x_resid is y
+
+
+def test_fused_decode_argument_errors():
+    a = Affine(64, 384, 4, 64, seed=1)                 # K / gs = 6: not a multiple of 8
+    x = torch.zeros(1, 384, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(gwb.GwbError, match="UNSUPPORTED"):
+        gwb.gemv_silu_gate(x, x, a.wq, a.sc, a.bi, 4, 64)
+    b = Affine(64, 512, 4, 64, seed=2)
+    x9 = torch.zeros(9, 512, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(gwb.GwbError, match="SHAPE"):
+        gwb.gemv_gate_up(x9, (b.wq, b.sc, b.bi), (b.wq, b.sc, b.bi), 4, 64)
+    y0g, y0u = gwb.gemv_gate_up(x9[:0], (b.wq, b.sc, b.bi), (b.wq, b.sc, b.bi), 4, 64)
+    assert y0g.shape == (0, 64) and y0u.shape == (0, 64)
+
+
 # --------------------------------------------------------------------------- AWQ zero convention
 class Awq:
     """The GPTQ tensors without g_idx, the stored zero used as is."""
@@ -427,6 +498,14 @@ def test_full_awq():
     a = Awq(4096, 11008, 128)
     for M in (1, 32, 1024):
         a.check_qmm(M)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_full_decode_mlp_fused(bits):
+    # Llama-3-8B MLP at decode: gate/up 14336 x 4096 and down 4096 x 14336 with the residual
+    for M in (1, 4):
+        _gate_up_case(14336, 4096, bits, 64, M, seed=40 + M)
+        _silu_case(4096, 14336, bits, 64, M, seed=50 + M, resid=True)
 
 
 @pytest.mark.parametrize("N,K", [(4096, 4096), (14336, 4096), (4096, 14336)])
