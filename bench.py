@@ -264,6 +264,7 @@ def run_gpu(args, world, rank, local):
 
     prefill = run_prefill(gwb, dev, stream, bf16_peak, peak_kind) if not args.no_prefill else None
     int8 = {}
+    int8["decode_mlp_fused"] = run_mlp_fused(gwb, dev, stream, hbm_peak)
     if not args.no_prefill:
         i8peak = int8_peak_tops(dev, stream)
         int8["w4a8_m4096"] = run_int8(gwb, dev, stream, "w4a8", 14336, 4096, 4096, i8peak, hbm_peak)
@@ -368,7 +369,8 @@ def run_int8(gwb, dev, stream, fmt, N, K, M, int8_peak, hbm_peak, reps=5):
         out.update({"value": round(tops, 1), "unit": "TOP/s",
                     "roofline": {"kernel": kern, "bound": "tensor", "achieved": round(tops, 1),
                                  "peak": round(int8_peak, 1), "unit": "TOP/s", "frac": round(tops / int8_peak, 4),
-                                 "peak_source": "measured in this run: torch._int_mm 8192^3 int8, best of 5"}})
+                                 "peak_source": "measured in this run: torch._int_mm 8192^3 int8, best of 5",
+                                 "traffic": traffic_for(f"k_tc2_{fmt}_m{M}")}})
     return out
 
 
@@ -408,6 +410,56 @@ def run_prefill(gwb, dev, stream, bf16_peak, peak_kind, reps=5):
                          "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(tf / bf16_peak, 4),
                          "peak_source": peak_kind, "traffic": traffic_for("k_tc2_affine4_m2048")},
             "shapes": per}
+
+
+def run_mlp_fused(gwb, dev, stream, hbm_peak, bits=4, M=1, reps=20):
+    """Decode MLP of a Llama-3-8B layer (hidden 4096, intermediate 14336, MLX affine gs 64) through
+    the fused products: gemv_gate_up, then gemv_silu_gate_resid.  One CUDA graph of `reps` MLPs
+    alternating two weight sets (> L2), timed by events around its replay."""
+    H, I = 4096, 14336
+    sets = []
+    for s_ in range(2):
+        ws = []
+        for j, (n, k) in enumerate(((I, H), (I, H), (H, I))):
+            g = torch.Generator(device=dev)
+            g.manual_seed(500 + 10 * s_ + j)
+            w = torch.randn((n, k), generator=g, device=dev, dtype=torch.float32) * 0.02
+            ws.append(gwb.qpack_affine(w, bits, GS))
+            del w
+        sets.append(ws)
+    x = synth.activations(M, H, seed=1).to(dev)
+    gate = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
+    up = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+
+    def mlp(i):
+        wg, wu, wd = sets[i % 2]
+        gwb.gemv_gate_up(x, wg, wu, bits, GS, y_gate=gate, y_up=up)
+        gwb.gemv_silu_gate(gate, up, *wd, bits, GS, x_resid=x, y=y)
+
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            mlp(i)
+        stream.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for i in range(reps):
+                mlp(i)
+        gr.replay()
+        stream.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        gr.replay()
+        b.record(stream)
+        b.synchronize()
+    us = a.elapsed_time(b) * 1e3 / reps
+    nbytes = (2 * gemv_bytes(I, H, bits, M=M) - 2 * M * H) + (gemv_bytes(H, I, bits, M=M) + 2 * M * I + 2 * M * H)
+    gbs = nbytes / us / 1e3
+    return {"value": round(gbs, 1), "unit": "GB/s", "M": M, "bits": bits, "group_size": GS,
+            "us_per_mlp": round(us, 2), "bytes_per_mlp": nbytes, "launches_per_mlp": 2,
+            "roofline": {"kernel": "k_gemv_pipe<dual> + k_gemv_pipe<silu> (Llama-3-8B MLP, hidden 4096)",
+                         "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4), "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}}
 
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
