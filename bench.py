@@ -265,6 +265,7 @@ def run_gpu(args, world, rank, local):
     prefill = run_prefill(gwb, dev, stream, bf16_peak, peak_kind) if not args.no_prefill else None
     int8 = {}
     int8["decode_mlp_fused"] = run_mlp_fused(gwb, dev, stream, hbm_peak)
+    int8["w4a8_decode_fused"] = run_w4a8_decode(gwb, dev, stream, hbm_peak)
     if not args.no_prefill:
         i8peak = int8_peak_tops(dev, stream)
         int8["w4a8_m4096"] = run_int8(gwb, dev, stream, "w4a8", 14336, 4096, 4096, i8peak, hbm_peak)
@@ -410,6 +411,52 @@ def run_prefill(gwb, dev, stream, bf16_peak, peak_kind, reps=5):
                          "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(tf / bf16_peak, 4),
                          "peak_source": peak_kind, "traffic": traffic_for("k_tc2_affine4_m2048")},
             "shapes": per}
+
+
+def run_w4a8_decode(gwb, dev, stream, hbm_peak, N=14336, K=4096, M=1, reps=20):
+    """W4A8 at decode: the fused product (activations quantized inside the kernel) against the
+    two-launch path (quant_per_token_i8, then gemm_i8i4), each a CUDA graph of `reps` launches
+    alternating two weight sets (> L2)."""
+    sets = [int8_operands(gwb, dev, "w4a8", N, K, M, seed=s_) for s_ in range(2)]
+    x = synth.activations(M, K, seed=1).to(dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    qx = torch.empty((M, K), dtype=torch.int8, device=dev)
+    sx = torch.empty((M,), dtype=torch.float32, device=dev)
+
+    def fused(i):
+        wq, sw, _, _ = sets[i % 2]
+        gwb.gemv_w4a8(x, wq, sw, y=y)
+
+    def two(i):
+        wq, sw, _, _ = sets[i % 2]
+        gwb.quant_per_token_i8(x, qx=qx, sx=sx)
+        gwb.gemm_i8i4(qx, sx, wq, sw, y=y)
+
+    out = {}
+    for name, fn in (("fused", fused), ("two_launch", two)):
+        with torch.cuda.stream(stream):
+            for i in range(2):
+                fn(i)
+            stream.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for i in range(reps):
+                    fn(i)
+            gr.replay()
+            stream.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            gr.replay()
+            b.record(stream)
+            b.synchronize()
+        out[name] = a.elapsed_time(b) * 1e3 / reps
+    nbytes = N * K // 2 + N * 4 + 2 * M * K + 2 * M * N
+    gbs = nbytes / out["fused"] / 1e3
+    return {"value": round(gbs, 1), "unit": "GB/s", "N": N, "K": K, "M": M,
+            "us_fused": round(out["fused"], 2), "us_two_launch": round(out["two_launch"], 2),
+            "roofline": {"kernel": "k_gemv_pipe<4,64,1,w4a8> (per-token int8 quantization inside)", "bound": "hbm",
+                         "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
+                         "bytes_per_launch": nbytes, "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}}
 
 
 def run_mlp_fused(gwb, dev, stream, hbm_peak, bits=4, M=1, reps=20):

@@ -39,6 +39,7 @@ SIGNATURES = {
     "gwb_quant_per_token_i8": [_P, _I64, _I64, _P, _P, _P],
     "gwb_qpack_sym_i4": [_P, _I64, _I64, _P, _P, _P],
     "gwb_gemm_i8i4": [_P, _P, _I64, _P, _P, _I64, _I64, _P, _P, _P],
+    "gwb_gemv_w4a8": [_P, _I64, _P, _P, _I64, _I64, _P, _P],
     "gwb_qpack_sym_i8": [_P, _I64, _I64, _P, _P, _P],
     "gwb_gemm_i8i8": [_P, _P, _I64, _P, _P, _I64, _I64, _P, _P, _P],
     "gwb_check_device_error": [_P],
@@ -300,6 +301,19 @@ def gemm_i8i4(qx, sx, wq, sw, want_y=True, want_acc=False, y=None, acc=None):
         acc = _out(acc, "acc", (M, N), torch.int32, qx.device)
     _call("gwb_gemm_i8i4", _ptr(qx), _ptr(sx), M, _ptr(wq), _ptr(sw), N, K, _ptr(y), _ptr(acc), _stream())
     return y, acc
+
+
+def gemv_w4a8(x, wq, sw, y=None):
+    """y bf16 [M, N] = W4A8 product of x bf16 [M, K] (quantized per token inside the kernel, M <= 8)
+    and the int4 weights (wq, sw) of qpack_sym_i4; bit-identical to quant_per_token_i8 + gemm_i8i4."""
+    _dev(x, "x", (torch.bfloat16,))
+    M, K = x.shape
+    N = wq.shape[0]
+    _dev(wq, "wq", _WORDS, (N, K // 8))
+    _dev(sw, "sw", (torch.float32,), (N,))
+    y = _out(y, "y", (M, N), torch.bfloat16, x.device)
+    _call("gwb_gemv_w4a8", _ptr(x), M, _ptr(wq), _ptr(sw), N, K, _ptr(y), _stream())
+    return y
 
 
 # ------------------------------------------------------------------ W8A8

@@ -82,7 +82,7 @@ const char *gwb_last_error(void) { return gwb::g_msg; }
 const char *gwb_version(void) { return "group_wise_bit_b200 0.1 (sm_100a)"; }
 
 gwb_status gwb_check_device_error(void *stream) {
-  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0, flag5 = 0, flag6 = 0, flag7 = 0;
+  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0, flag5 = 0, flag6 = 0, flag7 = 0, flag8 = 0;
   GWB_TRY(gwb::read_and_clear_device_error(as_stream(stream), &flag));
   GWB_TRY(gwb::read_and_clear_device_error_stream(as_stream(stream), &flag2));
   GWB_TRY(gwb::read_and_clear_device_error_tmem(as_stream(stream), &flag3));
@@ -90,7 +90,8 @@ gwb_status gwb_check_device_error(void *stream) {
   GWB_TRY(gwb::read_and_clear_device_error_tc2(as_stream(stream), &flag5));
   GWB_TRY(gwb::read_and_clear_device_error_gate_up(as_stream(stream), &flag6));
   GWB_TRY(gwb::read_and_clear_device_error_silu(as_stream(stream), &flag7));
-  flag |= flag2 | flag3 | flag4 | flag5 | flag6 | flag7;
+  GWB_TRY(gwb::read_and_clear_device_error_w4a8(as_stream(stream), &flag8));
+  flag |= flag2 | flag3 | flag4 | flag5 | flag6 | flag7 | flag8;
   if (flag) return fail(GWB_ERR_TIMEOUT, "a bounded device-side wait gave up (flag 0x%x)", flag);
   return GWB_OK;
 }
@@ -409,6 +410,30 @@ gwb_status gwb_gemm_i8i8(const int8_t *qx, const float *sx, int64_t M, const int
   GWB_TRY(need(sw, "sw"));
   if (!aligned16(qx) || !aligned16(wq)) return fail(GWB_ERR_ALIGN, "qx and wq must be 16-byte aligned");
   return gwb::launch_tc2_i8i8(qx, sx, M, wq, sw, N, K, y, acc, as_stream(stream));
+}
+
+gwb_status gwb_gemv_w4a8(const uint16_t *x, int64_t M, const uint32_t *wq, const float *sw, int64_t N, int64_t K,
+                         uint16_t *y, void *stream) {
+  if (M < 0 || N < 0 || K < 0)
+    return fail(GWB_ERR_INVALID_ARG, "negative size (M=%lld, N=%lld, K=%lld)", (long long)M, (long long)N,
+                (long long)K);
+  if (N >= kMaxDim || K >= kMaxDim) return fail(GWB_ERR_SHAPE, "N and K must be below 2^31");
+  if (M > 8) return fail(GWB_ERR_SHAPE, "gemv_w4a8 takes at most 8 tokens (M=%lld)", (long long)M);
+  if (K % 512 != 0 || K > 16384)
+    return fail(GWB_ERR_UNSUPPORTED, "gemv_w4a8 needs K %% 512 == 0 and K <= 16384 (K=%lld)", (long long)K);
+  if (M == 0 || N == 0) return GWB_OK;
+  GWB_TRY(need(y, "y"));
+  if (K == 0) return zero_fill(y, (size_t)M * N * 2, stream);
+  GWB_TRY(need(x, "x"));
+  GWB_TRY(need(wq, "wq"));
+  GWB_TRY(need(sw, "sw"));
+  if (!aligned16(x)) return fail(GWB_ERR_ALIGN, "x is not 16-byte aligned");
+  const gwb_status s = gwb::launch_gemv_w4a8(x, (int)M, wq, sw, N, K, y, as_stream(stream));
+  return s == GWB_ERR_UNSUPPORTED
+             ? fail(GWB_ERR_UNSUPPORTED,
+                    "gemv_w4a8: the staged activations of %lld tokens x K=%lld do not fit on chip; quantize with "
+                    "quant_per_token_i8 and call gemm_i8i4", (long long)M, (long long)K)
+             : s;
 }
 
 }  // extern "C"

@@ -48,6 +48,18 @@
 //     are staged (never written to memory), and an optional residual is added
 //     to the fp32 result before its single rounding to bf16.
 //
+// W4A8 with the per-token quantization fused (kOpW4A8; executorch PR #24467,
+// mlx::int8_int4_gemm, whose "staged" lowering quantizes the activations inside
+// the product kernel): the staging quantizes x to int8 per token (sx = max|x| /
+// 127 over all of K, q = rint(x / sx) clipped to +-127, in fp32 as the
+// standalone quantizer does), the weights are symmetric int4 codes with one
+// scale per row (no groups, no biases).  The fp16 MMAs then compute the exact
+// int32 sum: codes and q are exact in fp16, every partial sum is an integer
+// below 2^24 for K <= 16384 (the chains run 64 k at a time), and the signed
+// codes enter the magic-number unpack as code ^ 8 with the -8 folded into the
+// accumulator start.  y = bf16(acc * (sx[t] * sw[n])), bit-identical to the
+// two-launch path.  K is not split (the scale needs the whole row).
+//
 // This header holds the kernel template and its host-side planner; each
 // translation unit that includes it instantiates the modes it launches.
 #include <cooperative_groups.h>
@@ -78,6 +90,7 @@ constexpr int kSMs = 148;
 constexpr int kOpPlain = 0;   // y = x W^T
 constexpr int kOpDual = 1;    // y = x W^T and y2 = x W2^T, one grid over both weights' strips
 constexpr int kOpSilu = 2;    // y = (resid +) (silu(x) * x2) W^T, the product formed in the staging
+constexpr int kOpW4A8 = 3;    // y = (sum_k q[t,k] c[n,k]) sx[t] sw[n]: x quantized to int8 per token in the staging
 
 template <int BITS, int GS>
 struct PCfg {
@@ -224,6 +237,7 @@ struct PipeArgs {
   int NS;          // strips of 16 rows (dual: of both weights)
   int NSH;         // dual: strips of one weight (the second weight's strips follow)
   int sb_swap2;    // dual: sb_swap of the second weight
+  const float *sw;        // w4a8: per-row weight scales [N]
   int ns_per, ns_rem;   // strips per CTA: ns_per, and one more for the first ns_rem CTAs
   int w3d;         // packed words: one 3-D box per stage (else two 2-D boxes)
   int sb_joint;    // scales and biases: one 3-D box per stage (else one each)
@@ -291,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __shared__ float red[kCW][8];
   __shared__ PartRec rec[kCW][2];
   __shared__ volatile int abort_flag;
+  __shared__ float tok_sx[8];   // w4a8: the per-token activation scales
   unsigned char *base = align_smem_1024(smem_raw);
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -329,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if constexpr (OP == kOpSilu) {
         if (a.resid) v += bf16_val(a.resid[(int64_t)t * a.N + row]);
       }
+      if constexpr (OP == kOpW4A8) v = v * (tok_sx[t] * __ldg(a.sw + row));   // v is the exact int32 sum
       yp[(int64_t)t * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
     }
   };
@@ -339,8 +355,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     tma_prefetch_desc(&tm_w);
-    tma_prefetch_desc(&tm_sb);
-    if (!a.sb_joint) tma_prefetch_desc(&tm_b);
+    if (OP != kOpW4A8) {
+      tma_prefetch_desc(&tm_sb);
+      if (!a.sb_joint) tma_prefetch_desc(&tm_b);
+    }
     if (OP == kOpDual) {
       tma_prefetch_desc(&tm_w2);
       tma_prefetch_desc(&tm_sb2);
@@ -367,14 +385,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t ds = smem_u32(ringSB + slot * 2 * C::SBB);
     const int gsx = ks / GS;
     const int gbox = C::GST < 8 ? (gsx & ~7) : gsx;
-    mbar_arrive_expect_tx(&full[slot], C::WB + 2 * C::SBB);
+    mbar_arrive_expect_tx(&full[slot], C::WB + (OP == kOpW4A8 ? 0 : 2 * C::SBB));
     if (a.w3d) {
       tma_load_3d_l(dw, mw, 0, r0, ks / (32 * C::CPW), bar);
     } else {
       tma_load_2d_l(dw, mw, ks / C::CPW, r0, bar);
       tma_load_2d_l(dw + 2048, mw, ks / C::CPW + 32, r0, bar);
     }
-    if (a.sb_joint) {
+    if (OP == kOpW4A8) {
+      // no scale or bias boxes
+    } else if (a.sb_joint) {
       tma_load_3d_l(ds, msb, gbox, r0, 0, bar);
     } else {
       tma_load_2d_l(ds, msb, gbox, r0, bar);
@@ -437,9 +457,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (++is_st == NCS) { is_st = 0; ++is_strip; }
   }
 
+  // max|x| of token t over this CTA's K-slice (every thread derives it from red[])
+  auto token_amax = [&](int t) -> float {
+    float m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kCW; w++) m = fmaxf(m, red[w][t]);
+    return m;
+  };
   // Per-token power of two e: the largest |x| * 2^e lands in [2^13, 2^14), so
   // the rescaled activations fit fp16 (every thread derives it from red[]).
   auto token_exp = [&](int t) -> int {
+    if (OP == kOpW4A8) return 0;   // the quantized values need no rescale
     float m = 0.0f;
 #pragma unroll
     for (int w = 0; w < kCW; w++) m = fmaxf(m, red[w][t]);
@@ -499,6 +527,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // written straight into the accumulator start quads (XNF) and the
     // split-bf16 B operand of the bias MMAs (XF).
     {
+      if (OP == kOpW4A8 && threadIdx.x < MP) tok_sx[threadIdx.x] = __fdiv_rn(token_amax(threadIdx.x), 127.0f);
       const int total = items;
       for (int b0 = 0; b0 < total; b0 += PB * kThreads) {
       Item itb[PB];
@@ -521,6 +550,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int t = tq[u], c = cq[u], g = gq[u];
         const bool live = sq[u] != nullptr;
         const float sc = pow2f(live ? token_exp(t) : 0);
+        // w4a8: the token's int8 scale, max|x| / 127 over the whole row (K is not split)
+        const float sq = OP == kOpW4A8 ? __fdiv_rn(token_amax(t), 127.0f) : 0.0f;
         const Item &rawb = itb[u];
         float sx = 0.0f, sn = 0.0f;
         uint32_t pr[C::NREG];
@@ -529,7 +560,13 @@ __global__ void __launch_bounds__(kThreads, 2)
           uint16_t h[C::CPW];
 #pragma unroll
           for (int p = 0; p < C::CPW; p++) {
-            h[p] = __half_as_ushort(__float2half_rn(rawb.get(wi, p) * sc));
+            if constexpr (OP == kOpW4A8) {
+              // q = clip(round_half_even(x / sx), -127, 127), exactly as the standalone quantizer
+              const float q = sq == 0.0f ? 0.0f : fminf(fmaxf(rintf(__fdiv_rn(rawb.get(wi, p), sq)), -127.0f), 127.0f);
+              h[p] = __half_as_ushort(__float2half_rn(q));
+            } else {
+              h[p] = __half_as_ushort(__float2half_rn(rawb.get(wi, p) * sc));
+            }
             sx += __half2float(__ushort_as_half(h[p]));
           }
 #pragma unroll
@@ -552,7 +589,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         sx += __shfl_xor_sync(kFull, sx, 2);
         sn += __shfl_xor_sync(kFull, sn, 2);
         if (valid && c == 0) {
-          const float xn = live ? -1024.0f * sn : 0.0f, X = live ? sx : 0.0f;
+          // w4a8: the codes enter as (code ^ 8) = code + 8, so the start also takes 8 sum(q) off
+          const float xn = live ? (OP == kOpW4A8 ? -1024.0f * sn - 8.0f * sx : -1024.0f * sn) : 0.0f;
+          const float X = live ? sx : 0.0f;
           // accumulator quad of quad lane t / 2: components t % 2 and t % 2 + 2
           float *q = reinterpret_cast<float *>(XNF + g * 4 + (t >> 1));
           q[t & 1] = xn;
@@ -651,7 +690,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int p = 0; p < 8; p++)
         ldmatrix_x4(sw + (p >> 2) * 2048 + swz[p & 3], wd[2 * p][0], wd[2 * p][1], wd[2 * p + 1][0], wd[2 * p + 1][1]);
       uint32_t sA[NSW], sB[NSW];
-      {
+      if constexpr (OP == kOpW4A8) {
+#pragma unroll
+        for (int q = 0; q < NSW; q++) sA[q] = sB[q] = 0u;   // no group scales
+      } else {
         const uint32_t *ra = sp + g8 * SW + (jb >> 1), *rb = sp + (g8 + 8) * SW + (jb >> 1);
         if constexpr (NSW >= 4) {
 #pragma unroll
@@ -670,8 +712,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t ba0[C::NBM], ba1[C::NBM];
 #pragma unroll
       for (int b = 0; b < C::NBM; b++) {
-        ba0[b] = bp[g8 * SW + b * 4 + c];
-        ba1[b] = bp[(g8 + 8) * SW + b * 4 + c];
+        ba0[b] = OP == kOpW4A8 ? 0u : bp[g8 * SW + b * 4 + c];
+        ba1[b] = OP == kOpW4A8 ? 0u : bp[(g8 + 8) * SW + b * 4 + c];
       }
       __syncwarp();
       if (i + D < units) {   // the slot has been read: refill it D stages ahead
@@ -685,11 +727,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint4 *xst = xbl + st * (C::GST * (C::NMMA / 2) * xbs);   // this stage's B fragments
       const float4 *xnst = XNF + st * (C::GST * 4) + c;                // and accumulator start values
       // ---- bias term: sum over the box's groups of bias * (x sums of this stage)
+      if constexpr (OP != kOpW4A8) {   // (w4a8 has no biases)
 #pragma unroll
-      for (int b = 0; b < C::NBM; b++) {
-        const uint2 xf = XF[(st * C::NBM + b) * 32 + lane];
-        mma_bf16_1688(accb, ba0[b], ba1[b], xf.x);
-        mma_bf16_1688(accb, ba0[b], ba1[b], xf.y);
+        for (int b = 0; b < C::NBM; b++) {
+          const uint2 xf = XF[(st * C::NBM + b) * 32 + lane];
+          mma_bf16_1688(accb, ba0[b], ba1[b], xf.x);
+          mma_bf16_1688(accb, ba0[b], ba1[b], xf.y);
+        }
       }
       // ---- codes: GI groups at a time, their MMA chains interleaved (independent
       // accumulators), then each group's scale
@@ -703,8 +747,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int j = j0 + gi;
 #pragma unroll
           for (int wi = 0; wi < C::NCH; wi++) {
-            unpack_word<BITS>(wd[j * C::NCH + wi][0], &ra[gi][wi * C::RPW], mag);
-            unpack_word<BITS>(wd[j * C::NCH + wi][1], &rb[gi][wi * C::RPW], mag);
+            // w4a8: two's-complement nibbles flipped to code + 8 in [0, 15]
+            constexpr uint32_t flip = OP == kOpW4A8 ? 0x88888888u : 0u;
+            unpack_word<BITS>(wd[j * C::NCH + wi][0] ^ flip, &ra[gi][wi * C::RPW], mag);
+            unpack_word<BITS>(wd[j * C::NCH + wi][1] ^ flip, &rb[gi][wi * C::RPW], mag);
           }
           xg[gi] = xst + j * (C::NMMA / 2) * xbs;
         }
@@ -730,15 +776,25 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 #pragma unroll
         for (int gi = 0; gi < C::GI; gi++) {
-          const int j = j0 + gi;
-          const uint32_t su = sA[j >> 1], sv = sB[j >> 1];
-          const float fa = (j & 1) ? __uint_as_float(su & 0xffff0000u) : __uint_as_float(su << 16);
-          const float fb = (j & 1) ? __uint_as_float(sv & 0xffff0000u) : __uint_as_float(sv << 16);
-          acc[0] = fmaf(fa, p[gi][0], acc[0]);
-          acc[2] = fmaf(fb, p[gi][2], acc[2]);
-          if constexpr (MP > 1) {
-            acc[1] = fmaf(fa, p[gi][1], acc[1]);
-            acc[3] = fmaf(fb, p[gi][3], acc[3]);
+          if constexpr (OP == kOpW4A8) {
+            // exact integer sums: one scale per row, applied at the output
+            acc[0] += p[gi][0];
+            acc[2] += p[gi][2];
+            if constexpr (MP > 1) {
+              acc[1] += p[gi][1];
+              acc[3] += p[gi][3];
+            }
+          } else {
+            const int j = j0 + gi;
+            const uint32_t su = sA[j >> 1], sv = sB[j >> 1];
+            const float fa = (j & 1) ? __uint_as_float(su & 0xffff0000u) : __uint_as_float(su << 16);
+            const float fb = (j & 1) ? __uint_as_float(sv & 0xffff0000u) : __uint_as_float(sv << 16);
+            acc[0] = fmaf(fa, p[gi][0], acc[0]);
+            acc[2] = fmaf(fb, p[gi][2], acc[2]);
+            if constexpr (MP > 1) {
+              acc[1] = fmaf(fa, p[gi][1], acc[1]);
+              acc[3] = fmaf(fb, p[gi][3], acc[3]);
+            }
           }
         }
       }
@@ -873,6 +929,7 @@ CUresult encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint
 // vectors and resid the optional residual.
 struct PipeIn {
   const uint16_t *x = nullptr, *x2 = nullptr, *resid = nullptr;
+  const float *sw = nullptr;   // w4a8: per-row weight scales
   int M = 0;
   const uint32_t *wq = nullptr, *wq2 = nullptr;
   const uint16_t *scales = nullptr, *biases = nullptr, *scales2 = nullptr, *biases2 = nullptr;
@@ -888,7 +945,7 @@ struct PipeIn {
 template <int BITS, int GS>
 CUresult weight_maps(const uint32_t *wq, const uint16_t *scales, const uint16_t *biases, int64_t N, int64_t K,
                      bool allow_w3d, bool allow_joint, CUtensorMap &tw, CUtensorMap &tsb, CUtensorMap &tb, int &w3d,
-                     int &joint, int &swap) {
+                     int &joint, int &swap, bool with_sb = true) {
   using C = PCfg<BITS, GS>;
   const int64_t G = K / GS;
   const uint64_t words = (uint64_t)K / C::CPW;
@@ -907,9 +964,15 @@ CUresult weight_maps(const uint32_t *wq, const uint16_t *scales, const uint16_t 
   if (!w3d)
     r = encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, (uint64_t)N, words * 4, 32u, 16u,
                   CU_TENSOR_MAP_SWIZZLE_128B);
+  joint = 0;
+  swap = 0;
+  if (!with_sb) {   // (w4a8: no scale or bias boxes)
+    tsb = tw;
+    tb = tw;
+    return r;
+  }
   const uintptr_t ps = reinterpret_cast<uintptr_t>(scales), pb = reinterpret_cast<uintptr_t>(biases);
   const uint64_t diff = ps > pb ? ps - pb : pb - ps;
-  joint = 0;
   swap = pb < ps ? 1 : 0;
   if (r == CUDA_SUCCESS && allow_joint && diff != 0 && diff % 16 == 0 && diff < (1ull << 39)) {
     const cuuint64_t dims[3] = {(cuuint64_t)G, (cuuint64_t)N, 2};
@@ -997,13 +1060,14 @@ gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
   };
   if ((int64_t)NS * nst >= 2LL * kSMs * kCW * 4) consider(1, 2);
   consider(1, 1);
-  for (int S = 2; S <= 8; S *= 2) consider(S, 1);
+  if (OP != kOpW4A8)   // w4a8: the per-token scale needs each CTA to see the whole row
+    for (int S = 2; S <= 8; S *= 2) consider(S, 1);
   if (!have) return GWB_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(reinterpret_cast<const void *>(kern), best.smem))
     return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute failed for %zu bytes of shared memory", best.smem);
 
   PipeArgs a{};
-  a.x = in.x; a.x2 = in.x2; a.resid = in.resid;
+  a.x = in.x; a.x2 = in.x2; a.resid = in.resid; a.sw = in.sw;
   a.y = in.y; a.y2 = in.y2;
   a.M = in.M; a.N = (int)N; a.K = (int)K;
   a.NS = NS; a.NSH = NSH;
@@ -1013,7 +1077,8 @@ gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
 
   CUtensorMap tw, tsb, tb, tw2, tsb2, tb2;
   int w3d = 0, joint = 0, swap = 0, w3d2 = 0, joint2 = 0, swap2 = 0;
-  CUresult r = weight_maps<BITS, GS>(in.wq, in.scales, in.biases, N, K, true, true, tw, tsb, tb, w3d, joint, swap);
+  CUresult r = weight_maps<BITS, GS>(in.wq, in.scales, in.biases, N, K, true, true, tw, tsb, tb, w3d, joint, swap,
+                                     OP != kOpW4A8);
   if (OP == kOpDual && r == CUDA_SUCCESS) {
     r = weight_maps<BITS, GS>(in.wq2, in.scales2, in.biases2, N, K, true, true, tw2, tsb2, tb2, w3d2, joint2, swap2);
     // both weights take the same box forms (the kernel has one flag of each)

@@ -51,6 +51,9 @@ gwb_status launch_gemv_pipe(const uint16_t *x, int M, const uint32_t *wq, const 
 gwb_status read_and_clear_device_error_pipe(cudaStream_t st, unsigned int *flag);
 gwb_status read_and_clear_device_error_gate_up(cudaStream_t st, unsigned int *flag);
 gwb_status read_and_clear_device_error_silu(cudaStream_t st, unsigned int *flag);
+gwb_status read_and_clear_device_error_w4a8(cudaStream_t st, unsigned int *flag);
+gwb_status launch_gemv_w4a8(const uint16_t *x, int M, const uint32_t *wq, const float *sw, int64_t N, int64_t K,
+                            uint16_t *y, cudaStream_t st);
 gwb_status launch_gemv_gate_up(const uint16_t *x, int M, const uint32_t *wq_gate, const uint16_t *sc_gate,
                                const uint16_t *bi_gate, const uint32_t *wq_up, const uint16_t *sc_up,
                                const uint16_t *bi_up, int64_t N, int64_t K, int bits, int gs, uint16_t *y_gate,

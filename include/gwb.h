@@ -251,6 +251,25 @@ gwb_status gwb_gemm_i8i4(const int8_t *qx, const float *sx, int64_t M, const uin
                          const float *sw, int64_t N, int64_t K, uint16_t *y, int32_t *acc,
                          void *stream);
 
+/* gemv_w4a8 -- W4A8 at decode with the activation quantization fused into the
+ * product: x is quantized to int8 per token (as gwb_quant_per_token_i8 does)
+ * inside the kernel and never written to memory, then
+ *   acc[m,n] = sum_k q[m,k] * code(n,k);  y[m,n] = bf16_rne(fp32(acc) * (sx[m] * sw[n]))
+ * Source: W4A8 ("staged" lowering of mlx::int8_int4_gemm, which quantizes the
+ * activations inside the product kernel).  Bit-identical to
+ * gwb_quant_per_token_i8 followed by gwb_gemm_i8i4 on the same x.
+ *   x bf16 [M, K] (16-byte aligned), wq u32 [N, K/8] and sw fp32 [N] from
+ *   gwb_qpack_sym_i4, y bf16 [M, N].
+ * 1 <= M <= 8 (GWB_ERR_SHAPE beyond: quantize once with gwb_quant_per_token_i8
+ * and call gwb_gemm_i8i4), K % 512 == 0 and K <= 16384 (GWB_ERR_UNSUPPORTED
+ * otherwise: the kernel's fp16 tensor-core sums are exact integers only up to
+ * that K).  Every CTA keeps the whole quantized rows on chip (the per-token
+ * scale needs all of K), about 2 * K * P bytes with P = M rounded up to 1, 2,
+ * 4 or 8: K <= 8192 at P = 8 and K <= 15872 at P = 4; larger is
+ * GWB_ERR_UNSUPPORTED. */
+gwb_status gwb_gemv_w4a8(const uint16_t *x, int64_t M, const uint32_t *wq, const float *sw, int64_t N,
+                         int64_t K, uint16_t *y, void *stream);
+
 /* ------------------------------------------------------------------ W8A8 */
 
 /* qpack_sym_i8 -- symmetric per-output-channel int8 weights (qMax = 127):

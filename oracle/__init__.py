@@ -261,6 +261,13 @@ def gemm_i8i4(qx, sx, wq, sw, N, K, rows=None):
     return acc, y, bool(ovf)
 
 
+def w4a8_fused(x_bf16, wq, sw, N, K, rows=None):
+    """The W4A8 product with the activation quantization inside it: by definition the
+    per-token quantizer followed by the int8 x int4 product.  Returns (acc, y, overflow)."""
+    qx, sx = quant_per_token_i8(x_bf16)
+    return gemm_i8i4(qx, sx, wq, sw, N, K, rows=rows)
+
+
 # ----------------------------------------------------------------- W8A8
 def qpack_sym_i8(w):
     """Returns (wq int8 [N, K], sw float32 [N])."""

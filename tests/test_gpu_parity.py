@@ -439,6 +439,43 @@ def test_w8a8_rejects_misaligned_and_bad_k():
         gwb.gemm_i8i8(torch.zeros(4, 72, dtype=torch.int8, device=DEV), sx, wq[:, :72].contiguous(), sw)
 
 
+# --------------------------------------------------------------------------- W4A8, quantization fused
+@pytest.mark.parametrize("N,K", [(200, 1024), (4096, 4096), (1000, 8192), (1000, 14336)])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8])
+def test_gemv_w4a8_matches_two_launch_path(N, K, M):
+    """The fused product equals quant_per_token_i8 + gemm_i8i4 bit for bit, and the oracle within the
+    float tolerance.  More than 4 tokens of 14336 values do not fit on chip: a clear error."""
+    w = W4A8(N, K, seed=N + M)
+    if K == 14336 and M > 4:
+        with pytest.raises(gwb.GwbError, match="do not fit on chip"):
+            gwb.gemv_w4a8(torch.zeros(M, K, dtype=torch.bfloat16, device=DEV), w.wq, w.sw)
+        return
+    x = synth.activations(M, K, seed=M, outlier_frac=0.01)
+    xd = x.to(DEV)
+    y = gwb.gemv_w4a8(xd, w.wq, w.sw)
+    qx, sx = gwb.quant_per_token_i8(xd)
+    y2, _ = gwb.gemm_i8i4(qx, sx, w.wq, w.sw)
+    assert torch.equal(y, y2), "fused W4A8 differs from the two-launch path"
+    rows = _rows(M, N, K)
+    acc_o, y_o, ovf = oracle.w4a8_fused(synth.bits16(x), w.wq_o, w.sw_o, N, K, rows=rows)
+    assert not ovf
+    yg = y.float().cpu().numpy()
+    if rows is not None:
+        yg = yg[rows]
+    check_float(yg, y_o, K, float(np.max(np.abs(w.sw_o)) * 7), float(x.float().abs().max()), f"w4a8 fused M={M}")
+
+
+def test_gemv_w4a8_argument_errors():
+    w = W4A8(64, 256)
+    with pytest.raises(gwb.GwbError, match="UNSUPPORTED"):      # K % 512 != 0
+        gwb.gemv_w4a8(torch.zeros(1, 256, dtype=torch.bfloat16, device=DEV), w.wq, w.sw)
+    w2 = W4A8(64, 512)
+    with pytest.raises(gwb.GwbError, match="SHAPE"):            # more than 8 tokens
+        gwb.gemv_w4a8(torch.zeros(9, 512, dtype=torch.bfloat16, device=DEV), w2.wq, w2.sw)
+    z = gwb.gemv_w4a8(torch.zeros(2, 512, dtype=torch.bfloat16, device=DEV), w2.wq, w2.sw)
+    assert torch.all(z == 0)                                     # all-zero tokens: sx = 0, q = 0
+
+
 @pytest.mark.parametrize("bits,M", [(4, 512), (4, 300), (8, 512)])
 def test_qmm_affine_stream_k_split_tiles(bits, M):
     # 8 x 2 tiles of 256 x 256 and 32 K steps over 74 CTA pairs: every tile is

@@ -547,3 +547,20 @@ def test_qmv_silu_gate_is_matmul_of_silu_product():
     W = oracle.dequant_affine_f64(wq, sc, bi, N, K, bits, gs)
     y = oracle.qmv_silu_gate(gate, up, wq, sc, bi, N, K, bits, gs, rows=[3, 1])
     assert np.allclose(y, oracle.silu_mul(gate, up)[[3, 1]] @ W.T, rtol=1e-12, atol=1e-14)
+
+
+def test_w4a8_fused_exact_grid_case():
+    """x on the exact int8 grid of its own scale: x = q * 2^-3 with max|q| = 127 gives sx = 2^-3 and
+    the codes q back unchanged; acc = q . c^T for known int4 codes; y = acc * sx * sw."""
+    q = np.array([[127, -64, 0, 1, -127, 5, 3, -2] * 4, [-127, 2, 2, 2, 2, 2, 2, 2] * 4], np.int64)
+    K = q.shape[1]
+    x = _bf16((q * 0.125).astype(np.float32)).reshape(2, K)
+    rng = np.random.default_rng(9)
+    codes = rng.integers(-8, 8, size=(3, K)).astype(np.int64)
+    wq = np.zeros((3, K // 8), np.int64)
+    for j in range(8):
+        wq |= (codes.reshape(3, K // 8, 8)[:, :, j] & 0xF) << (4 * j)
+    sw = np.array([0.5, 0.25, 2.0], np.float32)
+    acc, y, ovf = oracle.w4a8_fused(x, wq.astype(np.uint32), sw, 3, K)
+    assert not ovf and np.array_equal(acc, q @ codes.T)
+    assert np.array_equal(y, (q @ codes.T) * 0.125 * sw.astype(np.float64)[None, :])
