@@ -354,8 +354,12 @@ def run_int8(gwb, dev, stream, fmt, N, K, M, int8_peak, hbm_peak, reps=5):
             if r >= 2:
                 ts.append(a.elapsed_time(b))
     ms = statistics.median(ts)
-    kern = "k_tc2<I8,4,256,pair,A in TMEM> (kind::i8)" if fmt == "w4a8" else \
-        "k_tc2<W8,8,%s> (kind::i8, both operands by TMA)" % ("256,pair" if M > 128 else "128" if M > 32 else "32")
+    if fmt == "w4a8":
+        kern = "k_tc2<I8,4,256,pair,A in TMEM> (kind::i8)"
+    elif M <= 8 and K % 512 == 0:
+        kern = "k_gemv_pipe<8,64,%d,i8w8> (int8 x int8 weight streaming, exact int32 sums)" % (M,)
+    else:
+        kern = "k_tc2<W8,8,%s> (kind::i8, both operands by TMA)" % ("256,pair" if M > 128 else "128" if M > 32 else "32")
     out = {"N": N, "K": K, "M": M, "us": round(ms * 1e3, 1)}
     if M <= 8:
         wbytes = N * K // (2 if fmt == "w4a8" else 1)

@@ -82,7 +82,7 @@ const char *gwb_last_error(void) { return gwb::g_msg; }
 const char *gwb_version(void) { return "group_wise_bit_b200 0.1 (sm_100a)"; }
 
 gwb_status gwb_check_device_error(void *stream) {
-  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0, flag5 = 0, flag6 = 0, flag7 = 0, flag8 = 0;
+  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0, flag5 = 0, flag6 = 0, flag7 = 0, flag8 = 0, flag9 = 0;
   GWB_TRY(gwb::read_and_clear_device_error(as_stream(stream), &flag));
   GWB_TRY(gwb::read_and_clear_device_error_stream(as_stream(stream), &flag2));
   GWB_TRY(gwb::read_and_clear_device_error_tmem(as_stream(stream), &flag3));
@@ -91,7 +91,8 @@ gwb_status gwb_check_device_error(void *stream) {
   GWB_TRY(gwb::read_and_clear_device_error_gate_up(as_stream(stream), &flag6));
   GWB_TRY(gwb::read_and_clear_device_error_silu(as_stream(stream), &flag7));
   GWB_TRY(gwb::read_and_clear_device_error_w4a8(as_stream(stream), &flag8));
-  flag |= flag2 | flag3 | flag4 | flag5 | flag6 | flag7 | flag8;
+  GWB_TRY(gwb::read_and_clear_device_error_i8w8(as_stream(stream), &flag9));
+  flag |= flag2 | flag3 | flag4 | flag5 | flag6 | flag7 | flag8 | flag9;
   if (flag) return fail(GWB_ERR_TIMEOUT, "a bounded device-side wait gave up (flag 0x%x)", flag);
   return GWB_OK;
 }
@@ -409,6 +410,11 @@ gwb_status gwb_gemm_i8i8(const int8_t *qx, const float *sx, int64_t M, const int
   GWB_TRY(need(wq, "wq"));
   GWB_TRY(need(sw, "sw"));
   if (!aligned16(qx) || !aligned16(wq)) return fail(GWB_ERR_ALIGN, "qx and wq must be 16-byte aligned");
+  if (M <= 8 && K % 512 == 0) {
+    // decode: the weight-streaming kernel (falls through when the rows do not fit on chip)
+    const gwb_status s = gwb::launch_gemv_i8w8(qx, sx, (int)M, wq, sw, N, K, y, acc, as_stream(stream));
+    if (s != GWB_ERR_UNSUPPORTED) return s;
+  }
   return gwb::launch_tc2_i8i8(qx, sx, M, wq, sw, N, K, y, acc, as_stream(stream));
 }
 

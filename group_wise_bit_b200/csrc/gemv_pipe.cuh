@@ -60,6 +60,14 @@
 // accumulator start.  y = bf16(acc * (sx[t] * sw[n])), bit-identical to the
 // two-launch path.  K is not split (the scale needs the whole row).
 //
+// W8A8 at decode (kOpI8W8; the 8da8w config of executorch PR #17234): int8
+// activations (already quantized) and int8 weights with one scale per row.
+// The codes enter the 8-bit unpack as code ^ 0x80 = code + 128 (the -128 is
+// folded into the accumulator start); each 64-k chain is an exact fp32
+// integer, and the chains are summed in int32 (the whole sum may pass 2^24),
+// through the partial-strip reduction too.  The int32 sums are exact; K is
+// not split.
+//
 // This header holds the kernel template and its host-side planner; each
 // translation unit that includes it instantiates the modes it launches.
 #include <cooperative_groups.h>
@@ -91,6 +99,7 @@ constexpr int kOpPlain = 0;   // y = x W^T
 constexpr int kOpDual = 1;    // y = x W^T and y2 = x W2^T, one grid over both weights' strips
 constexpr int kOpSilu = 2;    // y = (resid +) (silu(x) * x2) W^T, the product formed in the staging
 constexpr int kOpW4A8 = 3;    // y = (sum_k q[t,k] c[n,k]) sx[t] sw[n]: x quantized to int8 per token in the staging
+constexpr int kOpI8W8 = 4;    // acc = sum_k qx[t,k] wq[n,k] (int8 x int8, exact int32), y = acc sx[t] sw[n]
 
 template <int BITS, int GS>
 struct PCfg {
@@ -237,7 +246,9 @@ struct PipeArgs {
   int NS;          // strips of 16 rows (dual: of both weights)
   int NSH;         // dual: strips of one weight (the second weight's strips follow)
   int sb_swap2;    // dual: sb_swap of the second weight
-  const float *sw;        // w4a8: per-row weight scales [N]
+  const float *sw;        // w4a8, i8w8: per-row weight scales [N]
+  const float *sx;        // i8w8: per-token activation scales [M]
+  int32_t *acc;           // i8w8: optional int32 sums [M, N] (y may then be null)
   int ns_per, ns_rem;   // strips per CTA: ns_per, and one more for the first ns_rem CTAs
   int w3d;         // packed words: one 3-D box per stage (else two 2-D boxes)
   int sb_joint;    // scales and biases: one 3-D box per stage (else one each)
@@ -255,6 +266,14 @@ struct PartRec {   // a strip result that one warp holds only part of
 // (relative error far below the fp16 rounding the staged value takes next);
 // for g < -88 the exponential overflows to +inf and the reciprocal gives 0.
 __device__ __forceinline__ float silu_f(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+
+// One staged item of int8 activations: NCH runs of 4 values, one word each.
+template <int NCH>
+struct XItemI8 {
+  uint32_t r[NCH];
+  __device__ __forceinline__ float get(int wi, int p) const { return (float)(int8_t)(r[wi] >> (8 * p)); }
+  __device__ __forceinline__ float bound(int wi, int p) const { return fabsf(get(wi, p)); }
+};
 // An upper bound of |silu(g) * u| without the exponential: silu(g) <= g for
 // g >= 0, and |silu(g)| < 0.2785 for g < 0 (its minimum, near g = -1.278).
 __device__ __forceinline__ float silu_bound(float g, float u) { return fmaxf(g, 0.28f) * fabsf(u); }
@@ -300,7 +319,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const CUtensorMap &tm_w2 = maps.m[OP == kOpDual ? 3 : 0], &tm_sb2 = maps.m[OP == kOpDual ? 4 : 1],
                     &tm_b2 = maps.m[OP == kOpDual ? 5 : 2];
   using C = PCfg<BITS, GS>;
-  using Item = XItem<C::NCH, C::CPW, OP == kOpSilu>;
+  using Item = std::conditional_t<OP == kOpI8W8, XItemI8<C::NCH>, XItem<C::NCH, C::CPW, OP == kOpSilu>>;
+  static_assert(OP != kOpI8W8 || (BITS == 8 && C::CPW == 4), "int8 activations go with 8-bit codes");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ float red[kCW][8];
   __shared__ PartRec rec[kCW][2];
@@ -345,6 +365,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (a.resid) v += bf16_val(a.resid[(int64_t)t * a.N + row]);
       }
       if constexpr (OP == kOpW4A8) v = v * (tok_sx[t] * __ldg(a.sw + row));   // v is the exact int32 sum
+      if constexpr (OP == kOpI8W8) {
+        // v carries the bits of the int32 sum
+        const int vi = __float_as_int(v);
+        if (a.acc) a.acc[(int64_t)t * a.N + row] = vi;
+        if (yp) yp[(int64_t)t * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn((float)vi * (__ldg(a.sx + t) * __ldg(a.sw + row))));
+        return;
+      }
       yp[(int64_t)t * a.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
     }
   };
@@ -355,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     tma_prefetch_desc(&tm_w);
-    if (OP != kOpW4A8) {
+    if (OP != kOpW4A8 && OP != kOpI8W8) {
       tma_prefetch_desc(&tm_sb);
       if (!a.sb_joint) tma_prefetch_desc(&tm_b);
     }
@@ -385,14 +412,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t ds = smem_u32(ringSB + slot * 2 * C::SBB);
     const int gsx = ks / GS;
     const int gbox = C::GST < 8 ? (gsx & ~7) : gsx;
-    mbar_arrive_expect_tx(&full[slot], C::WB + (OP == kOpW4A8 ? 0 : 2 * C::SBB));
+    mbar_arrive_expect_tx(&full[slot], C::WB + (OP == kOpW4A8 || OP == kOpI8W8 ? 0 : 2 * C::SBB));
     if (a.w3d) {
       tma_load_3d_l(dw, mw, 0, r0, ks / (32 * C::CPW), bar);
     } else {
       tma_load_2d_l(dw, mw, ks / C::CPW, r0, bar);
       tma_load_2d_l(dw + 2048, mw, ks / C::CPW + 32, r0, bar);
     }
-    if (OP == kOpW4A8) {
+    if (OP == kOpW4A8 || OP == kOpI8W8) {
       // no scale or bias boxes
     } else if (a.sb_joint) {
       tma_load_3d_l(ds, msb, gbox, r0, 0, bar);
@@ -408,12 +435,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   // A thread loads its first item into registers before the ring fill below
   // (so the load latency hides behind the TMA issue) and keeps it for pass B.
   const int items = GR * MP * 4;
-  auto item_src = [&](int idx, int &t, int &c, int &g) -> const uint16_t * {
+  // the item's element offset t * K + (group start), or -1 when it holds nothing
+  auto item_src = [&](int idx, int &t, int &c, int &g) -> int64_t {
     c = idx & 3;
     t = (idx >> 2) % MP;
     g = (idx >> 2) / MP;
     const int kg = k0 + g * GS;
-    return (idx < items && t < a.M && kg < a.K) ? a.x + (int64_t)t * a.K + kg : nullptr;
+    return (idx < items && t < a.M && kg < a.K) ? (int64_t)t * a.K + kg : -1;
   };
   // CPW consecutive bf16 values at p, as CPW / 2 packed pairs
   auto load_pairs = [&](const uint16_t *p, uint32_t (&w)[C::CPW / 2]) {
@@ -428,11 +456,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   };
-  auto load_item = [&](const uint16_t *src, int c, Item &it) {
+  auto load_item = [&](int64_t off, int c, Item &it) {
 #pragma unroll
     for (int wi = 0; wi < C::NCH; wi++) {
-      const uint16_t *p = src ? src + k_in_group<BITS>(wi, c, 0) : nullptr;
-      if constexpr (OP == kOpSilu) {
+      const int64_t o = off + k_in_group<BITS>(wi, c, 0);
+      const uint16_t *p = off >= 0 ? a.x + o : nullptr;
+      if constexpr (OP == kOpI8W8) {
+        // 4 int8 values in one aligned word (K and the run start are multiples of 4)
+        it.r[wi] = off >= 0 ? __ldg(reinterpret_cast<const uint32_t *>(reinterpret_cast<const int8_t *>(a.x) + o)) : 0u;
+      } else if constexpr (OP == kOpSilu) {
         // the up value sits at the same offset of x2
 #pragma unroll
         for (int q = 0; q < C::CPW / 2; q++) it.g[wi][q] = it.u[wi][q] = 0u;
@@ -449,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   };
   Item raw0;
   int t0i, c0i, g0i;
-  const uint16_t *src0 = item_src(threadIdx.x, t0i, c0i, g0i);
+  const int64_t src0 = item_src(threadIdx.x, t0i, c0i, g0i);
   load_item(src0, c0i, raw0);
 
   for (int i = 0; i < (units < D ? units : D); i++) {
@@ -467,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // Per-token power of two e: the largest |x| * 2^e lands in [2^13, 2^14), so
   // the rescaled activations fit fp16 (every thread derives it from red[]).
   auto token_exp = [&](int t) -> int {
-    if (OP == kOpW4A8) return 0;   // the quantized values need no rescale
+    if (OP == kOpW4A8 || OP == kOpI8W8) return 0;   // integer values need no rescale
     float m = 0.0f;
 #pragma unroll
     for (int w = 0; w < kCW; w++) m = fmaxf(m, red[w][t]);
@@ -493,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int u = 0; u < PB; u++) {
           int t, c, g;
-          const uint16_t *src = item_src(b0 + u * kThreads + threadIdx.x, t, c, g);
+          const int64_t src = item_src(b0 + u * kThreads + threadIdx.x, t, c, g);
           if (b0 == 0 && u == 0) {
             itb[0] = raw0;
           } else {
@@ -532,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int b0 = 0; b0 < total; b0 += PB * kThreads) {
       Item itb[PB];
       int tq[PB], cq[PB], gq[PB];
-      const uint16_t *sq[PB];
+      int64_t sq[PB];
 #pragma unroll
       for (int u = 0; u < PB; u++) {
         sq[u] = item_src(b0 + u * kThreads + threadIdx.x, tq[u], cq[u], gq[u]);
@@ -548,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int idx = b0 + u * kThreads + threadIdx.x;
         const bool valid = idx < total;
         const int t = tq[u], c = cq[u], g = gq[u];
-        const bool live = sq[u] != nullptr;
+        const bool live = sq[u] >= 0;
         const float sc = pow2f(live ? token_exp(t) : 0);
         // w4a8: the token's int8 scale, max|x| / 127 over the whole row (K is not split)
         const float sq = OP == kOpW4A8 ? __fdiv_rn(token_amax(t), 127.0f) : 0.0f;
@@ -590,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         sn += __shfl_xor_sync(kFull, sn, 2);
         if (valid && c == 0) {
           // w4a8: the codes enter as (code ^ 8) = code + 8, so the start also takes 8 sum(q) off
-          const float xn = live ? (OP == kOpW4A8 ? -1024.0f * sn - 8.0f * sx : -1024.0f * sn) : 0.0f;
+          const float xn = live ? (OP == kOpW4A8 ? -1024.0f * sn - 8.0f * sx : OP == kOpI8W8 ? -1024.0f * sn - 128.0f * sx : -1024.0f * sn) : 0.0f;
           const float X = live ? sx : 0.0f;
           // accumulator quad of quad lane t / 2: components t % 2 and t % 2 + 2
           float *q = reinterpret_cast<float *>(XNF + g * 4 + (t >> 1));
@@ -646,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const bool whole = fst == 0 && lst == NCS - 1;
       float v[4];
 #pragma unroll
-      for (int i = 0; i < 4; i++) v[i] = (acc[i] + accb[i]) * ((i & 1) ? inv1 : inv0);
+      for (int i = 0; i < 4; i++) v[i] = OP == kOpI8W8 ? acc[i] : (acc[i] + accb[i]) * ((i & 1) ? inv1 : inv0);
       if (whole && S == 1) {
         const int rA = strip_ * 16 + g8;
 #pragma unroll
@@ -690,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int p = 0; p < 8; p++)
         ldmatrix_x4(sw + (p >> 2) * 2048 + swz[p & 3], wd[2 * p][0], wd[2 * p][1], wd[2 * p + 1][0], wd[2 * p + 1][1]);
       uint32_t sA[NSW], sB[NSW];
-      if constexpr (OP == kOpW4A8) {
+      if constexpr (OP == kOpW4A8 || OP == kOpI8W8) {
 #pragma unroll
         for (int q = 0; q < NSW; q++) sA[q] = sB[q] = 0u;   // no group scales
       } else {
@@ -712,8 +744,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t ba0[C::NBM], ba1[C::NBM];
 #pragma unroll
       for (int b = 0; b < C::NBM; b++) {
-        ba0[b] = OP == kOpW4A8 ? 0u : bp[g8 * SW + b * 4 + c];
-        ba1[b] = OP == kOpW4A8 ? 0u : bp[(g8 + 8) * SW + b * 4 + c];
+        ba0[b] = OP == kOpW4A8 || OP == kOpI8W8 ? 0u : bp[g8 * SW + b * 4 + c];
+        ba1[b] = OP == kOpW4A8 || OP == kOpI8W8 ? 0u : bp[(g8 + 8) * SW + b * 4 + c];
       }
       __syncwarp();
       if (i + D < units) {   // the slot has been read: refill it D stages ahead
@@ -727,7 +759,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint4 *xst = xbl + st * (C::GST * (C::NMMA / 2) * xbs);   // this stage's B fragments
       const float4 *xnst = XNF + st * (C::GST * 4) + c;                // and accumulator start values
       // ---- bias term: sum over the box's groups of bias * (x sums of this stage)
-      if constexpr (OP != kOpW4A8) {   // (w4a8 has no biases)
+      if constexpr (OP != kOpW4A8 && OP != kOpI8W8) {   // (the integer modes have no biases)
 #pragma unroll
         for (int b = 0; b < C::NBM; b++) {
           const uint2 xf = XF[(st * C::NBM + b) * 32 + lane];
@@ -747,8 +779,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int j = j0 + gi;
 #pragma unroll
           for (int wi = 0; wi < C::NCH; wi++) {
-            // w4a8: two's-complement nibbles flipped to code + 8 in [0, 15]
-            constexpr uint32_t flip = OP == kOpW4A8 ? 0x88888888u : 0u;
+            // w4a8 / i8w8: two's-complement nibbles / bytes flipped to code + 8 / code + 128
+            constexpr uint32_t flip = OP == kOpW4A8 ? 0x88888888u : OP == kOpI8W8 ? 0x80808080u : 0u;
             unpack_word<BITS>(wd[j * C::NCH + wi][0] ^ flip, &ra[gi][wi * C::RPW], mag);
             unpack_word<BITS>(wd[j * C::NCH + wi][1] ^ flip, &rb[gi][wi * C::RPW], mag);
           }
@@ -776,7 +808,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 #pragma unroll
         for (int gi = 0; gi < C::GI; gi++) {
-          if constexpr (OP == kOpW4A8) {
+          if constexpr (OP == kOpI8W8) {
+            // int32 sums (the bit pattern lives in the float registers): each
+            // chain is an exact integer, the total may pass 2^24
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+              if (MP > 1 || (q & 1) == 0) acc[q] = __int_as_float(__float_as_int(acc[q]) + __float2int_rn(p[gi][q]));
+          } else if constexpr (OP == kOpW4A8) {
             // exact integer sums: one scale per row, applied at the output
             acc[0] += p[gi][0];
             acc[2] += p[gi][2];
@@ -824,7 +862,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       float s = PART[(w * 2 + z) * 16 * MP + idx];
       for (int w2 = w; w2 < kCW; w2++)
         for (int z2 = 0; z2 < 2; z2++)
-          if ((w2 > w || z2 > z) && rec[w2][z2].strip == r.strip) s += PART[(w2 * 2 + z2) * 16 * MP + idx];
+          if ((w2 > w || z2 > z) && rec[w2][z2].strip == r.strip) {
+            const float pv = PART[(w2 * 2 + z2) * 16 * MP + idx];
+            s = OP == kOpI8W8 ? __int_as_float(__float_as_int(s) + __float_as_int(pv)) : s + pv;   // i8w8: int32 bits
+          }
       const int row = r.strip * 16 + idx / MP, t = idx % MP;
       if (S == 1) {
         put_y(row, t, s);
@@ -929,7 +970,9 @@ CUresult encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint
 // vectors and resid the optional residual.
 struct PipeIn {
   const uint16_t *x = nullptr, *x2 = nullptr, *resid = nullptr;
-  const float *sw = nullptr;   // w4a8: per-row weight scales
+  const float *sw = nullptr;   // w4a8, i8w8: per-row weight scales
+  const float *sx = nullptr;   // i8w8: per-token activation scales
+  int32_t *acc = nullptr;      // i8w8: optional int32 sums
   int M = 0;
   const uint32_t *wq = nullptr, *wq2 = nullptr;
   const uint16_t *scales = nullptr, *biases = nullptr, *scales2 = nullptr, *biases2 = nullptr;
@@ -1060,14 +1103,14 @@ gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
   };
   if ((int64_t)NS * nst >= 2LL * kSMs * kCW * 4) consider(1, 2);
   consider(1, 1);
-  if (OP != kOpW4A8)   // w4a8: the per-token scale needs each CTA to see the whole row
+  if (OP != kOpW4A8 && OP != kOpI8W8)   // w4a8: the per-token scale needs the whole row; i8w8: int32 sums
     for (int S = 2; S <= 8; S *= 2) consider(S, 1);
   if (!have) return GWB_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(reinterpret_cast<const void *>(kern), best.smem))
     return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute failed for %zu bytes of shared memory", best.smem);
 
   PipeArgs a{};
-  a.x = in.x; a.x2 = in.x2; a.resid = in.resid; a.sw = in.sw;
+  a.x = in.x; a.x2 = in.x2; a.resid = in.resid; a.sw = in.sw; a.sx = in.sx; a.acc = in.acc;
   a.y = in.y; a.y2 = in.y2;
   a.M = in.M; a.N = (int)N; a.K = (int)K;
   a.NS = NS; a.NSH = NSH;
@@ -1078,7 +1121,7 @@ gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
   CUtensorMap tw, tsb, tb, tw2, tsb2, tb2;
   int w3d = 0, joint = 0, swap = 0, w3d2 = 0, joint2 = 0, swap2 = 0;
   CUresult r = weight_maps<BITS, GS>(in.wq, in.scales, in.biases, N, K, true, true, tw, tsb, tb, w3d, joint, swap,
-                                     OP != kOpW4A8);
+                                     OP != kOpW4A8 && OP != kOpI8W8);
   if (OP == kOpDual && r == CUDA_SUCCESS) {
     r = weight_maps<BITS, GS>(in.wq2, in.scales2, in.biases2, N, K, true, true, tw2, tsb2, tb2, w3d2, joint2, swap2);
     // both weights take the same box forms (the kernel has one flag of each)

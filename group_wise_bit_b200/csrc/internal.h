@@ -52,6 +52,9 @@ gwb_status read_and_clear_device_error_pipe(cudaStream_t st, unsigned int *flag)
 gwb_status read_and_clear_device_error_gate_up(cudaStream_t st, unsigned int *flag);
 gwb_status read_and_clear_device_error_silu(cudaStream_t st, unsigned int *flag);
 gwb_status read_and_clear_device_error_w4a8(cudaStream_t st, unsigned int *flag);
+gwb_status read_and_clear_device_error_i8w8(cudaStream_t st, unsigned int *flag);
+gwb_status launch_gemv_i8w8(const int8_t *qx, const float *sx, int M, const int8_t *wq, const float *sw, int64_t N,
+                            int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 gwb_status launch_gemv_w4a8(const uint16_t *x, int M, const uint32_t *wq, const float *sw, int64_t N, int64_t K,
                             uint16_t *y, cudaStream_t st);
 gwb_status launch_gemv_gate_up(const uint16_t *x, int M, const uint32_t *wq_gate, const uint16_t *sc_gate,

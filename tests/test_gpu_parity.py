@@ -416,6 +416,14 @@ def test_w8a8_small(M):
     W8A8(200, 384, seed=M).check(M)
 
 
+@pytest.mark.parametrize("N,K", [(200, 1024), (1000, 8192), (4096, 14336)])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8])
+def test_w8a8_decode(N, K, M):
+    # M <= 8 with K % 512 == 0: the weight-streaming decode kernel with exact int32 sums (K = 14336
+    # with more than 4 tokens does not fit on chip and takes the tensor-core kernel)
+    W8A8(N, K, seed=M).check(M)
+
+
 @pytest.mark.parametrize("N,K,M", [(136, 96, 24), (264, 144, 40), (72, 272, 200)])
 def test_w8a8_k_tail(N, K, M):
     W8A8(N, K).check(M)    # K below or between 128-wide K steps
