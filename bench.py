@@ -143,12 +143,20 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The largest of the ranks' values (a device time: the job ends with its slowest rank)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_gbs(world, bytes_per_step, steps, ms_max):
+    """Whole-job throughput of `world` replicas that each moved bytes_per_step per step, timed as the
+    slowest rank: every rank processes its own copy of the workload (weak scaling)."""
+    return world * bytes_per_step * steps / (ms_max * 1e-3) / 1e9
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -227,7 +235,7 @@ def run_gpu(args, world, rank, local):
     ms = t0.elapsed_time(t1)
     ms_max = max_over_ranks(ms, world)
     ms_step = ms_max / args.steps
-    value = world * STEP_BYTES * args.steps / (ms_max * 1e-3) / 1e9
+    value = job_gbs(world, STEP_BYTES, args.steps, ms_max)
     lm_ms = float(np.mean([a.elapsed_time(b) for a, b in lm_events[:args.steps]]))
     lm_bytes = gemv_bytes(*LMHEAD)
     achieved = lm_bytes / (lm_ms * 1e-3) / 1e9
@@ -260,7 +268,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * STEP_BYTES * args.steps / (e_ms * 1e-3) / 1e9
+    e2e_value = job_gbs(world, STEP_BYTES, args.steps, e_ms)
 
     prefill = run_prefill(gwb, dev, stream, bf16_peak, peak_kind) if not args.no_prefill else None
     int8 = {}
