@@ -58,7 +58,9 @@
 // below 2^24 for K <= 16384 (the chains run 64 k at a time), and the signed
 // codes enter the magic-number unpack as code ^ 8 with the -8 folded into the
 // accumulator start.  y = bf16(acc * (sx[t] * sw[n])), bit-identical to the
-// two-launch path.  K is not split (the scale needs the whole row).
+// two-launch path.  When K is split over a cluster, the CTAs exchange their
+// per-token maxima through distributed shared memory before quantizing; the
+// partial sums stay exact integers, so their fp32 reduction is exact too.
 //
 // W8A8 at decode (kOpI8W8; the 8da8w config of executorch PR #17234): int8
 // activations (already quantized) and int8 weights with one scale per row.
@@ -489,9 +491,20 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (++is_st == NCS) { is_st = 0; ++is_strip; }
   }
 
-  // max|x| of token t over this CTA's K-slice (every thread derives it from red[])
+  // max|x| of token t over this CTA's K-slice (every thread derives it from red[]);
+  // w4a8 with K split over a cluster: over the whole row, from every CTA's red[]
+  // through distributed shared memory (after the cluster barrier that ends pass A)
   auto token_amax = [&](int t) -> float {
     float m = 0.0f;
+    if (OP == kOpW4A8 && S > 1) {
+      cg::cluster_group cluster = cg::this_cluster();
+      for (int q = 0; q < S; q++) {
+        const float *rr = cluster.map_shared_rank(&red[0][0], q);
+#pragma unroll
+        for (int w = 0; w < kCW; w++) m = fmaxf(m, rr[w * 8 + t]);
+      }
+      return m;
+    }
 #pragma unroll
     for (int w = 0; w < kCW; w++) m = fmaxf(m, red[w][t]);
     return m;
@@ -554,6 +567,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     __syncthreads();
+    // w4a8 with a K split: every CTA's maxima are complete before any CTA reads
+    // them (and red[] is not written again; no CTA leaves before the final
+    // cluster barrier of the split-K reduction)
+    if (OP == kOpW4A8 && S > 1) cg::this_cluster().sync();
     // Pass B: one thread per item: the B fragments of the lane's codes, and
     // (combined over c in order) the group's activation sum X and magic sum XN,
     // written straight into the accumulator start quads (XNF) and the
@@ -1103,7 +1120,7 @@ gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
   };
   if ((int64_t)NS * nst >= 2LL * kSMs * kCW * 4) consider(1, 2);
   consider(1, 1);
-  if (OP != kOpW4A8 && OP != kOpI8W8)   // w4a8: the per-token scale needs the whole row; i8w8: int32 sums
+  if (OP != kOpI8W8)   // i8w8: the int32 sums are not reduced across a cluster
     for (int S = 2; S <= 8; S *= 2) consider(S, 1);
   if (!have) return GWB_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(reinterpret_cast<const void *>(kern), best.smem))

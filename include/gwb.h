@@ -263,10 +263,10 @@ gwb_status gwb_gemm_i8i4(const int8_t *qx, const float *sx, int64_t M, const uin
  * 1 <= M <= 8 (GWB_ERR_SHAPE beyond: quantize once with gwb_quant_per_token_i8
  * and call gwb_gemm_i8i4), K % 512 == 0 and K <= 16384 (GWB_ERR_UNSUPPORTED
  * otherwise: the kernel's fp16 tensor-core sums are exact integers only up to
- * that K).  Every CTA keeps the whole quantized rows on chip (the per-token
- * scale needs all of K), about 2 * K * P bytes with P = M rounded up to 1, 2,
- * 4 or 8: K <= 8192 at P = 8 and K <= 15872 at P = 4; larger is
- * GWB_ERR_UNSUPPORTED. */
+ * that K).  The quantized rows are kept on chip; where a CTA cannot hold all
+ * of K, K is split over a cluster of CTAs that exchange their per-token maxima
+ * first (the scale is always the whole row's).  GWB_ERR_UNSUPPORTED only when
+ * no split fits. */
 gwb_status gwb_gemv_w4a8(const uint16_t *x, int64_t M, const uint32_t *wq, const float *sw, int64_t N,
                          int64_t K, uint16_t *y, void *stream);
 

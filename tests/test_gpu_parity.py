@@ -452,12 +452,9 @@ def test_w8a8_rejects_misaligned_and_bad_k():
 @pytest.mark.parametrize("M", [1, 2, 3, 5, 8])
 def test_gemv_w4a8_matches_two_launch_path(N, K, M):
     """The fused product equals quant_per_token_i8 + gemm_i8i4 bit for bit, and the oracle within the
-    float tolerance.  More than 4 tokens of 14336 values do not fit on chip: a clear error."""
+    float tolerance.  At K = 14336 with more than 4 tokens the rows do not fit one CTA: K is split
+    over a cluster whose CTAs exchange their per-token maxima."""
     w = W4A8(N, K, seed=N + M)
-    if K == 14336 and M > 4:
-        with pytest.raises(gwb.GwbError, match="do not fit on chip"):
-            gwb.gemv_w4a8(torch.zeros(M, K, dtype=torch.bfloat16, device=DEV), w.wq, w.sw)
-        return
     x = synth.activations(M, K, seed=M, outlier_frac=0.01)
     xd = x.to(DEV)
     y = gwb.gemv_w4a8(xd, w.wq, w.sw)
