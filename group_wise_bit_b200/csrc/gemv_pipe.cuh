@@ -600,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const bool live = sq[u] >= 0;
         const float sc = pow2f(live ? token_exp(t) : 0);
         // w4a8: the token's int8 scale, max|x| / 127 over the whole row (K is not split)
-        const float sq = OP == kOpW4A8 ? __fdiv_rn(token_amax(t), 127.0f) : 0.0f;
+        [[maybe_unused]] const float sq = OP == kOpW4A8 ? __fdiv_rn(token_amax(t), 127.0f) : 0.0f;
         const Item &rawb = itb[u];
         float sx = 0.0f, sn = 0.0f;
         uint32_t pr[C::NREG];
