@@ -44,7 +44,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_ranks_take_the_slowest_time_and_sum_the_work():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
     for rank in range(world):
         ms_max, gbs = out[rank]
