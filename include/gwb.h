@@ -7,13 +7,16 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
  *    never allocates, frees or retains them.  Tensors are dense and row-major
  *    with the shapes stated per call; no strides are taken.
- *  - The one device buffer the library owns is the prefill GEMM's stream-K
- *    workspace (partial tiles, about 19 MB): one per (device, stream),
- *    allocated by the first qmm_affine / gptq_qmm / gemm_i8i4 call with more
- *    than 128 tokens on that stream, and kept until the process exits.  A call
- *    made while its stream is being captured into a CUDA graph never
- *    allocates; it runs without the workspace (whole tiles per CTA pair).
- *    gwb_qmm_affine_noalloc is the entry point that allocates nothing.
+ *  - The one device buffer the library owns is the persistent tensor-core
+ *    GEMM's stream-K workspace (partial tiles, up to about 19 MB): one per
+ *    (device, stream), allocated by the first call on that stream that runs
+ *    that GEMM with split tiles (qmm_affine, gptq_qmm and awq_qmm above 128
+ *    tokens, gemm_i8i4 from 128, gemm_i8i8 off its decode path), grown once
+ *    if a later call needs more (after synchronizing the stream), and kept
+ *    until the process exits.  A call made while its stream is being captured
+ *    into a CUDA graph never allocates; it runs without the workspace (whole
+ *    tiles per CTA or pair).  gwb_qmm_affine_noalloc is the entry point that
+ *    allocates nothing.
  *  - bf16 and fp16 values are passed as their raw 16-bit patterns (uint16_t).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
  *    validates its arguments synchronously, on the host, before launching
@@ -35,8 +38,11 @@
  *                   scales  fp16   [K/gs, N]
  *                   qzeros  int32  [K/gs, N/8]  packed along OUT, stores zero-1
  *                   g_idx   int32  [K]          optional group of each in-feature
+ *                   (AWQ: the same tensors without g_idx, zero as stored)
  *      sym int4     wq      uint32 [N, K/8]     two's-complement nibbles along K
  *                   sw      fp32   [N]          w[n,k] = code*sw[n]
+ *      sym int8     wq      int8   [N, K]       w[n,k] = wq[n,k]*sw[n]
+ *                   sw      fp32   [N]
  *    A linear layer computes y[M,N] = x[M,K] . W^T, with W stored [N = out, K = in].
  *
  * Sources (page title, then section): "MLX" = metrale_gpu_runtime/mlx_int8.rs
