@@ -29,7 +29,7 @@
  *  - Device-side waits inside the tensor-core kernels are bounded; a wait that
  *    gives up records GWB_ERR_TIMEOUT in a device flag that
  *    gwb_check_device_error() reads and clears.
- *  - Quantized weights follow three layouts (bits b, group size gs):
+ *  - Quantized weights follow four layouts (bits b, group size gs):
  *      MLX affine   wq      uint32 [N, K*b/32]  codes packed along K, lowest bits
  *                                              = lowest column
  *                   scales  bf16   [N, K/gs]
