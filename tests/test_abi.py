@@ -84,12 +84,53 @@ def test_validation_codes(lib):
     assert gwb.lib().gwb_last_error().decode() != ""
 
 
+def test_validation_codes_of_the_next_step_entry_points(lib):
+    """Every case here fails (or is empty) before anything is launched."""
+    W = (OK16, OK16, OK16)
+    # fused decode products: at most 8 tokens, the affine layout rules, aligned x, outputs present
+    assert _st("gwb_gemv_gate_up", OK16, 9, *W, *W, 64, 512, 4, 64, OK16, OK16, NULL) == 2
+    assert _st("gwb_gemv_gate_up", OK16, 1, *W, *W, 64, 512, 3, 64, OK16, OK16, NULL) == 3
+    assert _st("gwb_gemv_gate_up", OK16, 1, *W, *W, 64, 96, 4, 64, OK16, OK16, NULL) == 2
+    assert _st("gwb_gemv_gate_up", OK16, 1, *W, *W, 64, 512, 4, 64, NULL, OK16, NULL) == 1
+    assert _st("gwb_gemv_gate_up", BAD, 1, *W, *W, 64, 512, 4, 64, OK16, OK16, NULL) == 4
+    assert _st("gwb_gemv_gate_up", NULL, 0, *W, *W, 64, 512, 4, 64, NULL, NULL, NULL) == 0
+    assert _st("gwb_gemv_silu_gate", OK16, OK16, 9, *W, 64, 512, 4, 64, OK16, NULL) == 2
+    assert _st("gwb_gemv_silu_gate", OK16, BAD, 1, *W, 64, 512, 4, 64, OK16, NULL) == 4
+    # K / group_size = 6 is not a multiple of 8: refused by the planner before any launch
+    assert _st("gwb_gemv_silu_gate", OK16, OK16, 1, *W, 64, 384, 4, 64, OK16, NULL) == 3
+    assert _st("gwb_gemv_silu_gate_resid", OK16, OK16, 1, *W, 64, 512, 4, 64, NULL, OK16, NULL) == 1
+    # fused W4A8 at decode
+    assert _st("gwb_gemv_w4a8", OK16, 9, OK16, OK16, 64, 512, OK16, NULL) == 2
+    assert _st("gwb_gemv_w4a8", OK16, 1, OK16, OK16, 64, 100, OK16, NULL) == 3
+    assert _st("gwb_gemv_w4a8", OK16, 1, OK16, OK16, 64, 32768, OK16, NULL) == 3
+    assert _st("gwb_gemv_w4a8", BAD, 1, OK16, OK16, 64, 512, OK16, NULL) == 4
+    assert _st("gwb_gemv_w4a8", NULL, 0, NULL, NULL, 64, 512, NULL, NULL) == 0
+    # W8A8
+    assert _st("gwb_qpack_sym_i8", OK16, 4, 40, OK16, OK16, NULL) == 2
+    assert _st("gwb_gemm_i8i8", OK16, OK16, 4, OK16, OK16, 64, 72, OK16, NULL, NULL) == 2
+    assert _st("gwb_gemm_i8i8", OK16, OK16, 4, OK16, OK16, 64, 262144, OK16, NULL, NULL) == 2
+    assert _st("gwb_gemm_i8i8", OK16, OK16, 4, OK16, OK16, 64, 128, NULL, NULL, NULL) == 1
+    assert _st("gwb_gemm_i8i8", BAD, OK16, 4, OK16, OK16, 64, 128, OK16, NULL, NULL) == 4
+    # AWQ: the GPTQ shape rules
+    assert _st("gwb_awq_dequant", OK16, OK16, OK16, 256, 12, 128, OK16, NULL) == 2
+    assert _st("gwb_awq_qmm", OK16, 1, OK16, OK16, OK16, 256, 16, 48, OK16, NULL) == 3
+
+
 def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 64, dtype=torch.bfloat16)
     wq = torch.zeros(8, 8, dtype=torch.int32)
     s = torch.zeros(8, 1, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         gwb.qmm_affine(x, wq, s, s, 4, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        gwb.gemv_gate_up(x, (wq, s, s), (wq, s, s), 4, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        gwb.gemv_silu_gate(x, x, wq, s, s, 4, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        gwb.gemv_w4a8(x, wq, torch.zeros(8))
+    with pytest.raises(ValueError, match="CUDA"):
+        gwb.gemm_i8i8(torch.zeros(1, 64, dtype=torch.int8), torch.zeros(1), torch.zeros(8, 64, dtype=torch.int8),
+                      torch.zeros(8))
 
 
 def test_oracle_builds_independently():
