@@ -10,12 +10,15 @@
 //
 // Work unit ("stage") = 16 output rows x 256 bytes of packed codes per row
 // (2048 / bits values of k), plus the scales and biases of those rows and
-// groups.  One CTA per SM (persistent) of 8 warps; a warp owns a contiguous
-// range of the CTA's stages and streams them through a private ring of D slots:
-//   * lane 0 issues, per stage, two TMA tile loads of the packed words (16 rows
-//     x 128 bytes each, 128-byte swizzle) and one TMA tile load each of the
-//     scale and bias boxes (16 rows x 8 or 16 groups), all completing on the
-//     slot's mbarrier, and refills a slot as soon as the warp has read it;
+// groups.  One CTA of 8 warps per SM (two when every warp gets at least four
+// stages), persistent; a warp owns a contiguous range of the CTA's stages and
+// streams them through a private ring of D slots:
+//   * lane 0 issues, per stage, one TMA load of the packed words as a 3-D box
+//     [2 segments][16 rows][128 bytes] (128-byte swizzle) and one of the scales
+//     and biases as a 3-D box over both arrays [2][16 rows][8 or 16 groups]
+//     (two 2-D loads each where the driver refuses those views), all
+//     completing on the slot's mbarrier, and refills a slot as soon as the
+//     warp has read it;
 //   * per stage the warp fetches the packed words with ldmatrix (lane c of a quad gets word c
 //     of each 16-byte chunk of its two rows), turns each code into an fp16
 //     value 1024 + code * 2^sigma with one LOP3 (two codes per register), and
