@@ -82,17 +82,16 @@ const char *gwb_last_error(void) { return gwb::g_msg; }
 const char *gwb_version(void) { return "group_wise_bit_b200 0.1 (sm_100a)"; }
 
 gwb_status gwb_check_device_error(void *stream) {
-  unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0, flag5 = 0, flag6 = 0, flag7 = 0, flag8 = 0, flag9 = 0;
+  unsigned int flag = 0, flag2 = 0, flag4 = 0, flag5 = 0, flag6 = 0, flag7 = 0, flag8 = 0, flag9 = 0;
   GWB_TRY(gwb::read_and_clear_device_error(as_stream(stream), &flag));
   GWB_TRY(gwb::read_and_clear_device_error_stream(as_stream(stream), &flag2));
-  GWB_TRY(gwb::read_and_clear_device_error_tmem(as_stream(stream), &flag3));
   GWB_TRY(gwb::read_and_clear_device_error_pipe(as_stream(stream), &flag4));
   GWB_TRY(gwb::read_and_clear_device_error_tc2(as_stream(stream), &flag5));
   GWB_TRY(gwb::read_and_clear_device_error_gate_up(as_stream(stream), &flag6));
   GWB_TRY(gwb::read_and_clear_device_error_silu(as_stream(stream), &flag7));
   GWB_TRY(gwb::read_and_clear_device_error_w4a8(as_stream(stream), &flag8));
   GWB_TRY(gwb::read_and_clear_device_error_i8w8(as_stream(stream), &flag9));
-  flag |= flag2 | flag3 | flag4 | flag5 | flag6 | flag7 | flag8 | flag9;
+  flag |= flag2 | flag4 | flag5 | flag6 | flag7 | flag8 | flag9;
   if (flag) return fail(GWB_ERR_TIMEOUT, "a bounded device-side wait gave up (flag 0x%x)", flag);
   return GWB_OK;
 }

@@ -66,10 +66,6 @@ gwb_status launch_gemv_silu_gate(const uint16_t *gate, const uint16_t *up, int M
                                  int gs, const uint16_t *resid, uint16_t *y, cudaStream_t st);
 // TMEM-operand tensor-core GEMV (the main decode kernel); GWB_ERR_UNSUPPORTED
 // (without a message) when the layout is outside what it covers.
-gwb_status launch_gemv_tmem(const uint16_t *x, int M, const uint32_t *wq, const uint16_t *scales,
-                            const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
-                            cudaStream_t st);
-gwb_status read_and_clear_device_error_tmem(cudaStream_t st, unsigned int *flag);
 gwb_status launch_gemv_gptq(const uint16_t *x, int M, const int32_t *qweight, const uint16_t *scales,
                             const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
                             uint16_t *y, cudaStream_t st, int zadd = 1);
