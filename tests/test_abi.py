@@ -68,6 +68,7 @@ def test_validation_codes(lib):
     # NULL and misaligned pointers
     assert _st("gwb_qmm_affine", OK16, 1, OK16, OK16, OK16, 64, 128, 4, 64, NULL, NULL) == 1
     assert _st("gwb_qmm_affine", OK16, 1, OK16, OK16, OK16, 64, 128, 4, 64, BAD, NULL) == 4
+    assert _st("gwb_qmm_affine", BAD, 1, OK16, OK16, OK16, 64, 128, 4, 64, OK16, NULL) == 4   # x
     assert _st("gwb_qpack_affine", BAD, 8, 64, 4, 64, OK16, OK16, OK16, NULL) == 4
     # empty problems are no-ops that succeed without launching anything
     assert _st("gwb_qmm_affine", NULL, 0, NULL, NULL, NULL, 64, 128, 4, 64, NULL, NULL) == 0
