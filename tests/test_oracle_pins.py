@@ -99,6 +99,28 @@ def test_dequant_affine_hand_case():
     assert w[0].tolist() == [-0.5, 0.0, 0.5, 1.0, 3.0, 1.0, -253.0, -507.0]
 
 
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_dequant_every_code_from_hand_packed_words(bits):
+    """Every code 0 .. 2^b - 1 of a bit width, packed into words by hand (numpy shifts written
+    here, lowest bits = lowest column), dequantizes to code * s + b exactly, with a different
+    power-of-two scale and bias per group: a wrong mask, shift or group index fails it."""
+    per = 32 // bits
+    ncode = 1 << bits
+    K = max(ncode, 64)
+    codes = np.arange(K) % ncode
+    words = np.zeros(K // per, np.uint64)
+    for k in range(K):
+        words[k // per] |= np.uint64(int(codes[k]) << ((k % per) * bits))
+    gs = 32
+    G = K // gs
+    s = 2.0 ** -np.arange(1, G + 1)
+    b = -(2.0 ** np.arange(G))
+    W = oracle.dequant_affine_f64(words.astype(np.uint32).reshape(1, -1), _bf16(s).reshape(1, G),
+                                  _bf16(b).reshape(1, G), 1, K, bits, gs)
+    g = np.arange(K) // gs
+    assert np.array_equal(W[0], codes * s[g] + b[g])
+
+
 # --------------------------------------------------------------------- affine quantizer
 @pytest.mark.parametrize("bits,gs", [(2, 32), (4, 64), (8, 128), (4, 32)])
 def test_qpack_affine_nearest_grid_bruteforce(bits, gs):
