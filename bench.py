@@ -5,8 +5,24 @@ MLX affine weights, group size 64): N x K in {2048x2048, 512x2048, 8192x2048,
 2048x8192, 128256x2048} at 4 bits, plus 8192x2048 at 2 and 8 bits.  The
 headline value is whole-job HBM throughput (algorithmic bytes: packed codes +
 bf16 scales and biases + activations + outputs, per call) in GB/s.  The same
-JSON line also carries the prefill GEMM at M = 2048 (4-bit, group size 64,
-shapes 4096x4096, 1024x4096, 14336x4096, 4096x14336) in TFLOP/s.
+JSON line carries the rest of the workloads, each with its roofline:
+
+  * prefill GEMM, 4-bit gs 64, shapes 4096x4096, 1024x4096, 14336x4096,
+    4096x14336 at M = 16 (GB/s), 128 (GB/s and TFLOP/s), 512 and 2048
+    (TFLOP/s); at M = 2048 also 8-bit gs 64 and 4-bit gs 32 / gs 128;
+  * GPTQ int4 (K = 4096, N = 11008, gs 128, with and without a permuted
+    g_idx): dequant (GB/s), qmm at M = 1 and 32 (GB/s) and 1024 (TFLOP/s);
+  * W4A8 and W8A8 on 4096x4096, 14336x4096, 4096x14336 at M = 8, 64 (GB/s)
+    and 512, 4096 (TOP/s); W8A8 at M = 1; the fused W4A8 decode product;
+  * the fused decode MLP of a Llama-3-8B layer (gate/up pair, silu product).
+
+Every workload is timed as a CUDA graph of back-to-back launches that rotate
+through enough copies of its weights that they exceed twice the L2 cache;
+the time per launch is the graph's device time (CUDA events) divided by the
+launches.  Before anything is timed, rank 0 at N = 1 runs the CPU baseline
+leg: the CPU oracle on sampled outputs of every workload (the bench's own
+device-drawn weights, copied to the host), which must match the GPU outputs
+(bit-exact integers, the float tolerance otherwise), else the run fails.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {gwb,reference}]
 
@@ -22,6 +38,7 @@ import json
 import math
 import os
 import statistics
+import sys
 import threading
 import time
 
@@ -35,8 +52,13 @@ DECODE = [  # (N, K, bits)
     (8192, 2048, 2), (8192, 2048, 8),
 ]
 PREFILL = [(4096, 4096), (1024, 4096), (14336, 4096), (4096, 14336)]
+PREFILL_M = (16, 128, 512, 2048)
+INT8_SHAPES = [(4096, 4096), (14336, 4096), (4096, 14336)]
+INT8_M = (8, 64, 512, 4096)
+GPTQ_K, GPTQ_N, GPTQ_GS = 4096, 11008, 128
 GS = 64
 M_PREFILL = 2048
+L2_BYTES = 126 * 2 ** 20
 METRIC = "qmm GB/s (M=1) and TFLOP/s (M=2048), % of roofline, 4-bit gs=64, 1 B200"
 WORKLOAD = ("decode GEMV sweep, M=1, bf16 x, MLX affine gs=64: 4-bit NxK 2048x2048, 512x2048, 8192x2048, "
             "2048x8192, 128256x2048; 2-bit and 8-bit 8192x2048")
@@ -48,8 +70,32 @@ def gemv_bytes(N, K, bits, M=1, gs=GS):
     return N * K * bits // 8 + 2 * 2 * N * (K // gs) + 2 * M * K + 2 * M * N
 
 
+def gptq_bytes(K, N, gs, M, g_idx):
+    """One GPTQ qmm call: int4 codes, fp16 scales, packed zeros, g_idx (if given), fp16 x and y."""
+    return K * N // 2 + 2 * N * (K // gs) + N * (K // gs) // 2 + (4 * K if g_idx else 0) + 2 * M * K + 2 * M * N
+
+
+def gptq_dequant_bytes(K, N, gs, g_idx):
+    """One GPTQ dequant call: the packed tensors in, the fp16 [N, K] weight out."""
+    return gptq_bytes(K, N, gs, 0, g_idx) + 2 * N * K
+
+
+def int8_bytes(N, K, M, wbits):
+    """One int8-activation GEMM call: weight codes, fp32 weight scales, int8 x, fp32 token scales, bf16 y."""
+    return N * K * wbits // 8 + 4 * N + M * K + 4 * M + 2 * M * N
+
+
 STEP_BYTES = sum(gemv_bytes(N, K, b) for N, K, b in DECODE)
 LMHEAD = (128256, 2048, 4)
+
+
+def copies_for(nbytes, cap=1 << 30):
+    """Weight copies a timing graph rotates through: their total exceeds twice the L2
+    (at least 2 copies, at most `cap` bytes unless 2 copies already pass it)."""
+    n = max(2, math.ceil(2 * L2_BYTES / max(nbytes, 1)) + 1)
+    while n > 2 and n * nbytes > cap:
+        n -= 1
+    return n
 
 
 def peaks():
@@ -80,8 +126,9 @@ class ClockSampler:
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index):
+    def __init__(self, index, period_s=0.0002):
         self.index, self.samples, self.reasons, self.max_mhz = index, [], set(), None
+        self.period = period_s
         self._stop = threading.Event()
         self._t = None
 
@@ -108,7 +155,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(self.period)
 
     def __exit__(self, *a):
         self._stop.set()
@@ -159,16 +206,67 @@ def job_gbs(world, bytes_per_step, steps, ms_max):
     return world * bytes_per_step * steps / (ms_max * 1e-3) / 1e9
 
 
-# ------------------------------------------------------------------ GPU arm
+def roofline(kernel, bound, achieved, peak, unit, peak_source, traffic=None, **extra):
+    out = {"kernel": kernel, "bound": bound, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
+           "frac": round(achieved / peak, 4), "peak_source": peak_source, "traffic": traffic}
+    out.update(extra)
+    return out
+
+
+# ------------------------------------------------------------------ GPU timing helpers
+def graph_us(launch, n, stream, replays=3):
+    """Device time per launch of a CUDA graph of `n` back-to-back launch(i), i = 0 .. n-1
+    (CUDA events around `replays` replays, after one untimed replay)."""
+    with torch.cuda.stream(stream):
+        for i in range(min(n, 2)):
+            launch(i)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                launch(i)
+        g.replay()
+        stream.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(replays):
+            g.replay()
+        b.record(stream)
+        b.synchronize()
+    us = a.elapsed_time(b) * 1e3 / (n * replays)
+    del g
+    return us
+
+
+def dev_weight(dev, N, K, seed):
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    return torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+
+
+def clone_all(ts, n):
+    """n copies of a tuple of tensors (copy 0 is the original)."""
+    return [ts] + [tuple(t.clone() for t in ts) for _ in range(n - 1)]
+
+
+# ------------------------------------------------------------------ workloads
+class Work:
+    """One timed workload: `launch(i)` runs the product on weight copy i (of n); `nbytes` and
+    `flops` are its algorithmic bytes and operations per launch; each of `checks` returns the
+    host copy of copy 0's output and inputs for the CPU baseline leg's comparison."""
+
+    def __init__(self, key, launch, n, nbytes, flops, kernel, checks=()):
+        self.key, self.launch, self.n, self.nbytes, self.flops = key, launch, n, nbytes, flops
+        self.kernel, self.checks = kernel, list(checks)
+
+
 def build_decode(gwb, dev, n_sets=2):
     """Quantizes every decode weight on the device (seeded N(0, 0.02)); n_sets copies rotate."""
     sets = []
     for s in range(n_sets):
         layers = []
         for i, (N, K, bits) in enumerate(DECODE):
-            g = torch.Generator(device=dev)
-            g.manual_seed(1000 * s + i)
-            w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+            w = dev_weight(dev, N, K, 1000 * s + i)
             wq, sc, bi = gwb.qpack_affine(w, bits, GS)
             del w
             x = synth.activations(1, K, seed=1).to(dev)
@@ -179,43 +277,315 @@ def build_decode(gwb, dev, n_sets=2):
     return sets
 
 
+def affine_work(gwb, dev, key, shapes, M, bits, gs, kernel, seed0=77):
+    """qmm_affine at M tokens over several N x K shapes (one Work per shape)."""
+    works = []
+    for j, (N, K) in enumerate(shapes):
+        w = dev_weight(dev, N, K, seed0 + j)
+        wt = gwb.qpack_affine(w, bits, gs)
+        del w
+        wbytes = gemv_bytes(N, K, bits, M=0, gs=gs)
+        cps = clone_all(wt, copies_for(wbytes))
+        x = synth.activations(M, K, seed=1, outlier_frac=0.01)
+        xd = x.to(dev)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+        def launch(i, cps=cps, xd=xd, y=y, bits=bits, gs=gs):
+            wq, sc, bi = cps[i % len(cps)]
+            gwb.qmm_affine(xd, wq, sc, bi, bits, gs, y=y)
+
+        def check(cps=cps, x=x, y=y, N=N, K=K, M=M, bits=bits, gs=gs):
+            return ("affine", dict(x=x, w=tuple(t.cpu() for t in cps[0]), y=y.cpu(), N=N, K=K, M=M, bits=bits,
+                                   gs=gs))
+
+        works.append(Work(f"{key} {N}x{K}", launch, len(cps), gemv_bytes(N, K, bits, M=M, gs=gs), 2.0 * M * N * K,
+                          kernel, [check]))
+    return works
+
+
+def gptq_work(gwb, dev, M, permuted, dequant=False):
+    K, N, gs = GPTQ_K, GPTQ_N, GPTQ_GS
+    qw, sc, qz, gi = synth.gptq_quartet(K, N, gs, seed=0, permuted=permuted)
+    d = (qw.to(dev), sc.to(dev), qz.to(dev))
+    gid = gi.to(dev) if permuted else None
+    cps = clone_all(d, copies_for(gptq_bytes(K, N, gs, 0, permuted)))
+    if dequant:
+        out = torch.empty((N, K), dtype=torch.float16, device=dev)
+
+        def launch(i):
+            q, s, z = cps[i % len(cps)]
+            gwb.gptq_dequant(q, s, z, gid, gs, out=out)
+
+        def check():
+            return ("gptq_dequant", dict(h=(qw, sc, qz, gi if permuted else None), y=out.cpu(), K=K, N=N, gs=gs))
+
+        return Work(f"gptq dequant perm={int(permuted)}", launch, len(cps), gptq_dequant_bytes(K, N, gs, permuted),
+                    0.0, "k_gptq_dequant", [check])
+    x = synth.activations(M, K, seed=1, dtype=torch.float16)
+    xd = x.to(dev)
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+
+    def launch(i):
+        q, s, z = cps[i % len(cps)]
+        gwb.gptq_qmm(xd, q, s, z, gid, gs, y=y)
+
+    def check():
+        return ("gptq", dict(x=x, h=(qw, sc, qz, gi if permuted else None), y=y.cpu(), K=K, N=N, gs=gs, M=M))
+
+    kern = "k_gemv_gptq" if M <= 8 else ("k_tc2<Gptq>" if M > 128 and not permuted else "k_tc<Gptq>")
+    return Work(f"gptq M={M} perm={int(permuted)}", launch, len(cps), gptq_bytes(K, N, gs, M, permuted),
+                2.0 * M * N * K, kern, [check])
+
+
+def int8_work(gwb, dev, fmt, shapes, M):
+    works = []
+    for j, (N, K) in enumerate(shapes):
+        w = dev_weight(dev, N, K, 91 + j)
+        wt = gwb.qpack_sym_i4(w) if fmt == "w4a8" else gwb.qpack_sym_i8(w)
+        del w
+        wbits = 4 if fmt == "w4a8" else 8
+        cps = clone_all(wt, copies_for(N * K * wbits // 8))
+        x = synth.activations(M, K, seed=1)
+        qx, sx = gwb.quant_per_token_i8(x.to(dev))
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        gemm = gwb.gemm_i8i4 if fmt == "w4a8" else gwb.gemm_i8i8
+
+        def launch(i, cps=cps, qx=qx, sx=sx, y=y, gemm=gemm):
+            wq, sw = cps[i % len(cps)]
+            gemm(qx, sx, wq, sw, y=y)
+
+        def check(cps=cps, qx=qx, sx=sx, x=x, y=y, N=N, K=K, gemm=gemm, fmt=fmt):
+            _, acc = gemm(qx, sx, cps[0][0], cps[0][1], want_y=False, want_acc=True)
+            return (fmt, dict(x=x, qx=qx.cpu(), sx=sx.cpu(), w=tuple(t.cpu() for t in cps[0]), y=y.cpu(),
+                              acc=acc.cpu(), N=N, K=K))
+
+        if fmt == "w4a8":
+            kern = "k_tc2<I8,4,256,pair>" if M >= 128 else "k_tc<I8>"
+        else:
+            kern = "k_gemv_pipe<8,64,M,i8w8>" if M <= 8 and K % 512 == 0 else "k_tc2<W8>"
+        works.append(Work(f"{fmt} {N}x{K} M={M}", launch, len(cps), int8_bytes(N, K, M, wbits), 2.0 * M * N * K,
+                          kern, [check]))
+    return works
+
+
+def run_works(works, stream):
+    """Times each Work's graph; returns [(work, us per launch)]."""
+    return [(w, graph_us(w.launch, w.n, stream)) for w in works]
+
+
+def aggregate(key, timed, peak, peak_source, unit, bound, traffic=None, extra=None):
+    """Sum of work over sum of time across a workload's shapes, with its roofline."""
+    work = (lambda w: w.nbytes) if bound == "hbm" else (lambda w: w.flops)
+    scale = 1e3 if bound == "hbm" else 1e6          # bytes/us -> GB/s; ops/us -> T(FL)OP/s
+    tot_us = sum(us for _, us in timed)
+    val = sum(work(w) for w, _ in timed) / tot_us / scale
+    kernels = sorted({w.kernel for w, _ in timed})
+    out = {"value": round(val, 1), "unit": unit,
+           "shapes": [{"case": w.key, "us": round(us, 2), unit: round(work(w) / us / scale, 1)} for w, us in timed],
+           "roofline": roofline(" + ".join(kernels), bound, val, peak, unit, peak_source, traffic)}
+    if extra:
+        out.update(extra)
+    return out
+
+
+# ------------------------------------------------------------------ CPU baseline leg (oracle)
+def _rows_of(M):
+    """The sampled rows of a bench workload's output: first, middle, last."""
+    return np.unique(np.array([0, M // 2, M - 1] if M > 2 else list(range(M)), dtype=np.int64))
+
+
+def _w16(t):
+    """Raw 16-bit patterns (np.uint16) of a bf16 / fp16 torch tensor, or the words of an int32 one."""
+    if t.dtype in (torch.bfloat16, torch.float16):
+        return synth.bits16(t)
+    return t.numpy()
+
+
+def check_item(item):
+    """Compares one workload's GPU output (copied to the host) with the CPU oracle on sampled
+    rows; raises AssertionError on a mismatch.  item = (kind, dict of host tensors and sizes)."""
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from tol import check_float
+
+    kind, d = item
+    if kind == "affine":
+        wq, sc, bi = (_w16(t) for t in d["w"])
+        wq = wq.view(np.uint32)
+        r = _rows_of(d["M"])
+        ref = oracle.qmm_affine(synth.bits16(d["x"]), wq, sc, bi, d["N"], d["K"], d["bits"], d["gs"], rows=r)
+        s = oracle.bf16_array_to_f64(sc)
+        b = oracle.bf16_array_to_f64(bi)
+        wmax = float(np.max(np.maximum(np.abs(b), np.abs(b + ((1 << d["bits"]) - 1) * s))))
+        check_float(d["y"].float().numpy()[r], ref, d["K"], wmax, float(d["x"].float().abs().max()),
+                    f"affine {d['N']}x{d['K']} b{d['bits']} gs{d['gs']} M={d['M']}")
+    elif kind == "gptq":
+        qw, sc, qz, gi = d["h"]
+        h = (qw.numpy(), synth.bits16(sc), qz.numpy(), None if gi is None else gi.numpy())
+        r = _rows_of(d["M"])
+        ref = oracle.gptq_qmm(synth.bits16(d["x"]), *h, d["K"], d["N"], d["gs"], rows=r)
+        # an upper bound of max|w|: scale * 16 (|code - zero| <= 15 under the "+1" convention)
+        wmax = float(sc.float().abs().max()) * 16
+        check_float(d["y"].float().numpy()[r], ref, d["K"], wmax, float(d["x"].float().abs().max()),
+                    f"gptq M={d['M']}")
+    elif kind == "gptq_dequant":
+        qw, sc, qz, gi = d["h"]
+        ref = oracle.gptq_dequant_f16(qw.numpy(), synth.bits16(sc), qz.numpy(), None if gi is None else gi.numpy(),
+                                      d["K"], d["N"], d["gs"])
+        if not np.array_equal(synth.bits16(d["y"]), ref):
+            raise AssertionError("gptq_dequant: fp16 weights differ")
+    elif kind in ("w4a8", "w8a8"):
+        qx, sx = d["qx"].numpy(), d["sx"].numpy()
+        qx_o, sx_o = oracle.quant_per_token_i8(synth.bits16(d["x"]))
+        if not (np.array_equal(qx, qx_o) and np.array_equal(sx, sx_o)):
+            raise AssertionError(f"{kind}: per-token int8 activations differ")
+        wq, sw = (t.numpy() for t in d["w"])
+        r = _rows_of(qx.shape[0])
+        if kind == "w4a8":
+            acc_o, y_o, ovf = oracle.gemm_i8i4(qx, sx, wq.view(np.uint32), sw, d["N"], d["K"], rows=r)
+            wmax = float(np.abs(sw).max() * 7)
+        else:
+            acc_o, y_o, ovf = oracle.gemm_i8i8(qx, sx, wq, sw, d["N"], d["K"], rows=r)
+            wmax = float(np.abs(sw).max() * 127)
+        if ovf or not np.array_equal(d["acc"].numpy().astype(np.int64)[r], acc_o):
+            raise AssertionError(f"{kind} {d['N']}x{d['K']}: int32 accumulators differ")
+        check_float(d["y"].float().numpy()[r], y_o, d["K"], wmax, float(d["x"].float().abs().max()),
+                    f"{kind} {d['N']}x{d['K']} M={qx.shape[0]}")
+    else:
+        raise ValueError(f"unknown check kind {kind}")
+    return True
+
+
+def cpu_leg(checks, sets, budget_s, threads):
+    """The CPU oracle on bounded samples: first timed over the decode sweep on the bench's own
+    weights (rows 0 .. n of every layer, single thread), then compared with every workload's
+    GPU output on sampled rows (bit-exact integers; the float tolerance otherwise, the same as
+    the parity tests).  Returns (cpu_baseline dict, parity dict)."""
+    import concurrent.futures as cf
+
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from tol import check_float
+
+    def bf16_max_w(sc, bi, bits):
+        s = oracle.bf16_array_to_f64(sc)
+        b = oracle.bf16_array_to_f64(bi)
+        return float(np.max(np.maximum(np.abs(b), np.abs(b + ((1 << bits) - 1) * s))))
+
+    # ---- timed: the decode sweep on a row sample of weight set 0
+    frac = 0.25
+    layers = []
+    for (wq, sc, bi, x, y, bits), (N, K, _) in zip(sets[0], DECODE):
+        n = max(8, int(N * frac))
+        layers.append((synth.bits16(x.cpu()), wq[:n].cpu().numpy().view(np.uint32), synth.bits16(sc[:n].cpu()),
+                       synth.bits16(bi[:n].cpu()), n, K, bits, y.cpu()))
+    t0 = time.perf_counter()
+    nbytes, passes, refs = 0, 0, None
+    while passes < 1 or time.perf_counter() - t0 < budget_s:
+        refs = []
+        for xh, wq, sc, bi, n, K, bits, _ in layers:
+            refs.append(oracle.qmm_affine(xh, wq, sc, bi, n, K, bits, GS))
+            nbytes += gemv_bytes(n, K, bits)
+        passes += 1
+    dt = time.perf_counter() - t0
+    cpu = {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": f"{passes} pass(es) over the first {frac:.0%} of the output rows of every decode layer "
+                     f"(M=1, gs=64, the bench's own weights), single-threaded C, fp64, {dt:.1f} s"}
+
+    failures, checked = [], 0
+    for (xh, wq, sc, bi, n, K, bits, yg), ref, (N, _, _) in zip(layers, refs, DECODE):
+        try:
+            check_float(yg.float().numpy()[:, :n], ref, K, bf16_max_w(sc, bi, bits),
+                        float(np.abs(oracle.bf16_array_to_f64(xh)).max()), f"decode {N}x{K} b{bits}")
+            checked += 1
+        except AssertionError as e:
+            failures.append(str(e))
+
+    # ---- every other workload, on sampled rows (threads: the oracle's C calls release the GIL)
+    with cf.ThreadPoolExecutor(max(1, threads)) as ex:
+        futs = [ex.submit(check_item, c) for c in checks]
+        for f in futs:
+            try:
+                f.result()
+                checked += 1
+            except Exception as e:   # a mismatch, or a check that could not run: both fail the line
+                failures.append(f"{type(e).__name__}: {e}")
+    parity = {"checked": checked, "failed": len(failures), "ok": not failures,
+              "how": "CPU oracle on sampled rows of every workload before timing (bit-exact integers, "
+                     "max-abs 2e-2*sqrt(K)*max|w|*max|x| and rel. Frobenius 5e-3 for floats)"}
+    if failures:
+        parity["failures"] = failures[:10]
+    return cpu, parity
+
+
+# ------------------------------------------------------------------ GPU arm
 def run_gpu(args, world, rank, local):
     import group_wise_bit_b200 as gwb
 
     dev = torch.device("cuda", local)
     hbm_peak, bf16_peak, peak_kind = peaks()
+    hbm_src = f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback"
+    bf16_src = f"{peak_kind} (MEASURED_PEAKS.json bf16_tflops, burst)" if peak_kind == "measured" else "fallback"
+    stream = torch.cuda.Stream(device=dev)
     sets = build_decode(gwb, dev)
     lm_idx = DECODE.index(LMHEAD)
+    full = not args.no_prefill
 
-    # One CUDA graph per step: [event] lm_head GEMV [event] the six other GEMVs, with
-    # programmatic launch chaining the GEMVs.  Each step has its own graph and its
-    # own event-record nodes, so the lm_head launch of every timed step is timed on
-    # the device; consecutive steps alternate between the two weight sets.
-    n_graphs = max(args.steps, 1)
-    stream = torch.cuda.Stream(device=dev)
-    graphs, lm_events = [], []
+    # ---- every other workload: set up, run once (the CPU leg compares these outputs)
+    groups = {}
+    if full:
+        pk = "k_tc2<Affine,4,256,pair,A in TMEM>"
+        groups["prefill_m16"] = affine_work(gwb, dev, "prefill M=16", PREFILL, 16, 4, GS, "k_tc<Affine>")
+        groups["prefill_m128"] = affine_work(gwb, dev, "prefill M=128", PREFILL, 128, 4, GS, "k_tc2<Affine,4,128>")
+        groups["prefill_m512"] = affine_work(gwb, dev, "prefill M=512", PREFILL, 512, 4, GS, pk)
+        groups["prefill_m2048"] = affine_work(gwb, dev, "prefill M=2048", PREFILL, M_PREFILL, 4, GS, pk)
+        groups["prefill_m2048_b8"] = affine_work(gwb, dev, "prefill M=2048 8-bit", PREFILL, M_PREFILL, 8, GS,
+                                                 "k_tc2<Affine,8,256,pair,A in TMEM>")
+        groups["prefill_m2048_gs32"] = affine_work(gwb, dev, "prefill M=2048 gs32", PREFILL, M_PREFILL, 4, 32, pk)
+        groups["prefill_m2048_gs128"] = affine_work(gwb, dev, "prefill M=2048 gs128", PREFILL, M_PREFILL, 4, 128, pk)
+        groups["gptq_dequant"] = [gptq_work(gwb, dev, 0, p, dequant=True) for p in (False, True)]
+        for M in (1, 32, 1024):
+            groups[f"gptq_m{M}"] = [gptq_work(gwb, dev, M, p) for p in (False, True)]
+        for fmt in ("w4a8", "w8a8"):
+            for M in INT8_M:
+                groups[f"{fmt}_m{M}"] = int8_work(gwb, dev, fmt, INT8_SHAPES, M)
+        groups["w8a8_m1"] = int8_work(gwb, dev, "w8a8", [(14336, 4096)], 1)
     with torch.cuda.stream(stream):
         for layers in sets:
-            for (wq, sc, bi, x, y, bits) in layers:           # warm the launch path before capture
+            for (wq, sc, bi, x, y, bits) in layers:
                 gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+        for ws in groups.values():
+            for w in ws:
+                w.launch(0)
+    torch.cuda.synchronize()
+    gwb.check_device_error()
+
+    # ---- CPU baseline leg: the oracle, timed, and compared with the outputs above
+    cpu, parity = None, None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        with torch.cuda.stream(stream):
+            checks = [c() for ws in groups.values() for w in ws for c in w.checks]
+        torch.cuda.synchronize()
+        cpu, parity = cpu_leg(checks, sets, args.cpu_seconds, threads=min(16, os.cpu_count() or 1))
+        if not parity["ok"]:
+            print(json.dumps({"metric": METRIC, "error": "parity check before timing failed", "parity": parity}),
+                  flush=True)
+            sys.exit(1)
+
+    # ---- the decode step: one CUDA graph per step of the seven GEMVs (programmatic launch
+    # chains them); consecutive steps alternate between the two weight sets
+    n_graphs = max(args.steps, 1)
+    graphs = []
+    with torch.cuda.stream(stream):
         torch.cuda.synchronize()
         for gi in range(n_graphs):
             layers = sets[gi % len(sets)]
-            ev = (torch.cuda.Event(enable_timing=True, external=True),
-                  torch.cuda.Event(enable_timing=True, external=True))
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                wq, sc, bi, x, y, bits = layers[lm_idx]
-                ev[0].record(stream)
-                gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
-                ev[1].record(stream)
-                for i, (wq, sc, bi, x, y, bits) in enumerate(layers):
-                    if i != lm_idx:
-                        gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+                for (wq, sc, bi, x, y, bits) in layers:
+                    gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
             graphs.append(g)
-            lm_events.append(ev)
     torch.cuda.synchronize()
-
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             graphs[i % n_graphs].replay()
@@ -236,23 +606,38 @@ def run_gpu(args, world, rank, local):
     ms_max = max_over_ranks(ms, world)
     ms_step = ms_max / args.steps
     value = job_gbs(world, STEP_BYTES, args.steps, ms_max)
-    lm_ms = float(np.mean([a.elapsed_time(b) for a, b in lm_events[:args.steps]]))
-    lm_bytes = gemv_bytes(*LMHEAD)
-    achieved = lm_bytes / (lm_ms * 1e-3) / 1e9
     del graphs
 
-    # End to end through the public API: pinned host x -> device, qmm, y -> pinned host, every layer.
-    host_x = [l[3].cpu().pin_memory() for l in sets[0]]
-    host_y = [torch.empty(l[4].shape, dtype=torch.bfloat16).pin_memory() for l in sets[0]]
-    h2d = sum(t.numel() * 2 for t in host_x)
-    d2h = sum(t.numel() * 2 for t in host_y)
+    # ---- the dominant kernel alone: the lm_head GEMV in a graph of back-to-back launches
+    # alternating the two weight sets (296 MB, over twice the L2)
+    def lm_launch(i):
+        wq, sc, bi, x, y, bits = sets[i % 2][lm_idx]
+        gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+
+    lm_us = graph_us(lm_launch, 20, stream, replays=5)
+    lm_bytes = gemv_bytes(*LMHEAD)
+    achieved = lm_bytes / (lm_us * 1e-6) / 1e9
+
+    # ---- end to end through the public API: per step one H2D copy of the seven activation
+    # vectors from pinned host memory, the seven qmm_affine calls, one D2H copy of the outputs
+    Ks = [K for _, K, _ in DECODE]
+    Ns = [N for N, _, _ in DECODE]
+    xoff = np.concatenate([[0], np.cumsum(Ks)])
+    yoff = np.concatenate([[0], np.cumsum(Ns)])
+    host_x = torch.cat([l[3].cpu().reshape(-1) for l in sets[0]]).pin_memory()
+    host_y = torch.empty(int(yoff[-1]), dtype=torch.bfloat16).pin_memory()
+    dev_x = torch.empty_like(host_x, device=dev)
+    dev_y = torch.empty(int(yoff[-1]), dtype=torch.bfloat16, device=dev)
+    xs = [dev_x[xoff[j]:xoff[j + 1]].view(1, -1) for j in range(len(DECODE))]
+    ys = [dev_y[yoff[j]:yoff[j + 1]].view(1, -1) for j in range(len(DECODE))]
+    h2d, d2h = host_x.numel() * 2, host_y.numel() * 2
 
     def e2e_step(i):
         layers = sets[i % len(sets)]
-        for j, (wq, sc, bi, x, y, bits) in enumerate(layers):
-            x.copy_(host_x[j], non_blocking=True)
-            gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
-            host_y[j].copy_(y, non_blocking=True)
+        dev_x.copy_(host_x, non_blocking=True)
+        for j, (wq, sc, bi, _, _, bits) in enumerate(layers):
+            gwb.qmm_affine(xs[j], wq, sc, bi, bits, GS, y=ys[j])
+        host_y.copy_(dev_y, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -270,39 +655,69 @@ def run_gpu(args, world, rank, local):
     e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = job_gbs(world, STEP_BYTES, args.steps, e_ms)
 
-    prefill = run_prefill(gwb, dev, stream, bf16_peak, peak_kind) if not args.no_prefill else None
-    int8 = {}
-    int8["decode_mlp_fused"] = run_mlp_fused(gwb, dev, stream, hbm_peak)
-    int8["w4a8_decode_fused"] = run_w4a8_decode(gwb, dev, stream, hbm_peak)
-    if not args.no_prefill:
-        i8peak = int8_peak_tops(dev, stream)
-        int8["w4a8_m4096"] = run_int8(gwb, dev, stream, "w4a8", 14336, 4096, 4096, i8peak, hbm_peak)
-        int8["w8a8_m4096"] = run_int8(gwb, dev, stream, "w8a8", 14336, 4096, 4096, i8peak, hbm_peak)
-        int8["w8a8_m1"] = run_int8(gwb, dev, stream, "w8a8", 14336, 4096, 1, i8peak, hbm_peak)
-
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": 1, "group_size": GS, "bytes_per_step": STEP_BYTES,
                    "l2": "inputs larger than L2: 192 MB of weights per step, two weight sets rotate (384 MB)",
-                   "graphs": "each step replays its own CUDA graph of the seven GEMVs (lm_head first, bracketed by event nodes)",
+                   "graphs": "each step replays its own CUDA graph of the seven GEMVs",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "k_gemv_pipe<4,64,1> (lm_head 128256x2048)", "bound": "hbm",
-                     "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "peak_source": peak_kind,
-                     "bytes_per_launch": lm_bytes, "avg_launch_us": round(lm_ms * 1e3, 2),
-                     "traffic": traffic_for("k_gemv_pipe_lmhead")},
+        "roofline": roofline("k_gemv_pipe<4,64,1> (lm_head 128256x2048)", "hbm", achieved, hbm_peak, "GB/s", hbm_src,
+                             traffic_for("k_gemv_pipe_lmhead"), bytes_per_launch=lm_bytes,
+                             avg_launch_us=round(lm_us, 2),
+                             timing="CUDA graph of 20 back-to-back lm_head launches alternating two weight sets "
+                                    "(296 MB), events around 5 replays"),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "note": "weights resident in HBM; per layer: H2D of x, qmm_affine call, D2H of y"},
+                "note": "weights resident in HBM; per step: one H2D copy of the 7 activation vectors (pinned), "
+                        "7 qmm_affine calls through the public API, one D2H copy of the 7 outputs"},
         "gpu_launches": len(DECODE) * args.steps,
         "clocks": clk.summary(),
     }
-    if prefill:
-        out["prefill_m2048"] = prefill
-    out.update(int8)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    if parity is not None:
+        out["parity"] = parity
+
+    if full:
+        i8peak = int8_peak_tops(dev, stream)
+        i8src = "measured in this run: torch._int_mm 8192^3 int8, best of 5"
+        t = {k: run_works(ws, stream) for k, ws in groups.items()}
+        for M in PREFILL_M:
+            key = f"prefill_m{M}"
+            if M <= 128:
+                out[key] = aggregate(key, t[key], hbm_peak, hbm_src, "GB/s", "hbm",
+                                     traffic=traffic_for(f"k_tc_affine4_m{M}"))
+            if M >= 128:
+                k2 = key if M > 128 else key + "_tflops"
+                out[k2] = aggregate(key, t[key], bf16_peak, bf16_src, "TFLOP/s", "tensor",
+                                    traffic=traffic_for(f"k_tc2_affine4_m{M}"))
+        for key in ("prefill_m2048_b8", "prefill_m2048_gs32", "prefill_m2048_gs128"):
+            out[key] = aggregate(key, t[key], bf16_peak, bf16_src, "TFLOP/s", "tensor")
+        out["gptq_dequant"] = aggregate("gptq_dequant", t["gptq_dequant"], hbm_peak, hbm_src, "GB/s", "hbm")
+        for M in (1, 32, 1024):
+            key = f"gptq_m{M}"
+            tm = t[key]
+            if M >= 512:
+                out[key] = aggregate(key, tm[:1], bf16_peak, bf16_src + " (fp16 peak taken equal to bf16)",
+                                     "TFLOP/s", "tensor", extra={"permuted_g_idx": aggregate(
+                                         key, tm[1:], bf16_peak, bf16_src, "TFLOP/s", "tensor")})
+            else:
+                out[key] = aggregate(key, tm[:1], hbm_peak, hbm_src, "GB/s", "hbm",
+                                     extra={"permuted_g_idx": aggregate(key, tm[1:], hbm_peak, hbm_src, "GB/s", "hbm")})
+        for fmt in ("w4a8", "w8a8"):
+            for M in INT8_M:
+                key = f"{fmt}_m{M}"
+                if M >= 512:
+                    out[key] = aggregate(key, t[key], i8peak, i8src, "TOP/s", "tensor",
+                                         traffic=traffic_for(f"k_tc2_{fmt}_m{M}"))
+                else:
+                    out[key] = aggregate(key, t[key], hbm_peak, hbm_src, "GB/s", "hbm")
+        out["w8a8_m1"] = aggregate("w8a8_m1", t["w8a8_m1"], hbm_peak, hbm_src, "GB/s", "hbm")
+        out["int8_peak_tops"] = round(i8peak, 1)
+    out["decode_mlp_fused"] = run_mlp_fused(gwb, dev, stream, hbm_peak, hbm_src)
+    out["w4a8_decode_fused"] = run_w4a8_decode(gwb, dev, stream, hbm_peak, hbm_src)
+    if cpu is not None:
+        out["cpu_baseline"] = cpu
+    gwb.check_device_error()
     if rank == 0:
         print(json.dumps(out), flush=True)
 
@@ -327,9 +742,7 @@ def int8_peak_tops(dev, stream, reps=5):
 
 def int8_operands(gwb, dev, fmt, N, K, M, seed=91):
     """Quantized weights (fmt 'w4a8': int4 codes, 'w8a8': int8) and per-token int8 activations."""
-    g = torch.Generator(device=dev)
-    g.manual_seed(seed)
-    w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+    w = dev_weight(dev, N, K, seed)
     wq, sw = gwb.qpack_sym_i4(w) if fmt == "w4a8" else gwb.qpack_sym_i8(w)
     del w
     x = synth.activations(M, K, seed=1).to(dev)
@@ -341,187 +754,68 @@ def int8_gemm(gwb, fmt):
     return gwb.gemm_i8i4 if fmt == "w4a8" else gwb.gemm_i8i8
 
 
-def run_int8(gwb, dev, stream, fmt, N, K, M, int8_peak, hbm_peak, reps=5):
-    """int8-activation GEMM (fmt 'w4a8' or 'w8a8', int32 accumulation, bf16 out) on an N x K
-    weight at M tokens, each launch timed alone with an L2 flush before it.  M = 1 is
-    HBM-bound (bytes = weights + scales + activations + output); larger M is tensor-bound
-    (ops = 2 M N K)."""
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
-    wq, sw, qx, sx = int8_operands(gwb, dev, fmt, N, K, M)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    gemm = int8_gemm(gwb, fmt)
-    ts = []
-    with torch.cuda.stream(stream):
-        for r in range(reps + 2):
-            flush.fill_(r)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            gemm(qx, sx, wq, sw, y=y)
-            b.record(stream)
-            b.synchronize()
-            if r >= 2:
-                ts.append(a.elapsed_time(b))
-    ms = statistics.median(ts)
-    if fmt == "w4a8":
-        kern = "k_tc2<I8,4,256,pair,A in TMEM> (kind::i8)"
-    elif M <= 8 and K % 512 == 0:
-        kern = "k_gemv_pipe<8,64,%d,i8w8> (int8 x int8 weight streaming, exact int32 sums)" % (M,)
-    else:
-        kern = "k_tc2<W8,8,%s> (kind::i8, both operands by TMA)" % ("256,pair" if M > 128 else "128" if M > 32 else "32")
-    out = {"N": N, "K": K, "M": M, "us": round(ms * 1e3, 1)}
-    if M <= 8:
-        wbytes = N * K // (2 if fmt == "w4a8" else 1)
-        nbytes = wbytes + N * 4 + M * K + M * 4 + M * N * 2
-        gbs = nbytes / (ms * 1e-3) / 1e9
-        out.update({"value": round(gbs, 1), "unit": "GB/s",
-                    "roofline": {"kernel": kern, "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak,
-                                 "unit": "GB/s", "frac": round(gbs / hbm_peak, 4), "bytes_per_launch": nbytes,
-                                 "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}})
-    else:
-        tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
-        out.update({"value": round(tops, 1), "unit": "TOP/s",
-                    "roofline": {"kernel": kern, "bound": "tensor", "achieved": round(tops, 1),
-                                 "peak": round(int8_peak, 1), "unit": "TOP/s", "frac": round(tops / int8_peak, 4),
-                                 "peak_source": "measured in this run: torch._int_mm 8192^3 int8, best of 5",
-                                 "traffic": traffic_for(f"k_tc2_{fmt}_m{M}")}})
-    return out
-
-
-def run_prefill(gwb, dev, stream, bf16_peak, peak_kind, reps=5):
-    """M = 2048 prefill GEMMs (4-bit, gs 64), each launch timed alone with an L2 flush before it."""
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
-    total_flop, total_ms, per = 0.0, 0.0, []
-    for i, (N, K) in enumerate(PREFILL):
-        g = torch.Generator(device=dev)
-        g.manual_seed(77 + i)
-        w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
-        wq, sc, bi = gwb.qpack_affine(w, 4, GS)
-        del w
-        x = synth.activations(M_PREFILL, K, seed=1, outlier_frac=0.01).to(dev)
-        y = torch.empty((M_PREFILL, N), dtype=torch.bfloat16, device=dev)
-        ts = []
-        with torch.cuda.stream(stream):
-            for r in range(reps + 2):
-                flush.fill_(r)
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                gwb.qmm_affine(x, wq, sc, bi, 4, GS, y=y)
-                b.record(stream)
-                b.synchronize()
-                if r >= 2:
-                    ts.append(a.elapsed_time(b))
-        ms = statistics.median(ts)
-        flop = 2.0 * M_PREFILL * N * K
-        total_flop += flop
-        total_ms += ms
-        per.append({"N": N, "K": K, "us": round(ms * 1e3, 1), "tflops": round(flop / (ms * 1e-3) / 1e12, 1)})
-    tf = total_flop / (total_ms * 1e-3) / 1e12
-    return {"value": round(tf, 1), "unit": "TFLOP/s", "M": M_PREFILL, "bits": 4, "group_size": GS,
-            "l2": "256 MB buffer written before every timed launch",
-            "roofline": {"kernel": "k_tc2<Affine,4,256,pair,A in TMEM> (persistent, stream-K)", "bound": "tensor",
-                         "achieved": round(tf, 1),
-                         "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(tf / bf16_peak, 4),
-                         "peak_source": peak_kind, "traffic": traffic_for("k_tc2_affine4_m2048")},
-            "shapes": per}
-
-
-def run_w4a8_decode(gwb, dev, stream, hbm_peak, N=14336, K=4096, M=1, reps=20):
+def run_w4a8_decode(gwb, dev, stream, hbm_peak, hbm_src, N=14336, K=4096, M=1):
     """W4A8 at decode: the fused product (activations quantized inside the kernel) against the
-    two-launch path (quant_per_token_i8, then gemm_i8i4), each a CUDA graph of `reps` launches
-    alternating two weight sets (> L2)."""
-    sets = [int8_operands(gwb, dev, "w4a8", N, K, M, seed=s_) for s_ in range(2)]
+    two-launch path (quant_per_token_i8, then gemm_i8i4), each a CUDA graph of back-to-back
+    launches rotating through weight copies (> 2x L2)."""
+    wq, sw, _, _ = int8_operands(gwb, dev, "w4a8", N, K, M)
+    cps = clone_all((wq, sw), copies_for(N * K // 2))
     x = synth.activations(M, K, seed=1).to(dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     qx = torch.empty((M, K), dtype=torch.int8, device=dev)
     sx = torch.empty((M,), dtype=torch.float32, device=dev)
 
     def fused(i):
-        wq, sw, _, _ = sets[i % 2]
-        gwb.gemv_w4a8(x, wq, sw, y=y)
+        w, s = cps[i % len(cps)]
+        gwb.gemv_w4a8(x, w, s, y=y)
 
     def two(i):
-        wq, sw, _, _ = sets[i % 2]
+        w, s = cps[i % len(cps)]
         gwb.quant_per_token_i8(x, qx=qx, sx=sx)
-        gwb.gemm_i8i4(qx, sx, wq, sw, y=y)
+        gwb.gemm_i8i4(qx, sx, w, s, y=y)
 
-    out = {}
-    for name, fn in (("fused", fused), ("two_launch", two)):
-        with torch.cuda.stream(stream):
-            for i in range(2):
-                fn(i)
-            stream.synchronize()
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr, stream=stream):
-                for i in range(reps):
-                    fn(i)
-            gr.replay()
-            stream.synchronize()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            gr.replay()
-            b.record(stream)
-            b.synchronize()
-        out[name] = a.elapsed_time(b) * 1e3 / reps
+    us_f = graph_us(fused, len(cps), stream)
+    us_t = graph_us(two, len(cps), stream)
     nbytes = N * K // 2 + N * 4 + 2 * M * K + 2 * M * N
-    gbs = nbytes / out["fused"] / 1e3
+    gbs = nbytes / us_f / 1e3
     return {"value": round(gbs, 1), "unit": "GB/s", "N": N, "K": K, "M": M,
-            "us_fused": round(out["fused"], 2), "us_two_launch": round(out["two_launch"], 2),
-            "roofline": {"kernel": "k_gemv_pipe<4,64,1,w4a8> (per-token int8 quantization inside)", "bound": "hbm",
-                         "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
-                         "bytes_per_launch": nbytes, "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}}
+            "us_fused": round(us_f, 2), "us_two_launch": round(us_t, 2),
+            "roofline": roofline("k_gemv_pipe<4,64,1,w4a8> (per-token int8 quantization inside)", "hbm", gbs,
+                                 hbm_peak, "GB/s", hbm_src, bytes_per_launch=nbytes)}
 
 
-def run_mlp_fused(gwb, dev, stream, hbm_peak, bits=4, M=1, reps=20):
+def run_mlp_fused(gwb, dev, stream, hbm_peak, hbm_src, bits=4, M=1):
     """Decode MLP of a Llama-3-8B layer (hidden 4096, intermediate 14336, MLX affine gs 64) through
-    the fused products: gemv_gate_up, then gemv_silu_gate_resid.  One CUDA graph of `reps` MLPs
-    alternating two weight sets (> L2), timed by events around its replay."""
+    the fused products: gemv_gate_up, then gemv_silu_gate_resid.  A CUDA graph of back-to-back
+    MLPs rotating through weight copies (> 2x L2)."""
     H, I = 4096, 14336
-    sets = []
-    for s_ in range(2):
-        ws = []
-        for j, (n, k) in enumerate(((I, H), (I, H), (H, I))):
-            g = torch.Generator(device=dev)
-            g.manual_seed(500 + 10 * s_ + j)
-            w = torch.randn((n, k), generator=g, device=dev, dtype=torch.float32) * 0.02
-            ws.append(gwb.qpack_affine(w, bits, GS))
-            del w
-        sets.append(ws)
+    ws = []
+    for j, (n, k) in enumerate(((I, H), (I, H), (H, I))):
+        w = dev_weight(dev, n, k, 500 + j)
+        ws.append(gwb.qpack_affine(w, bits, GS))
+        del w
+    mlp_w = sum(gemv_bytes(n, k, bits, M=0) for n, k in ((I, H), (I, H), (H, I)))
+    cps = [ws] + [[tuple(t.clone() for t in w3) for w3 in ws] for _ in range(copies_for(mlp_w) - 1)]
     x = synth.activations(M, H, seed=1).to(dev)
     gate = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
     up = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
     y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
 
     def mlp(i):
-        wg, wu, wd = sets[i % 2]
+        wg, wu, wd = cps[i % len(cps)]
         gwb.gemv_gate_up(x, wg, wu, bits, GS, y_gate=gate, y_up=up)
         gwb.gemv_silu_gate(gate, up, *wd, bits, GS, x_resid=x, y=y)
 
-    with torch.cuda.stream(stream):
-        for i in range(2):
-            mlp(i)
-        stream.synchronize()
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=stream):
-            for i in range(reps):
-                mlp(i)
-        gr.replay()
-        stream.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        gr.replay()
-        b.record(stream)
-        b.synchronize()
-    us = a.elapsed_time(b) * 1e3 / reps
+    us = graph_us(mlp, len(cps), stream)
     nbytes = (2 * gemv_bytes(I, H, bits, M=M) - 2 * M * H) + (gemv_bytes(H, I, bits, M=M) + 2 * M * I + 2 * M * H)
     gbs = nbytes / us / 1e3
     return {"value": round(gbs, 1), "unit": "GB/s", "M": M, "bits": bits, "group_size": GS,
             "us_per_mlp": round(us, 2), "bytes_per_mlp": nbytes, "launches_per_mlp": 2,
-            "roofline": {"kernel": "k_gemv_pipe<dual> + k_gemv_pipe<silu> (Llama-3-8B MLP, hidden 4096)",
-                         "bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                         "frac": round(gbs / hbm_peak, 4), "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}}
+            "roofline": roofline("k_gemv_pipe<dual> + k_gemv_pipe<silu> (Llama-3-8B MLP, hidden 4096)", "hbm", gbs,
+                                 hbm_peak, "GB/s", hbm_src)}
 
 
-# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+# ------------------------------------------------------------------ CPU oracle (reference arm)
 def oracle_sample(frac, seed=0):
     """A row sample of every decode layer, quantized by the oracle (untimed preparation)."""
     import oracle
@@ -542,19 +836,6 @@ def oracle_pass(layers):
         oracle.qmm_affine(x, wq, sc, bi, n, K, bits, GS)
         nbytes += gemv_bytes(n, K, bits)
     return nbytes
-
-
-def cpu_baseline(budget_s=12.0, frac=0.25):
-    layers = oracle_sample(frac)
-    t = time.perf_counter()
-    nbytes, passes = 0, 0
-    while passes < 1 or time.perf_counter() - t < budget_s:
-        nbytes += oracle_pass(layers)
-        passes += 1
-    dt = time.perf_counter() - t
-    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{passes} pass(es) over the first {frac:.0%} of the output rows of every decode layer "
-                      f"(M=1, gs=64), single-threaded C, fp64, {dt:.1f} s"}
 
 
 def run_reference(args, world, rank):
@@ -585,8 +866,8 @@ def run_reference(args, world, rank):
 
 
 def run_layer(args):
-    """One layer only (for profiling): qmm_affine (or, with --fmt, the int8-activation GEMM) on an
-    N x K weight at M tokens, replayed in a CUDA graph of 20 launches that alternate between two
+    """One layer only (for profiling): qmm_affine (or, with --fmt, another product) on an N x K
+    weight at M tokens, replayed in a CUDA graph of 20 launches that alternate between two
     weight sets (> L2)."""
     import group_wise_bit_b200 as gwb
     N, K, bits, M = (list(map(int, args.layer.split(","))) + [1])[:4]
@@ -595,9 +876,7 @@ def run_layer(args):
     if args.fmt == "affine":
         sets = []
         for s in range(2):
-            g = torch.Generator(device=dev)
-            g.manual_seed(s)
-            w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+            w = dev_weight(dev, N, K, s)
             sets.append(gwb.qpack_affine(w, bits, GS))
             del w
         x = synth.activations(M, K, seed=1).to(dev)
@@ -610,9 +889,7 @@ def run_layer(args):
         for s in range(2):
             ws = []
             for j in range(2 if args.fmt == "gate_up" else 1):
-                g = torch.Generator(device=dev)
-                g.manual_seed(10 * s + j)
-                w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32) * 0.02
+                w = dev_weight(dev, N, K, 10 * s + j)
                 ws.append(gwb.qpack_affine(w, bits, GS))
                 del w
             sets.append(ws)
@@ -627,6 +904,18 @@ def run_layer(args):
                 gwb.gemv_gate_up(x, ws[0], ws[1], bits, GS, y_gate=y, y_up=y2)
             else:
                 gwb.gemv_silu_gate(x, x2, *ws[0], bits, GS, x_resid=res, y=y)
+    elif args.fmt == "gptq":
+        sets = []
+        for s in range(2):
+            qw, sc, qz, _ = synth.gptq_quartet(K, N, GPTQ_GS, seed=s)
+            sets.append((qw.to(dev), sc.to(dev), qz.to(dev)))
+        x = synth.activations(M, K, seed=1, dtype=torch.float16).to(dev)
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        bits = 4
+
+        def launch(i):
+            q, s, z = sets[i % 2]
+            gwb.gptq_qmm(x, q, s, z, None, GPTQ_GS, y=y)
     else:
         sets = [int8_operands(gwb, dev, args.fmt, N, K, M, seed=s) for s in range(2)]
         gemm = int8_gemm(gwb, args.fmt)
@@ -660,14 +949,16 @@ def run_layer(args):
         nbytes = 2 * gemv_bytes(N, K, bits, M=M) - 2 * M * K      # x is read once
     elif args.fmt == "silu_resid":
         nbytes = gemv_bytes(N, K, bits, M=M) + 2 * M * K + 2 * M * N   # up and the residual
+    elif args.fmt == "gptq":
+        nbytes = gptq_bytes(K, N, GPTQ_GS, M, False) if M <= 32 else None
     else:
-        nbytes = (N * K * bits // 8 + N * 4 + M * K + M * 4 + M * N * 2) if M <= 8 else None
+        nbytes = int8_bytes(N, K, M, bits) if M <= 64 else None
     out = {"layer": {"fmt": args.fmt, "N": N, "K": K, "bits": bits, "group_size": GS, "M": M},
            "us_per_launch": round(us, 2)}
     if nbytes:
         out["GB/s"] = round(nbytes / us / 1e3, 1)
     else:
-        out["TFLOP/s" if args.fmt == "affine" else "TOP/s"] = round(2.0 * M * N * K / us / 1e6, 1)
+        out["TFLOP/s" if args.fmt in ("affine", "gptq") else "TOP/s"] = round(2.0 * M * N * K / us / 1e6, 1)
     print(json.dumps(out), flush=True)
 
 
@@ -677,10 +968,12 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["gwb", "reference"], default="gwb")
-    ap.add_argument("--no-prefill", action="store_true")
-    ap.add_argument("--fmt", choices=["affine", "w4a8", "w8a8", "gate_up", "silu_resid"], default="affine",
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="time the decode sweep (and the fused decode products) only")
+    ap.add_argument("--fmt", choices=["affine", "w4a8", "w8a8", "gate_up", "silu_resid", "gptq"], default="affine",
                     help="--layer: weight format (affine: MLX group-wise, bits from --layer)")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the CPU baseline leg (and with it the parity check before timing)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-frac", type=float, default=1 / 16)
     ap.add_argument("--layer", default=None,

@@ -43,6 +43,8 @@ SIGNATURES = {
     "gwb_qpack_sym_i8": [_P, _I64, _I64, _P, _P, _P],
     "gwb_gemm_i8i8": [_P, _P, _I64, _P, _P, _I64, _I64, _P, _P, _P],
     "gwb_check_device_error": [_P],
+    "gwb_debug_set_wait_cycles": [ctypes.c_ulonglong],
+    "gwb_debug_inject_stream_k_stall": [_INT],
 }
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "UNSUPPORTED", 4: "ALIGN", 5: "CUDA", 6: "TIMEOUT"}
@@ -346,3 +348,16 @@ def gemm_i8i8(qx, sx, wq, sw, want_y=True, want_acc=False, y=None, acc=None):
 def check_device_error():
     """Synchronizes the current stream; raises GwbError(TIMEOUT) if a bounded device wait gave up."""
     _call("gwb_check_device_error", _stream())
+
+
+def debug_set_wait_cycles(cycles):
+    """Failure-path testing: SM clock cycles after which device waits give up on the
+    current device (0 restores the default, about 2 s)."""
+    _call("gwb_debug_set_wait_cycles", int(cycles))
+
+
+def debug_inject_stream_k_stall(armed=True):
+    """Failure-path testing: the next stream-K launch of the persistent GEMM waits for
+    partial tiles that nothing publishes, so its bounded waits run out (see gwb.h);
+    armed=False disarms it."""
+    _call("gwb_debug_inject_stream_k_stall", 1 if armed else 0)

@@ -82,17 +82,16 @@ const char *gwb_last_error(void) { return gwb::g_msg; }
 const char *gwb_version(void) { return "group_wise_bit_b200 0.1 (sm_100a)"; }
 
 gwb_status gwb_check_device_error(void *stream) {
-  unsigned int flag = 0, flag2 = 0, flag4 = 0, flag5 = 0, flag6 = 0, flag7 = 0, flag8 = 0, flag9 = 0;
+  unsigned int flag = 0;
   GWB_TRY(gwb::read_and_clear_device_error(as_stream(stream), &flag));
-  GWB_TRY(gwb::read_and_clear_device_error_stream(as_stream(stream), &flag2));
-  GWB_TRY(gwb::read_and_clear_device_error_pipe(as_stream(stream), &flag4));
-  GWB_TRY(gwb::read_and_clear_device_error_tc2(as_stream(stream), &flag5));
-  GWB_TRY(gwb::read_and_clear_device_error_gate_up(as_stream(stream), &flag6));
-  GWB_TRY(gwb::read_and_clear_device_error_silu(as_stream(stream), &flag7));
-  GWB_TRY(gwb::read_and_clear_device_error_w4a8(as_stream(stream), &flag8));
-  GWB_TRY(gwb::read_and_clear_device_error_i8w8(as_stream(stream), &flag9));
-  flag |= flag2 | flag4 | flag5 | flag6 | flag7 | flag8 | flag9;
   if (flag) return fail(GWB_ERR_TIMEOUT, "a bounded device-side wait gave up (flag 0x%x)", flag);
+  return GWB_OK;
+}
+
+gwb_status gwb_debug_set_wait_cycles(unsigned long long cycles) { return gwb::set_wait_cycles(cycles); }
+
+gwb_status gwb_debug_inject_stream_k_stall(int armed) {
+  gwb::inject_stream_k_stall(armed != 0);
   return GWB_OK;
 }
 
@@ -133,7 +132,6 @@ gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, cons
   GWB_TRY(need(wq, "wq"));
   GWB_TRY(need(scales, "scales"));
   GWB_TRY(need(biases, "biases"));
-  if (!aligned16(x)) return fail(GWB_ERR_ALIGN, "x is not 16-byte aligned");
   if (M <= 8 && gwb::gemv_affine_supported(bits, group_size)) {
     gwb_status s =
         gwb::launch_gemv_pipe(x, (int)M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));

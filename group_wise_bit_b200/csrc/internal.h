@@ -15,6 +15,16 @@ gwb_status fail(gwb_status st, const char *fmt, ...);
 // Maps the launch error (if any) of the last kernel to a gwb_status.
 gwb_status check_launch(const char *what);
 
+// Synchronizes `st`, then reads and clears the device error flag (bit 0: a
+// bounded device wait gave up) of the current device.
+gwb_status read_and_clear_device_error(cudaStream_t st, unsigned int *flag);
+// Sets the clock cycles after which device waits give up on the current
+// device (0: the default, about 2 s).
+gwb_status set_wait_cycles(unsigned long long cycles);
+// armed: the next stream-K launch of the persistent GEMM waits for a partial
+// tile that no CTA publishes (failure-path testing); false disarms it.
+void inject_stream_k_stall(bool armed);
+
 // ------------------------------------------------------------ elementwise kernels
 void launch_qpack_affine(const float *w, int64_t N, int64_t K, int bits, int gs, uint32_t *wq,
                          uint16_t *scales, uint16_t *biases, cudaStream_t st);
@@ -42,17 +52,11 @@ gwb_status launch_gemv_affine(const uint16_t *x, int M, const uint32_t *wq, cons
 gwb_status launch_gemv_stream(const uint16_t *x, int M, const uint32_t *wq, const uint16_t *scales,
                               const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
                               cudaStream_t st);
-gwb_status read_and_clear_device_error_stream(cudaStream_t st, unsigned int *flag);
 // Producer/consumer decode GEMV (the main decode kernel); GWB_ERR_UNSUPPORTED
 // (without a message) for layouts it does not cover (K / gs not a multiple of 8).
 gwb_status launch_gemv_pipe(const uint16_t *x, int M, const uint32_t *wq, const uint16_t *scales,
                             const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,
                             cudaStream_t st);
-gwb_status read_and_clear_device_error_pipe(cudaStream_t st, unsigned int *flag);
-gwb_status read_and_clear_device_error_gate_up(cudaStream_t st, unsigned int *flag);
-gwb_status read_and_clear_device_error_silu(cudaStream_t st, unsigned int *flag);
-gwb_status read_and_clear_device_error_w4a8(cudaStream_t st, unsigned int *flag);
-gwb_status read_and_clear_device_error_i8w8(cudaStream_t st, unsigned int *flag);
 gwb_status launch_gemv_i8w8(const int8_t *qx, const float *sx, int M, const int8_t *wq, const float *sw, int64_t N,
                             int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 gwb_status launch_gemv_w4a8(const uint16_t *x, int M, const uint32_t *wq, const float *sw, int64_t N, int64_t K,
@@ -79,7 +83,6 @@ gwb_status launch_tc_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, 
                           uint16_t *y, cudaStream_t st, int zadd = 1);
 gwb_status launch_tc_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
                           int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
-gwb_status read_and_clear_device_error(cudaStream_t st, unsigned int *flag);
 // Persistent tensor-core GEMM (M >= 128); GWB_ERR_UNSUPPORTED (without a
 // message) when the layout needs the per-tile kernel (unstaged scales, g_idx).
 gwb_status launch_tc2_affine(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
@@ -92,7 +95,6 @@ gwb_status launch_tc2_i8i8(const int8_t *qx, const float *sx, int64_t M, const i
                            int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 gwb_status launch_tc2_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
                            int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
-gwb_status read_and_clear_device_error_tc2(cudaStream_t st, unsigned int *flag);
 // The persistent GEMM with its stream-K scratch in a fixed device array (no
 // allocation); M must exceed 128.
 gwb_status launch_tc2_affine_noalloc(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,

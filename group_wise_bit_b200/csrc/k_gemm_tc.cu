@@ -488,13 +488,4 @@ gwb_status launch_tc_i8i4(const int8_t *qx, const float *sx, int64_t M, const ui
   return dispatch_bt<Fmt::I8, 4>(M, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, a, st);
 }
 
-gwb_status read_and_clear_device_error(cudaStream_t st, unsigned int *flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaStreamSynchronize(st);
-  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(flag, g_device_error, sizeof(unsigned int));
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
-  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "device error check: %s", cudaGetErrorString(e));
-  return GWB_OK;
-}
-
 }  // namespace gwb

@@ -103,18 +103,23 @@ __device__ __forceinline__ void tma_load_3d_sb(void *dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(0), "r"(smem_u32(bar))
       : "memory");
 }
+// An epoch no launch takes (launch epochs run from 1 to 0x7ffffffe): a head CTA
+// told to wait for it gives up (tests of the bounded-wait failure path).
+constexpr uint32_t kNeverEpoch = 0xffffffffu;
+
 // Stream-K handshake on a global word: publish (release) the epoch once this
 // CTA's partial is stored; wait (acquire, bounded) until a peer published it.
 __device__ __forceinline__ void flag_publish(uint32_t *f, uint32_t epoch) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(epoch) : "memory");
 }
 __device__ __forceinline__ bool flag_wait(const uint32_t *f, uint32_t epoch) {
+  const unsigned long long limit = g_wait_cycles;
   const unsigned long long t0 = clock64();
   while (true) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
     if (v == epoch) return true;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(&g_device_error, 1u);
       return false;
     }
@@ -188,7 +193,8 @@ struct Args {
   // stream-K: partial tiles through a workspace (null: whole tiles per unit)
   uint32_t *ws;             // [CTAs][BT tokens][128 rows] fp32 (i8: s32) partial accumulators
   uint32_t *flags;          // [CTAs] epoch at which the CTA's partial is complete
-  uint32_t epoch;           // this launch's epoch (never 0)
+  uint32_t *ctr;            // [2]: launches so far (the epoch counter), CTAs finished in this launch
+  int stall;                // a test made this launch's heads wait for an epoch nobody publishes
 };
 
 // A unit's contiguous share of the flattened (tile, K step) iteration space,
@@ -411,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *accempty = accfull + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accempty + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  uint32_t *epoch_slot = tmem_slot + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = (a.K + BK - 1) / BK;
@@ -428,6 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; b++) { mbar_init(&accfull[b], 1); mbar_init(&accempty[b], 4 * PAIR); }
     *abort_flag = 0;
+    // stream-K: this launch's epoch, from the workspace's launch counter (so a CUDA
+    // graph that replays the launch gets a fresh epoch every time); never 0, the
+    // flags' initial value, nor kNeverEpoch
+    *epoch_slot = a.ws ? *reinterpret_cast<volatile uint32_t *>(a.ctr) % 0x7ffffffeu + 1u : 0u;
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
     if (F == Fmt::Affine && a.sc_tma) tma_prefetch_desc(&tm_sb);
@@ -673,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lead_thread) {
           for (int v = vfirst; v <= vlast; v++) {
             const uint32_t *f = a.flags + v * PAIR + rank;
-            if (!flag_wait(f, a.epoch)) { *abort_flag = 1; break; }
+            if (!flag_wait(f, a.stall ? kNeverEpoch : *epoch_slot)) { *abort_flag = 1; break; }
           }
         }
         named_bar_sync(1, 128);
@@ -815,7 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (contrib) {   // publish the partial once all four warps stored theirs
         __threadfence();
         named_bar_sync(1, 128);
-        if (lead_thread) flag_publish(a.flags + blockIdx.x, a.epoch);
+        if (lead_thread) flag_publish(a.flags + blockIdx.x, *epoch_slot);
       }
     }
   }
@@ -826,6 +837,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     if constexpr (PAIR == 2) tmem_dealloc_pair(tmem, NCOLS);
     else tmem_dealloc(tmem, NCOLS);
+  }
+  if (a.ws && threadIdx.x == 0) {
+    // the last CTA of the launch to finish advances the epoch counter: every CTA has
+    // read it by then, and the next launch on the stream starts after this one ends
+    __threadfence();
+    if (atomicAdd(&a.ctr[1], 1u) == gridDim.x - 1) {
+      a.ctr[1] = 0u;
+      atomicAdd(&a.ctr[0], 1u);
+    }
   }
 }
 
@@ -859,9 +879,10 @@ gwb_status map2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64
 
 // Stream-K workspace, owned by the library: one per (device, stream), so that
 // GEMMs on different streams never share partial slots; allocated (and its
-// flags zeroed) on the first call that needs it, outside stream capture, and
-// kept until the process exits.  Each launch takes a fresh epoch, so the flags
-// never need clearing again.
+// flags and counters zeroed) on the first call that needs it, outside stream
+// capture, and kept until the process exits.  Each launch takes a fresh epoch
+// from the workspace's launch counter on the device (graph replays included),
+// so the flags never need clearing again.
 struct Workspace {
   uint32_t *base = nullptr;
   size_t partial_bytes = 0;
@@ -869,7 +890,9 @@ struct Workspace {
 };
 std::mutex g_ws_mu;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
-std::atomic<uint32_t> g_epoch{0};
+// Armed by inject_stream_k_stall(): the next stream-K launch's heads wait for
+// kNeverEpoch (tests of the bounded-wait failure path).
+std::atomic<int> g_stall_next{0};
 
 bool stream_workspace(cudaStream_t st, size_t partial_bytes, int nflags, uint32_t **ws, uint32_t **flags) {
   int dev = 0;
@@ -931,23 +954,26 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
   int grid_units = a.T < units ? a.T : units;
   a.ws = nullptr;
   a.flags = nullptr;
-  a.epoch = 0;
+  a.ctr = nullptr;
+  a.stall = 0;
   if (a.T % units != 0 && (int64_t)a.T * nk >= 4LL * units) {
-    uint32_t *ws = nullptr, *fl = nullptr;
+    uint32_t *ws = nullptr, *fl = nullptr, *ctr = nullptr;
     bool have_ws = false;
     if (fixed_ws) {
+      // flags of the units, then the two counters, cleared for this call
       ws = fixed_ws;
       fl = fixed_ws + (size_t)units * PAIR * BT * kTileN;
-      have_ws = cudaMemsetAsync(fl, 0, (size_t)units * PAIR * 4, st) == cudaSuccess;
+      ctr = fl + units * PAIR;
+      have_ws = cudaMemsetAsync(fl, 0, ((size_t)units * PAIR + 2) * 4, st) == cudaSuccess;
     } else {
-      have_ws = stream_workspace(st, (size_t)kSMs * BT * kTileN * 4, kSMs, &ws, &fl);
+      have_ws = stream_workspace(st, (size_t)kSMs * BT * kTileN * 4, kSMs + 2, &ws, &fl);
+      ctr = fl + kSMs;
     }
     if (have_ws) {
       a.ws = ws;
       a.flags = fl;
-      uint32_t e = g_epoch.fetch_add(1) + 1;
-      if (e == 0) e = g_epoch.fetch_add(1) + 1;
-      a.epoch = e;
+      a.ctr = ctr;
+      a.stall = g_stall_next.exchange(0);
       grid_units = units;
     }
   }
@@ -978,18 +1004,30 @@ gwb_status dispatch2(int64_t M, const void *x, CUtensorMapDataType xdt, int xele
   return run_tc2<F, BITS, 256, 2, kAInTmem>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
 }
 
+}  // namespace
+
+void inject_stream_k_stall(bool armed) { g_stall_next.store(armed ? 1 : 0); }
+
+namespace {
+
 // ---------------------------------------------------------------- scratch without allocation
 // Some callers cannot allocate device memory: code running under an allocator
 // that owns all of the GPU's memory (a framework's caching pool, a serving
 // runtime that reserves memory up front), or code that must not call
 // cudaMalloc / cudaFree at all, since both may synchronize the device.  For
 // them the prefill GEMM can run with its stream-K scratch in this fixed array:
-// the partial tiles of at most kScratchPairs CTA pairs (8 MiB) and their flags.
+// the partial tiles of at most kScratchPairs CTA pairs (8 MiB), their flags and
+// the launch counters (512 bytes).
 // It lives in every GPU that loads the library until the process exits.
 constexpr int kScratchPairs = 32;
 constexpr size_t kScratchPartialWords = (size_t)kScratchPairs * 2 * 256 * kTileN;
-constexpr size_t kScratchFlagWords = 64;
+constexpr size_t kScratchFlagWords = 128;
 static __device__ __align__(256) uint32_t g_noalloc_scratch[kScratchPartialWords + kScratchFlagWords];
+// one 256-token x 128-row partial per CTA of the pairs, one flag per CTA and the
+// two launch counters
+static_assert(kScratchPartialWords == (size_t)kScratchPairs * 2 * 256 * kTileN &&
+                  kScratchFlagWords >= (size_t)kScratchPairs * 2 + 2,
+              "the scratch array must hold every pair's partials and flags");
 
 // Device address of the array on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
@@ -1059,15 +1097,11 @@ gwb_status launch_tc2_affine_noalloc(const uint16_t *x, int64_t M, const uint32_
                                      cudaStream_t st) {
   if (M <= 128)
     return fail(GWB_ERR_SHAPE, "qmm_affine_noalloc runs the prefill GEMM: M must exceed 128 (M=%lld)", (long long)M);
-  if ((K / gs) % 2 != 0 || (((uintptr_t)scales | (uintptr_t)biases) & 3) != 0)
+  if ((K / gs) % 2 != 0)
     return fail(GWB_ERR_UNSUPPORTED, "qmm_affine_noalloc needs an even number of groups per row (K/gs=%lld)",
                 (long long)(K / gs));
-  // the scratch holds one 256-token x 128-row fp32 partial per CTA of at most
-  // kScratchPairs pairs, plus their flags
-  const size_t need = (size_t)kScratchPairs * 2 * 256 * kTileN + (size_t)kScratchPairs * 2;
-  if (need > kScratchPartialWords + kScratchFlagWords)
-    return fail(GWB_ERR_SHAPE, "qmm_affine_noalloc: %zu scratch words needed, %zu available", need,
-                kScratchPartialWords + kScratchFlagWords);
+  if ((((uintptr_t)scales | (uintptr_t)biases) & 3) != 0)
+    return fail(GWB_ERR_ALIGN, "qmm_affine_noalloc needs 4-byte aligned scales and biases");
   uint32_t *scratch = nullptr;
   gwb_status s = noalloc_scratch(&scratch);
   if (s != GWB_OK) return s;
@@ -1129,15 +1163,6 @@ gwb_status launch_tc2_i8i8(const int8_t *qx, const float *sx, int64_t M, const i
   if (M <= 32) return run_tc2<Fmt::W8, 8, 32, 1, false>(qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
   if (M <= 128) return run_tc2<Fmt::W8, 8, 128, 1, false>(qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
   return run_tc2<Fmt::W8, 8, 256, 2, false>(qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
-}
-
-gwb_status read_and_clear_device_error_tc2(cudaStream_t st, unsigned int *flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaStreamSynchronize(st);
-  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(flag, g_device_error, sizeof(unsigned int));
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
-  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "device error check: %s", cudaGetErrorString(e));
-  return GWB_OK;
 }
 
 }  // namespace gwb

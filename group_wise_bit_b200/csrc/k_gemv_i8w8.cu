@@ -21,13 +21,4 @@ gwb_status launch_gemv_i8w8(const int8_t *qx, const float *sx, int M, const int8
   return run_pipe<8, 64, 8, kOpI8W8>(in, st);
 }
 
-gwb_status read_and_clear_device_error_i8w8(cudaStream_t st, unsigned int *flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaStreamSynchronize(st);
-  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(flag, g_device_error, sizeof(unsigned int));
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
-  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "device error check: %s", cudaGetErrorString(e));
-  return GWB_OK;
-}
-
 }  // namespace gwb

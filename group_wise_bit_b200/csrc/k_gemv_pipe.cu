@@ -21,13 +21,4 @@ gwb_status launch_gemv_pipe(const uint16_t *x, int M, const uint32_t *wq, const 
   return GWB_ERR_UNSUPPORTED;
 }
 
-gwb_status read_and_clear_device_error_pipe(cudaStream_t st, unsigned int *flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaStreamSynchronize(st);
-  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(flag, g_device_error, sizeof(unsigned int));
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
-  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "device error check: %s", cudaGetErrorString(e));
-  return GWB_OK;
-}
-
 }  // namespace gwb

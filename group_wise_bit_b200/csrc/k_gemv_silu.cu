@@ -25,13 +25,4 @@ gwb_status launch_gemv_silu_gate(const uint16_t *gate, const uint16_t *up, int M
   return GWB_ERR_UNSUPPORTED;
 }
 
-gwb_status read_and_clear_device_error_silu(cudaStream_t st, unsigned int *flag) {
-  unsigned int zero = 0;
-  cudaError_t e = cudaStreamSynchronize(st);
-  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(flag, g_device_error, sizeof(unsigned int));
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
-  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "device error check: %s", cudaGetErrorString(e));
-  return GWB_OK;
-}
-
 }  // namespace gwb

@@ -1,7 +1,8 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads, tcgen05
 // (TMEM allocation, MMA, commit, loads) and proxy fences.  Every wait is
-// bounded: a wait that does not complete within kWaitCycles sets the device
-// error flag and reports failure to its caller, which then stops issuing work.
+// bounded: a wait that does not complete within g_wait_cycles clock cycles sets
+// the device error flag and reports failure to its caller, which then stops
+// issuing work.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -9,12 +10,28 @@
 
 namespace gwb {
 
-// Device error flag (bit 0: a bounded wait gave up).  Each translation unit
-// that includes this header has its own copy and exposes a host function that
-// reads and clears it; gwb_check_device_error() reads all of them.
-static __device__ unsigned int g_device_error = 0;
-
+// Device error flag (bit 0: a bounded wait gave up) and the wait limit in
+// clock cycles (kWaitCycles unless a test lowered it).  Device code is compiled
+// per translation unit, so each unit that includes this header has its own
+// copy of both; every unit registers them (below), and the host reads and
+// clears all flags in one step and sets all limits together (device_state.cu).
 constexpr unsigned long long kWaitCycles = 4000000000ull;  // ~2 s at 1.9 GHz
+static __device__ unsigned int g_device_error = 0;
+static __device__ unsigned long long g_wait_cycles = kWaitCycles;
+
+// Device addresses of one unit's flag and limit on the current device.
+using DeviceStateAddrs = cudaError_t (*)(unsigned int **flag, unsigned long long **wait);
+void register_device_state(DeviceStateAddrs addrs);   // device_state.cu
+
+namespace {
+cudaError_t unit_device_state(unsigned int **flag, unsigned long long **wait) {
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(flag), g_device_error);
+  if (e == cudaSuccess) e = cudaGetSymbolAddress(reinterpret_cast<void **>(wait), g_wait_cycles);
+  return e;
+}
+// registers this unit's lookup when the library is loaded (no CUDA call then)
+[[maybe_unused]] const bool g_unit_device_state_registered = (register_device_state(&unit_device_state), true);
+}  // namespace
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -71,9 +88,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // raises the device error flag) when the wait gives up.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long limit = g_wait_cycles;
   const unsigned long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(&g_device_error, 1u);
       return false;
     }

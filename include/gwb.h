@@ -14,9 +14,11 @@
  *    tokens, gemm_i8i4 from 128, gemm_i8i8 off its decode path), grown once
  *    if a later call needs more (after synchronizing the stream), and kept
  *    until the process exits.  A call made while its stream is being captured
- *    into a CUDA graph never allocates; it runs without the workspace (whole
- *    tiles per CTA or pair).  gwb_qmm_affine_noalloc is the entry point that
- *    allocates nothing.
+ *    into a CUDA graph never allocates: it uses the stream's workspace if an
+ *    earlier call made one, else it runs without (whole tiles per CTA or pair).
+ *    Each launch takes its stream-K epoch from a counter in the workspace, on
+ *    the device, so graph replays stay correct.  gwb_qmm_affine_noalloc is the
+ *    entry point that allocates nothing.
  *  - bf16 and fp16 values are passed as their raw 16-bit patterns (uint16_t).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
  *    validates its arguments synchronously, on the host, before launching
@@ -77,11 +79,33 @@ const char *gwb_last_error(void);
 /* Library version string. */
 const char *gwb_version(void);
 
-/* Synchronizes `stream`, then reads and clears the device error flag that the
- * bounded waits of the tensor-core kernels set.  Returns GWB_OK when no wait
+/* Synchronizes `stream`, then reads and clears the current device's error
+ * flag, which every bounded wait of the library's kernels sets when it gives
+ * up (one flag per device, shared by all kernels).  Returns GWB_OK when no wait
  * gave up since the last check, GWB_ERR_TIMEOUT otherwise, GWB_ERR_CUDA when
- * the synchronization itself failed. */
+ * the synchronization itself failed.  A kernel whose wait gave up stops
+ * issuing work, lets the copies it started land, frees its tensor memory and
+ * returns, so the context stays usable; its outputs are then undefined.
+ * Source: metrale_gpu_runtime/mlx_int8.rs, MlxInt8Weight::load (failures are
+ * returned as errors, never as a crash). */
 gwb_status gwb_check_device_error(void *stream);
+
+/* Failure-path testing hooks (the pages have no counterpart; they exist so
+ * that the bounded-wait path above can be exercised without faulting a GPU).
+ *
+ * gwb_debug_set_wait_cycles -- sets, on the current device, the number of SM
+ * clock cycles after which a device wait gives up (0 restores the default of
+ * 4e9 cycles, about 2 s).  Takes effect for kernels launched afterwards;
+ * synchronous.  GWB_ERR_CUDA if the device symbol cannot be written. */
+gwb_status gwb_debug_set_wait_cycles(unsigned long long cycles);
+
+/* gwb_debug_inject_stream_k_stall -- armed != 0: the next launch in this
+ * process of the persistent tensor-core GEMM that splits tiles between CTA
+ * pairs (stream-K) waits for partial tiles that no CTA publishes; its head
+ * CTAs' bounded waits run out, the kernel returns early with undefined outputs,
+ * and the next gwb_check_device_error() reports GWB_ERR_TIMEOUT.  One-shot: that
+ * launch disarms it.  armed == 0 disarms it.  Always GWB_OK. */
+gwb_status gwb_debug_inject_stream_k_stall(int armed);
 
 /* ------------------------------------------------------------------ MLX affine */
 
@@ -135,11 +159,11 @@ gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, cons
  * Same arguments, layouts and result as gwb_qmm_affine, for M > 128 only
  * (GWB_ERR_SHAPE otherwise: smaller M needs no scratch, call gwb_qmm_affine).
  * The GEMM's stream-K scratch (partial tiles and their flags) is a file-scope
- * device array of the library, 8 MiB + 256 bytes, which holds the partials of
+ * device array of the library, 8 MiB + 512 bytes, which holds the partials of
  * at most 32 CTA pairs, so the GEMM runs on at most 32 pairs (64 of the 148
- * SMs) and every problem size fits; a size whose scratch would not fit is
- * rejected with GWB_ERR_SHAPE and a message.  Every GPU that loads the library
- * holds the array until the process exits.
+ * SMs); every problem size fits, because a pair's share of the work grows with
+ * the problem while its partial tile does not.  Every GPU that loads the
+ * library holds the array until the process exits.
  *  - The call allocates nothing: no cudaMalloc, cudaFree or allocating library
  *    routine.  The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and caches it; make that
@@ -148,8 +172,8 @@ gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, cons
  *    call clears the flags it needs before its kernel runs.  Calls that overlap
  *    on the GPU (concurrent streams, or several devices' threads racing on one
  *    device) race on the array and give wrong results: serialize them.
- * Also GWB_ERR_UNSUPPORTED when K/group_size is odd or scales/biases are not
- * 4-byte aligned. */
+ * Also GWB_ERR_UNSUPPORTED when K/group_size is odd, and GWB_ERR_ALIGN when x,
+ * y or the weight tensors are not 16-byte aligned. */
 gwb_status gwb_qmm_affine_noalloc(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
                                   const uint16_t *biases, int64_t N, int64_t K, int bits, int group_size,
                                   uint16_t *y, void *stream);

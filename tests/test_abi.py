@@ -62,9 +62,11 @@ def test_validation_codes(lib):
     # bits / group size / divisibility / negative sizes
     assert _st("gwb_qmm_affine", OK16, 1, OK16, OK16, OK16, 64, 128, 3, 64, OK16, NULL) == 3
     assert _st("gwb_qmm_affine", OK16, 1, OK16, OK16, OK16, 64, 128, 4, 48, OK16, NULL) == 3
+    assert "group_size=48" in gwb.lib().gwb_last_error().decode()
     assert _st("gwb_qmm_affine", OK16, 1, OK16, OK16, OK16, 64, 96, 4, 64, OK16, NULL) == 2
+    assert "multiple of group_size" in gwb.lib().gwb_last_error().decode()
     assert _st("gwb_qmm_affine", OK16, -1, OK16, OK16, OK16, 64, 128, 4, 64, OK16, NULL) == 1
-    assert "group_size" in gwb.lib().gwb_last_error().decode() or True
+    assert "negative M" in gwb.lib().gwb_last_error().decode()
     # NULL and misaligned pointers
     assert _st("gwb_qmm_affine", OK16, 1, OK16, OK16, OK16, 64, 128, 4, 64, NULL, NULL) == 1
     assert _st("gwb_qmm_affine", OK16, 1, OK16, OK16, OK16, 64, 128, 4, 64, BAD, NULL) == 4
@@ -112,6 +114,13 @@ def test_validation_codes_of_the_next_step_entry_points(lib):
     assert _st("gwb_gemm_i8i8", OK16, OK16, 4, OK16, OK16, 64, 262144, OK16, NULL, NULL) == 2
     assert _st("gwb_gemm_i8i8", OK16, OK16, 4, OK16, OK16, 64, 128, NULL, NULL, NULL) == 1
     assert _st("gwb_gemm_i8i8", BAD, OK16, 4, OK16, OK16, 64, 128, OK16, NULL, NULL) == 4
+    # the allocation-free prefill GEMM: M > 128 only, aligned operands, even K/gs
+    assert _st("gwb_qmm_affine_noalloc", OK16, 64, OK16, OK16, OK16, 64, 128, 4, 64, OK16, NULL) == 2
+    assert _st("gwb_qmm_affine_noalloc", BAD, 256, OK16, OK16, OK16, 64, 128, 4, 64, OK16, NULL) == 4
+    assert "x is not 16-byte aligned" in gwb.lib().gwb_last_error().decode()
+    assert _st("gwb_qmm_affine_noalloc", OK16, 256, OK16, BAD, OK16, 64, 128, 4, 64, OK16, NULL) == 4
+    assert _st("gwb_qmm_affine_noalloc", OK16, 256, OK16, OK16, OK16, 64, 192, 4, 64, OK16, NULL) == 3
+    assert "even number of groups" in gwb.lib().gwb_last_error().decode()
     # AWQ: the GPTQ shape rules
     assert _st("gwb_awq_dequant", OK16, OK16, OK16, 256, 12, 128, OK16, NULL) == 2
     assert _st("gwb_awq_qmm", OK16, 1, OK16, OK16, OK16, 256, 16, 48, OK16, NULL) == 3

@@ -7,6 +7,9 @@ tolerance in tests/tol.py.  Small cases span several tiles and ragged tails in
 N, M and K; the full-size cases use the workloads' shapes, with the oracle
 evaluated on sampled output rows where all rows would take too long.
 """
+import concurrent.futures as cf
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -29,14 +32,40 @@ def _words(t):
     return t.cpu().numpy().view(np.uint32)
 
 
+TOKEN_BLOCK = 128   # the smallest token tile of the tensor-core kernels (256-token tiles hold two blocks)
+
+
 def _rows(M, N, K, seed=0, budget=3e8):
-    """All rows when the oracle finishes quickly, else the first, the last and a
-    seeded sample of rows in between (about `budget` multiply-adds in total)."""
+    """All rows when the oracle finishes quickly, else: the first and last rows, one
+    seeded row inside every block of TOKEN_BLOCK tokens (so every token tile of
+    every kernel, and with all N columns every output tile and every stream-K
+    share, is compared), and a seeded sample of further rows (about `budget`
+    multiply-adds on top)."""
     if M * N * K <= budget or M <= 2:
         return None
+    rng = np.random.default_rng(seed)
+    blocks = [b + int(rng.integers(0, min(TOKEN_BLOCK, M - b))) for b in range(0, M, TOKEN_BLOCK)]
     n = int(max(0, min(M - 2, budget // (N * K) - 2)))
-    r = np.random.default_rng(seed).choice(np.arange(1, M - 1), size=n, replace=False) if n else []
-    return np.unique(np.concatenate([[0, M - 1], r]).astype(np.int64))
+    r = rng.choice(np.arange(1, M - 1), size=n, replace=False) if n else []
+    return np.unique(np.concatenate([[0, M - 1], blocks, r]).astype(np.int64))
+
+
+ORACLE_THREADS = max(1, min(32, os.cpu_count() or 1))
+
+
+def _by_rows(fn, *args, rows=None, **kw):
+    """fn(*args, rows=..., **kw) of the oracle, with a long row list split over
+    threads (the oracle's C calls release the GIL); the results are put back
+    together in row order: arrays concatenated, flags or-ed."""
+    if rows is None or len(rows) < 2 * ORACLE_THREADS // 4 or ORACLE_THREADS == 1:
+        return fn(*args, rows=rows, **kw)
+    chunks = [c for c in np.array_split(np.asarray(rows), min(ORACLE_THREADS, len(rows))) if len(c)]
+    with cf.ThreadPoolExecutor(len(chunks)) as ex:
+        parts = list(ex.map(lambda c: fn(*args, rows=c, **kw), chunks))
+    if isinstance(parts[0], tuple):
+        return tuple(np.concatenate([p[i] for p in parts]) if isinstance(parts[0][i], np.ndarray)
+                     else any(p[i] for p in parts) for i in range(len(parts[0])))
+    return np.concatenate(parts)
 
 
 def _affine_max_w(sc, bi, bits):
@@ -65,8 +94,8 @@ class Affine:
         x = synth.activations(M, self.K, seed=seed, outlier_frac=outlier_frac)
         y = gwb.qmm_affine(x.to(DEV), self.wq, self.sc, self.bi, self.bits, self.gs)
         rows = _rows(M, self.N, self.K)
-        y_ref = oracle.qmm_affine(synth.bits16(x), self.wq_o, self.sc_o, self.bi_o, self.N, self.K, self.bits,
-                                  self.gs, rows=rows)
+        y_ref = _by_rows(oracle.qmm_affine, synth.bits16(x), self.wq_o, self.sc_o, self.bi_o, self.N, self.K,
+                         self.bits, self.gs, rows=rows)
         yg = y.float().cpu().numpy()
         if rows is not None:
             yg = yg[rows]
@@ -136,6 +165,15 @@ def test_qmm_affine_tensor_core_small(bits, gs, M):
     a.check_qmm(M, outlier_frac=0.01, label=f"tc b{bits} gs{gs} M{M}")
 
 
+@pytest.mark.parametrize("gs", [32, 64])
+@pytest.mark.parametrize("M", [9, 16, 40, 130, 300])
+def test_qmm_affine_tensor_core_odd_groups(gs, M):
+    # K = 192: three groups per row at gs 64 (six at gs 32), 3 K steps of 64; an odd
+    # number of groups per row is staged by the per-tile kernel at every M
+    a = Affine(300, 192, 4, gs, seed=gs + 1)
+    a.check_qmm(M, outlier_frac=0.01, label=f"tc K=192 gs{gs} M{M}")
+
+
 @pytest.mark.parametrize("M", [1, 5])
 def test_qmm_affine_gemv_register_fed_fallback(M):
     # an odd number of groups per row (K / gs = 3) is served by the register-fed GEMV
@@ -201,8 +239,8 @@ class Gptq:
         max_w = self.check_dequant()
         x = synth.activations(M, self.K, seed=seed, dtype=torch.float16)
         y = gwb.gptq_qmm(x.to(DEV), *self.d, self.gs)
-        rows = _rows(M, self.N, self.K, budget=1e8)
-        y_ref = oracle.gptq_qmm(synth.bits16(x), *self.h, self.K, self.N, self.gs, rows=rows)
+        rows = _rows(M, self.N, self.K, budget=2e9)
+        y_ref = _by_rows(oracle.gptq_qmm, synth.bits16(x), *self.h, self.K, self.N, self.gs, rows=rows)
         yg = y.float().cpu().numpy()
         if rows is not None:
             yg = yg[rows]
@@ -312,8 +350,8 @@ class Awq:
         max_w = self.check_dequant()
         x = synth.activations(M, self.K, seed=seed, dtype=torch.float16)
         y = gwb.awq_qmm(x.to(DEV), *self.d, self.gs)
-        rows = _rows(M, self.N, self.K, budget=1e8)
-        y_ref = oracle.awq_qmm(synth.bits16(x), *self.h, self.K, self.N, self.gs, rows=rows)
+        rows = _rows(M, self.N, self.K, budget=2e9)
+        y_ref = _by_rows(oracle.awq_qmm, synth.bits16(x), *self.h, self.K, self.N, self.gs, rows=rows)
         yg = y.float().cpu().numpy()
         if rows is not None:
             yg = yg[rows]
@@ -361,7 +399,7 @@ class W4A8:
         assert np.array_equal(qx.cpu().numpy(), qx_o) and np.array_equal(sx.cpu().numpy(), sx_o)
         y, acc = gwb.gemm_i8i4(qx, sx, self.wq, self.sw, want_y=True, want_acc=True)
         rows = _rows(M, self.N, self.K)
-        acc_o, y_o, ovf = oracle.gemm_i8i4(qx_o, sx_o, self.wq_o, self.sw_o, self.N, self.K, rows=rows)
+        acc_o, y_o, ovf = _by_rows(oracle.gemm_i8i4, qx_o, sx_o, self.wq_o, self.sw_o, self.N, self.K, rows=rows)
         assert not ovf
         a = acc.cpu().numpy().astype(np.int64)
         yg = y.float().cpu().numpy()
@@ -397,7 +435,7 @@ class W8A8:
         assert np.array_equal(qx.cpu().numpy(), qx_o) and np.array_equal(sx.cpu().numpy(), sx_o)
         y, acc = gwb.gemm_i8i8(qx, sx, self.wq, self.sw, want_y=True, want_acc=True)
         rows = _rows(M, self.N, self.K)
-        acc_o, y_o, ovf = oracle.gemm_i8i8(qx_o, sx_o, self.wq_o, self.sw_o, self.N, self.K, rows=rows)
+        acc_o, y_o, ovf = _by_rows(oracle.gemm_i8i8, qx_o, sx_o, self.wq_o, self.sw_o, self.N, self.K, rows=rows)
         assert not ovf
         a = acc.cpu().numpy().astype(np.int64)
         yg = y.float().cpu().numpy()
@@ -492,6 +530,36 @@ def test_w4a8_stream_k_split_tiles():
     W4A8(2048, 2048).check(512)
 
 
+def test_stream_k_gemm_replayed_in_a_cuda_graph_with_new_inputs():
+    """A stream-K GEMM captured into a CUDA graph: every replay takes a fresh epoch on the
+    device, so replays with new activations in the same buffer are exactly the eager result
+    (the same split and summation order), and match the oracle."""
+    N, K, M = 2048, 2048, 512
+    a = Affine(N, K, 4, 64, seed=12)
+    xs = [synth.activations(M, K, seed=s, outlier_frac=0.01) for s in (5, 6)]
+    eager = [gwb.qmm_affine(x.to(DEV), a.wq, a.sc, a.bi, 4, 64) for x in xs]
+    st = torch.cuda.Stream()
+    xd = xs[0].to(DEV)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    with torch.cuda.stream(st):
+        gwb.qmm_affine(xd, a.wq, a.sc, a.bi, 4, 64, y=y)      # the stream's workspace exists before capture
+        st.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            gwb.qmm_affine(xd, a.wq, a.sc, a.bi, 4, 64, y=y)
+        for j in (0, 1, 0, 1, 1):
+            xd.copy_(xs[j].to(DEV))
+            y.fill_(float("nan"))
+            g.replay()
+            st.synchronize()
+            assert torch.equal(y, eager[j]), f"replay with input {j} differs from the eager call"
+    rows = np.array([0, 255, 256, 511])
+    ref = oracle.qmm_affine(synth.bits16(xs[1]), a.wq_o, a.sc_o, a.bi_o, N, K, 4, 64, rows=rows)
+    check_float(y.float().cpu().numpy()[rows], ref, K, a.max_w, float(xs[1].float().abs().max()), "graph replay")
+    del g
+    gwb.check_device_error()
+
+
 # --------------------------------------------------------------------------- full sizes
 def test_full_single_affine_linear_512():
     a = Affine(512, 512, 4, 64)
@@ -513,20 +581,27 @@ def test_full_decode_gemv(N, K, bits):
 PREFILL_SHAPES = [(4096, 4096), (1024, 4096), (14336, 4096), (4096, 14336)]
 
 
+PREFILL_M = (16, 128, 512, 2048)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("N,K", PREFILL_SHAPES)
-def test_full_prefill_gemm_4bit_gs64(N, K):
-    a = Affine(N, K, 4, 64)
+def test_full_prefill_gemm_gs64(N, K, bits):
+    a = Affine(N, K, bits, 64)
     a.check_pack()
-    for M in (16, 128, 2048):
-        a.check_qmm(M, outlier_frac=0.01, label=f"prefill {N}x{K} M={M}")
+    for M in PREFILL_M:
+        a.check_qmm(M, outlier_frac=0.01, label=f"prefill {N}x{K} b{bits} M={M}")
 
 
 @pytest.mark.parametrize("bits,gs", [(8, 32), (8, 128), (4, 32), (4, 128)])
-def test_full_prefill_other_formats(bits, gs):
+def test_full_prefill_other_group_sizes(bits, gs):
     a = Affine(4096, 4096, bits, gs)
     a.check_pack()
     for M in (16, 512):
-        a.check_qmm(M, outlier_frac=0.01, label=f"prefill b{bits} gs{gs} M={M}")
+        a.check_qmm(M, outlier_frac=0.01, label=f"prefill 4096x4096 b{bits} gs{gs} M={M}")
+    b = Affine(14336, 4096, bits, gs, seed=1)
+    for M in (128, 512):
+        b.check_qmm(M, outlier_frac=0.01, label=f"prefill 14336x4096 b{bits} gs{gs} M={M}")
 
 
 @pytest.mark.parametrize("permuted", [False, True])
