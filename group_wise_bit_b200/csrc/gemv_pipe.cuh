@@ -98,13 +98,6 @@ constexpr int kCWLog = 3;
 constexpr int kThreads = kCW * 32;
 constexpr int kSmemPerSM = 232448;
 constexpr int kSMs = 148;
-// Shared memory a CTA may take: half an SM, so that a CTA of the next kernel in
-// the stream (launched early by programmatic serialization) fits next to it
-// and runs its prologue and L2 prefetches while this one streams.
-#ifndef GWB_PIPE_CTA_SMEM
-#define GWB_PIPE_CTA_SMEM (kSmemPerSM / 2)
-#endif
-constexpr int kCtaSmem = GWB_PIPE_CTA_SMEM;
 
 // What the kernel computes around the quantized product (see the file comment).
 constexpr int kOpPlain = 0;   // y = x W^T
@@ -179,22 +172,6 @@ __device__ __forceinline__ void tma_load_3d_l(uint32_t dst, const CUtensorMap *m
           dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
-}
-
-// L2 prefetch of a tensor box (no shared memory written, no barrier): only
-// brings the lines into L2, so it may run before the previous kernel's writes
-// are visible (the L2 is the point of coherence of device memory).
-__device__ __forceinline__ void tma_prefetch_2d_l2(const CUtensorMap *map, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_3d_l2(const CUtensorMap *map, int32_t x, int32_t y, int32_t z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
 }
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -423,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   fence_mbar_init();
   __syncthreads();
   pdl_launch_dependents();
+  pdl_wait();   // the previous kernel's writes (x, and possibly the weights) are visible from here on
 
   // loads the stage (strip, st) of this warp into its ring slot: packed words
   // as one 3-D box ([2 segments][16 rows][128 bytes], or two 2-D boxes) and the
@@ -455,40 +433,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_load_2d_l(ds + C::SBB, mb, gbox, r0, bar);
     }
   };
-  // the same boxes as issue(strip, st, .), into L2 only
-  auto prefetch = [&](int strip, int st) {
-    const bool hi = OP == kOpDual && strip >= a.NSH;
-    const int r0 = (hi ? strip - a.NSH : strip) * 16;
-    const CUtensorMap *mw = hi ? &tm_w2 : &tm_w, *msb = hi ? &tm_sb2 : &tm_sb, *mb = hi ? &tm_b2 : &tm_b;
-    const int ks = k0 + st * C::KST;
-    const int gsx = ks / GS;
-    const int gbox = C::GST < 8 ? (gsx & ~7) : gsx;
-    if (a.w3d) {
-      tma_prefetch_3d_l2(mw, 0, r0, ks / (32 * C::CPW));
-    } else {
-      tma_prefetch_2d_l2(mw, ks / C::CPW, r0);
-      tma_prefetch_2d_l2(mw, ks / C::CPW + 32, r0);
-    }
-    if (OP == kOpW4A8 || OP == kOpI8W8) {
-    } else if (a.sb_joint) {
-      tma_prefetch_3d_l2(msb, gbox, r0, 0);
-    } else {
-      tma_prefetch_2d_l2(msb, gbox, r0);
-      tma_prefetch_2d_l2(mb, gbox, r0);
-    }
-  };
-  // Before waiting for the previous kernel: pull this warp's first ring fill into
-  // L2 (the loads issued after the wait then hit L2).  The prefetch reads no
-  // data into the kernel, so it is correct whatever the previous kernel writes.
-  if (lane == 0) {
-    int ps = sb + ub(warp) / NCS, pst = ub(warp) % NCS;
-    for (int i = 0; i < (units < D ? units : D); i++) {
-      prefetch(ps, pst);
-      if (++pst == NCS) { pst = 0; ++ps; }
-    }
-  }
-  pdl_wait();   // the previous kernel's writes (x, and possibly the weights) are visible from here on
-
   // issue-side position (strip, stage) of this warp, advanced without divisions
   int is_strip = sb + ub(warp) / NCS, is_st = ub(warp) % NCS;
   // ---- activations of the K-slice, staged per item = (group, token, quad lane c):
@@ -1139,7 +1083,6 @@ gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
   // strips (one wave), ring depth D and shared memory; per_sm = 2 puts two
   // CTAs on an SM (twice the warps to hide latency, half the ring each).
   struct Plan { int S, P, D, NCS, out_strips; size_t smem; double est; };
-  int cta_cap = kCtaSmem;   // shared memory a CTA may take (raised to the whole SM when nothing fits)
   auto plan_for = [&](int S, int per_sm, Plan &pl) -> bool {
     if (nst % S != 0) return false;
     const int NCS = nst / S, KR = NCS * C::KST, GR = KR / GS;
@@ -1154,7 +1097,7 @@ gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
                          (size_t)NCS * C::NBM * 32 * 8 + (size_t)kCW * 2 * 16 * MP * 4 +
                          (S > 1 ? (size_t)out_strips * 16 * MP * 4 : 0);
     const size_t per = (size_t)kCW * (C::WB + 2 * C::SBB + 8);
-    const size_t avail = (size_t)(kSmemPerSM / per_sm < cta_cap ? kSmemPerSM / per_sm : cta_cap) - 4096 - 1024;
+    const size_t avail = (size_t)kSmemPerSM / per_sm - 4096 - 1024;
     if (fixed + 2 * per > avail) return false;
     int D = (int)((avail - fixed) / per);
     D = D > 6 ? 6 : D;
@@ -1178,13 +1121,10 @@ gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
       have = true;
     }
   };
-  for (int pass = 0; pass < 2 && !have; pass++) {
-    if (pass == 1) cta_cap = kSmemPerSM;   // no plan fits next to a neighbour: take the whole SM
-    if ((int64_t)NS * nst >= 2LL * kSMs * kCW * 4) consider(1, 2);
-    consider(1, 1);
-    if (OP != kOpI8W8)   // i8w8: the int32 sums are not reduced across a cluster
-      for (int S = 2; S <= 8; S *= 2) consider(S, 1);
-  }
+  if ((int64_t)NS * nst >= 2LL * kSMs * kCW * 4) consider(1, 2);
+  consider(1, 1);
+  if (OP != kOpI8W8)   // i8w8: the int32 sums are not reduced across a cluster
+    for (int S = 2; S <= 8; S *= 2) consider(S, 1);
   if (!have) return GWB_ERR_UNSUPPORTED;
   if (!ensure_smem_attr(reinterpret_cast<const void *>(kern), best.smem))
     return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute failed for %zu bytes of shared memory", best.smem);

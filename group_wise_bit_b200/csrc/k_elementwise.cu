@@ -133,34 +133,57 @@ __global__ void __launch_bounds__(256) k_dequant_affine(const uint32_t *__restri
 }
 
 // ----------------------------------------------------------------------------
-// gptq_dequant: one thread per qweight word (k-octet kq, out-feature o); reads
-// are coalesced along o, and the eight outputs W[o, 8kq .. 8kq+7] are one
-// 16-byte store.  scale * (int4 - zero) is exact in fp32 (an 11-bit scale times
-// a 5-bit integer), so __float2half_rn is the single rounding.
+// gptq_dequant: one CTA per tile of 64 out-features x 256 in-features.  The
+// qweight words are read coalesced along the out-features (one 256-byte row
+// segment per k-octet), each word becomes its eight fp16 weights in shared
+// memory, and the tile leaves as 512-byte runs of each out-feature's row (the
+// output is [N, K], K contiguous).  scale * (int4 - zero) is exact in fp32 (an
+// 11-bit scale times a 5-bit integer), so __float2half_rn is the single rounding.
+constexpr int kGdN = 64, kGdK = 256;                  // tile: out-features x in-features
+constexpr int kGdRow = kGdK * 2 + 16;                 // bytes per staged row (16 bytes of padding: no bank conflicts)
+
 __global__ void __launch_bounds__(256) k_gptq_dequant(const int32_t *__restrict__ qweight,
                                                       const uint16_t *__restrict__ scales,
                                                       const int32_t *__restrict__ qzeros,
                                                       const int32_t *__restrict__ g_idx, int64_t K, int64_t N,
                                                       int gs, int zadd, uint16_t *__restrict__ out) {
-  const int64_t total = (K / 8) * N;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t kq = idx / N, o = idx % N;
-    const uint32_t word = static_cast<uint32_t>(qweight[idx]);
-    uint32_t packed[4];
+  __shared__ __align__(16) unsigned char tile[kGdN * kGdRow];
+  const int64_t n0 = (int64_t)blockIdx.x * kGdN, k0 = (int64_t)blockIdx.y * kGdK;
+  const int t = threadIdx.x;
+  const int nl = t % kGdN, kb = t / kGdN;             // this thread: out-feature nl, k-octets kb*8 .. kb*8+7
+  const int64_t o = n0 + nl;
+  if (o < N) {
+#pragma unroll 2
+    for (int i = 0; i < 8; i++) {
+      const int kql = kb * 8 + i;                     // k-octet within the tile
+      const int64_t kq = k0 / 8 + kql;
+      if (kq * 8 >= K) break;
+      const uint32_t word = static_cast<uint32_t>(__ldg(qweight + kq * N + o));
+      uint32_t packed[4];
 #pragma unroll
-    for (int j = 0; j < 8; j++) {
-      const int64_t k = kq * 8 + j;
-      const int64_t g = g_idx ? (int64_t)g_idx[k] : k / gs;
-      const float s = __half2float(__ushort_as_half(scales[g * N + o]));
-      const uint32_t zw = static_cast<uint32_t>(qzeros[g * (N / 8) + o / 8]);
-      const int zero = (int)((zw >> ((o % 8) * 4)) & 0xFu) + zadd;
-      const int q = (int)((word >> (j * 4)) & 0xFu);
-      const uint16_t h = __half_as_ushort(__float2half_rn(__fmul_rn(s, (float)(q - zero))));
-      if (j & 1) packed[j / 2] |= (uint32_t)h << 16;
-      else packed[j / 2] = h;
+      for (int j = 0; j < 8; j++) {
+        const int64_t k = kq * 8 + j;
+        const int64_t g = g_idx ? (int64_t)__ldg(g_idx + k) : k / gs;
+        const float s = __half2float(__ushort_as_half(__ldg(scales + g * N + o)));
+        const uint32_t zw = static_cast<uint32_t>(__ldg(qzeros + g * (N / 8) + o / 8));
+        const int zero = (int)((zw >> ((o % 8) * 4)) & 0xFu) + zadd;
+        const int q = (int)((word >> (j * 4)) & 0xFu);
+        const uint16_t h = __half_as_ushort(__float2half_rn(__fmul_rn(s, (float)(q - zero))));
+        if (j & 1) packed[j / 2] |= (uint32_t)h << 16;
+        else packed[j / 2] = h;
+      }
+      *reinterpret_cast<uint4 *>(tile + nl * kGdRow + kql * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
-    *reinterpret_cast<uint4 *>(out + o * K + kq * 8) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  }
+  __syncthreads();
+  // each warp writes whole row runs: 32 lanes x 16 bytes = the row's 256 in-features
+  const int lane = t & 31, warp = t >> 5;
+  const int64_t kcols = K - k0 < kGdK ? K - k0 : kGdK;   // a multiple of 8 (K % gs == 0, gs % 8 == 0)
+  for (int r = warp; r < kGdN; r += 8) {
+    const int64_t orow = n0 + r;
+    if (orow >= N) break;
+    if ((int64_t)lane * 8 < kcols)
+      *reinterpret_cast<uint4 *>(out + orow * K + k0 + lane * 8) = *reinterpret_cast<const uint4 *>(tile + r * kGdRow + lane * 16);
   }
 }
 
@@ -347,7 +370,8 @@ void launch_dequant_affine(const uint32_t *wq, const uint16_t *scales, const uin
 void launch_gptq_dequant(const int32_t *qweight, const uint16_t *scales, const int32_t *qzeros,
                          const int32_t *g_idx, int64_t K, int64_t N, int gs, uint16_t *w_out, cudaStream_t st,
                          int zadd) {
-  k_gptq_dequant<<<grid_for((K / 8) * N, 256), 256, 0, st>>>(qweight, scales, qzeros, g_idx, K, N, gs, zadd, w_out);
+  const dim3 grid((unsigned)((N + kGdN - 1) / kGdN), (unsigned)((K + kGdK - 1) / kGdK));
+  k_gptq_dequant<<<grid, 256, 0, st>>>(qweight, scales, qzeros, g_idx, K, N, gs, zadd, w_out);
 }
 
 void launch_quant_per_token_i8(const uint16_t *x, int64_t M, int64_t K, int8_t *qx, float *sx,
