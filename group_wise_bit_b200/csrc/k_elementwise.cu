@@ -152,7 +152,37 @@ __global__ void __launch_bounds__(256) k_gptq_dequant(const int32_t *__restrict_
   const int t = threadIdx.x;
   const int nl = t % kGdN, kb = t / kGdN;             // this thread: out-feature nl, k-octets kb*8 .. kb*8+7
   const int64_t o = n0 + nl;
-  if (o < N) {
+  if (o < N && g_idx == nullptr) {
+    // gs is a multiple of 8: the eight in-features of a word share one group, so
+    // each word takes one scale and one zero, and all loads are issued up front
+    uint32_t word[8], zw[8];
+    uint16_t sh[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const int64_t kq = k0 / 8 + kb * 8 + i;
+      const bool in = kq * 8 < K;
+      const int64_t g = in ? kq * 8 / gs : 0;
+      word[i] = in ? static_cast<uint32_t>(__ldg(qweight + kq * N + o)) : 0u;
+      sh[i] = __ldg(scales + g * N + o);
+      zw[i] = static_cast<uint32_t>(__ldg(qzeros + g * (N / 8) + o / 8));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const int kql = kb * 8 + i;
+      const float s = __half2float(__ushort_as_half(sh[i]));
+      const int zero = (int)((zw[i] >> ((o % 8) * 4)) & 0xFu) + zadd;
+      uint32_t packed[4];
+#pragma unroll
+      for (int j = 0; j < 8; j++) {
+        const int q = (int)((word[i] >> (j * 4)) & 0xFu);
+        const uint16_t h = __half_as_ushort(__float2half_rn(__fmul_rn(s, (float)(q - zero))));
+        if (j & 1) packed[j / 2] |= (uint32_t)h << 16;
+        else packed[j / 2] = h;
+      }
+      *reinterpret_cast<uint4 *>(tile + nl * kGdRow + kql * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+  } else if (o < N) {
+    // g_idx: every in-feature has its own group
 #pragma unroll 2
     for (int i = 0; i < 8; i++) {
       const int kql = kb * 8 + i;                     // k-octet within the tile
@@ -163,7 +193,7 @@ __global__ void __launch_bounds__(256) k_gptq_dequant(const int32_t *__restrict_
 #pragma unroll
       for (int j = 0; j < 8; j++) {
         const int64_t k = kq * 8 + j;
-        const int64_t g = g_idx ? (int64_t)__ldg(g_idx + k) : k / gs;
+        const int64_t g = (int64_t)__ldg(g_idx + k);
         const float s = __half2float(__ushort_as_half(__ldg(scales + g * N + o)));
         const uint32_t zw = static_cast<uint32_t>(__ldg(qzeros + g * (N / 8) + o / 8));
         const int zero = (int)((zw >> ((o % 8) * 4)) & 0xFu) + zadd;

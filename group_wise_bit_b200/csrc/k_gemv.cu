@@ -356,14 +356,26 @@ __global__ void __launch_bounds__(kThreads, 2)
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int ub = ks; ub < units; ub += KW * U) {
     uint32_t wa[U], wb[U];
+    // without g_idx the octet's group scale and zero word are loaded with its
+    // codes (gs is a multiple of 8: one group per octet), not after them
+    [[maybe_unused]] uint16_t sa_[U], sb_[U];
+    [[maybe_unused]] uint32_t za_[U], zb_[U];
 #pragma unroll
     for (int u = 0; u < U; u++) {
       const int un = ub + u * KW;
       wa[u] = wb[u] = 0u;
+      if constexpr (!GIDX) { sa_[u] = sb_[u] = 0; za_[u] = zb_[u] = 0u; }
       if (un < units) {
         const int64_t kq = (k0 + un * UNIT) / 8 + c;
         if (vA) wa[u] = (uint32_t)__ldg(qweight + kq * N + nA);
         if (vB) wb[u] = (uint32_t)__ldg(qweight + kq * N + nB);
+        if constexpr (!GIDX) {
+          const int64_t gq = (k0 + un * UNIT + c * 8) / gs;
+          sa_[u] = __ldg(scales + gq * N + nA);
+          sb_[u] = __ldg(scales + gq * N + nB);
+          za_[u] = (uint32_t)__ldg(qzeros + gq * NZ + nA / 8);
+          zb_[u] = (uint32_t)__ldg(qzeros + gq * NZ + nB / 8);
+        }
       }
     }
 #pragma unroll
@@ -375,11 +387,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       unpack_word<4>(wa[u], ra);
       unpack_word<4>(wb[u], rb);
       if constexpr (!GIDX) {
-        const int gq = (k0 + kbase) / gs;  // gs is a multiple of 8: one group per octet
-        const __half sAh = __ushort_as_half(__ldg(scales + (int64_t)gq * N + nA));
-        const __half sBh = __ushort_as_half(__ldg(scales + (int64_t)gq * N + nB));
-        const uint32_t zwA = (uint32_t)__ldg(qzeros + (int64_t)gq * NZ + nA / 8);
-        const uint32_t zwB = (uint32_t)__ldg(qzeros + (int64_t)gq * NZ + nB / 8);
+        const __half sAh = __ushort_as_half(sa_[u]);
+        const __half sBh = __ushort_as_half(sb_[u]);
+        const uint32_t zwA = za_[u];
+        const uint32_t zwB = zb_[u];
         const uint32_t zA = 0x6400u | (((zwA >> ((nA % 8) * 4)) & 0xFu) + (uint32_t)zadd);
         const uint32_t zB = 0x6400u | (((zwB >> ((nB % 8) * 4)) & 0xFu) + (uint32_t)zadd);
         const __half2 zA2 = __halves2half2(__ushort_as_half(zA), __ushort_as_half(zA));
