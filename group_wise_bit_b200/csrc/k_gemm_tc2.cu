@@ -569,6 +569,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer (the leader's)
     if (lane == 0 && leader) {
       int xi = 0, tc = 0, t, k0, k1;
+      // ring positions and phases, advanced without divisions; the operand
+      // descriptors of a slot differ from slot 0's only in the start-address field
+      // (16-byte units, shared-memory addresses stay below 2^18)
+      int sx = 0, sa = 0;
+      uint32_t px = 0, pa = 0;
+      const uint64_t xdesc0 = smem_desc_sw128(smem_u32(ringX)), adesc0 = smem_desc_sw128(smem_u32(ringA));
       bool ok = true;
       SegWalk sw(a, nk, unit, units);
       for (; ok && sw.next(t, k0, k1); tc++) {
@@ -577,17 +583,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(buf * BT);
         for (int k = k0; k < k1; k++, xi++) {
-          const int sx = xi % SX, sa = xi % SA;
-          if (*abort_flag || !mbar_wait(&afull[sa], (xi / SA) & 1) || !mbar_wait(&xfull[sx], (xi / SX) & 1)) {
+          // (a role that gave up makes these waits give up too: no flag check per step)
+          if (!mbar_wait(&afull[sa], pa) || !mbar_wait(&xfull[sx], px)) {
             *abort_flag = 1;
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(ringA + sa * P::AB), b0 = smem_u32(ringX + sx * P::XB);
+          const uint64_t ad0 = adesc0 + (uint64_t)(sa * (P::AB >> 4)), bd0 = xdesc0 + (uint64_t)(sx * (P::XB >> 4));
 #pragma unroll
           for (int kk = 0; kk < T::NMMA; kk++) {
-            const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
+            const uint64_t ad = ad0 + (uint64_t)(2 * kk), bd = bd0 + (uint64_t)(2 * kk);
             if constexpr (ATM) {
               const uint32_t at = tmem + ACOL + (uint32_t)(32 * sa + 8 * kk);
               if constexpr (kInt) umma_i8_ts_pair(d, at, bd, IDESC, (k - k0) | kk);
@@ -608,6 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(&xempty[sx]);
             umma_commit(&aempty[sa]);
           }
+          if (++sx == SX) { sx = 0; px ^= 1; }
+          if (++sa == SA) { sa = 0; pa ^= 1; }
         }
         if (!ok) break;
         if constexpr (PAIR == 2) umma_commit_pair(&accfull[buf]);
@@ -744,6 +752,120 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           named_bar_sync(1, 128);   // the staging tile is free for the next segment
+          continue;
+        }
+        if ((contrib || head) && (!kInt || a.acc == nullptr)) {
+          // Split tile, in chunks of 32 tokens through the staging buffer: two fp32
+          // (s32) partial chunks [32 tokens][128 rows] (double-buffered), then the
+          // bf16 / fp16 output chunk.  A contributing segment copies each chunk to its
+          // workspace slot with coalesced 16-byte stores.  The head pulls the next
+          // chunk of the first later unit's partial with cp.async while it finishes
+          // the current one (adding any further units' partials, in unit order, and
+          // its own accumulator), then writes the output chunk.
+          constexpr int CT = 32, NCH = BT / CT, CW = CT * kTileN / 4;        // tokens, chunks, 16-byte words
+          uint32_t *pq = reinterpret_cast<uint32_t *>(stage);                  // [2][CT][128] 32-bit
+          uint16_t *po = stage + 2 * CT * kTileN * 2;                            // [CT][128] 16-bit
+          const int tid = threadIdx.x - kFirstEpi * 32;
+          auto part = [&](int v, int c) {   // chunk c of CTA slot v's partial, as 16-byte words
+            return reinterpret_cast<const uint4 *>(a.ws + ((size_t)(v * PAIR + rank) * BT + c * CT) * kTileN);
+          };
+          auto pull = [&](int c) {          // chunk c of the first later unit's partial -> pq[c % 2]
+            const uint4 *src = part(vfirst, c);
+            uint4 *dst = reinterpret_cast<uint4 *>(pq + (c & 1) * CT * kTileN);
+#pragma unroll
+            for (int i = 0; i < CW / 128; i++) cp_async_16(dst + tid + 128 * i, src + tid + 128 * i, 16u);
+            cp_async_commit();
+          };
+          if (head && vlast >= vfirst) pull(0);
+          for (int c = 0; c < NCH; c++) {
+            uint32_t *pc = pq + (c & 1) * CT * kTileN;
+            if (head && vlast >= vfirst) {
+              if (c + 1 < NCH) {
+                pull(c + 1);
+                cp_async_wait<1>();
+              } else {
+                cp_async_wait<0>();
+              }
+              // further units' partials of this chunk, added to the words this thread pulled
+              for (int vv = vfirst + 1; vv <= vlast; vv++) {
+                const uint4 *src = part(vv, c);
+#pragma unroll
+                for (int i = 0; i < CW / 128; i++) {
+                  const uint4 w = __ldcg(src + tid + 128 * i);
+                  uint4 &d = reinterpret_cast<uint4 *>(pc)[tid + 128 * i];
+                  if constexpr (kInt) {
+                    d.x = (uint32_t)((int)d.x + (int)w.x); d.y = (uint32_t)((int)d.y + (int)w.y);
+                    d.z = (uint32_t)((int)d.z + (int)w.z); d.w = (uint32_t)((int)d.w + (int)w.w);
+                  } else {
+                    d.x = __float_as_uint(__uint_as_float(d.x) + __uint_as_float(w.x));
+                    d.y = __float_as_uint(__uint_as_float(d.y) + __uint_as_float(w.y));
+                    d.z = __float_as_uint(__uint_as_float(d.z) + __uint_as_float(w.z));
+                    d.w = __float_as_uint(__uint_as_float(d.w) + __uint_as_float(w.w));
+                  }
+                }
+              }
+              named_bar_sync(1, 128);
+            }
+            uint32_t v0[16], v1[16];
+            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * CT), v0);
+            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * CT + 16), v1);
+            tmem_ld_wait();
+            if (c == NCH - 1) {   // the accumulator is free for the next segment
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                if constexpr (PAIR == 2) mbar_arrive_remote(lead_accempty + buf * 8);
+                else mbar_arrive(&accempty[buf]);
+              }
+            }
+            if (contrib) {
+#pragma unroll
+              for (int j = 0; j < CT; j++) pc[j * kTileN + lrow] = j < 16 ? v0[j] : v1[j - 16];
+              named_bar_sync(1, 128);
+              uint4 *d4 = reinterpret_cast<uint4 *>(a.ws + ((size_t)blockIdx.x * BT + c * CT) * kTileN);
+#pragma unroll
+              for (int i = 0; i < CW / 128; i++) d4[tid + 128 * i] = reinterpret_cast<const uint4 *>(pc)[tid + 128 * i];
+              // (the next chunk fills the other buffer: no barrier needed here)
+            } else {
+#pragma unroll
+              for (int j = 0; j < CT; j++) {
+                const uint32_t u = j < 16 ? v0[j] : v1[j - 16];
+                const uint32_t p = vlast >= vfirst ? pc[j * kTileN + lrow] : 0u;
+                float f;
+                if constexpr (kInt) {
+                  const int m = m0 + c * CT + j;
+                  const int s32 = (int)u + (int)p;
+                  const int acc = F == Fmt::I8 ? s32 >> 4 : s32;
+                  f = (float)acc * ((m < a.M ? __ldg(a.sx + m) : 0.f) * swn);
+                } else {
+                  f = __uint_as_float(u) + __uint_as_float(p);
+                }
+                po[j * kTileN + lrow] = F == Fmt::Gptq ? __half_as_ushort(__float2half_rn(f))
+                                                       : __bfloat16_as_ushort(__float2bfloat16_rn(f));
+              }
+              named_bar_sync(1, 128);
+              const bool vec = (a.N % 8) == 0;
+#pragma unroll
+              for (int i = 0; i < CT * (kTileN / 8) / 128; i++) {
+                const int e = tid + 128 * i;
+                const int tok = e / (kTileN / 8), c8 = (e % (kTileN / 8)) * 8;
+                const int m = m0 + c * CT + tok, n = n0 + c8;
+                if (m >= a.M || n >= a.N) continue;
+                const uint16_t *src = po + tok * kTileN + c8;
+                if (vec && n + 8 <= a.N) {
+                  *reinterpret_cast<uint4 *>(a.y + (int64_t)m * a.N + n) = *reinterpret_cast<const uint4 *>(src);
+                } else {
+                  for (int k2 = 0; k2 < 8 && n + k2 < a.N; k2++) a.y[(int64_t)m * a.N + n + k2] = src[k2];
+                }
+              }
+              named_bar_sync(1, 128);   // po and this chunk's partial buffer are free
+            }
+          }
+          if (contrib) {   // publish the partial once all four warps stored theirs
+            __threadfence();
+            named_bar_sync(1, 128);
+            if (lead_thread) flag_publish(a.flags + blockIdx.x, *epoch_slot);
+          }
           continue;
         }
       }

@@ -113,6 +113,13 @@ __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *src, uin
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(src), "r"(src_bytes)
                : "memory");
 }
+// Groups this thread's cp.async copies issued so far; waits until at most N
+// of its groups are still in flight.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 // Arrive on `bar` once this thread's prior cp.async copies complete (the
 // barrier's expected count must include this arrival).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
