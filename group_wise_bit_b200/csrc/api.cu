@@ -142,7 +142,7 @@ gwb_status gwb_qmm_affine(const uint16_t *x, int64_t M, const uint32_t *wq, cons
   }
   if (bits == 2 && K % 64 != 0)
     return fail(GWB_ERR_UNSUPPORTED, "bits=2 needs K %% 64 == 0 on the tensor-core path (K=%lld)", (long long)K);
-  if (M >= 128) {
+  {   // the persistent stream-K GEMM; the per-tile kernel takes the layouts it does not stage
     const gwb_status s =
         gwb::launch_tc2_affine(x, M, wq, scales, biases, N, K, bits, group_size, y, as_stream(stream));
     if (s != GWB_ERR_UNSUPPORTED) return s;
@@ -289,7 +289,7 @@ gwb_status gptq_qmm_impl(const uint16_t *x, int64_t M, const int32_t *qweight, c
   if (M <= 8)
     return gwb::launch_gemv_gptq(x, (int)M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream),
                                  zadd);
-  if (M >= 128) {
+  {   // the persistent stream-K GEMM without g_idx; the per-tile kernel with it
     const gwb_status s =
         gwb::launch_tc2_gptq(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream), zadd);
     if (s != GWB_ERR_UNSUPPORTED) return s;
@@ -369,8 +369,7 @@ gwb_status gwb_gemm_i8i4(const int8_t *qx, const float *sx, int64_t M, const uin
   GWB_TRY(need(sx, "sx"));
   GWB_TRY(need(wq, "wq"));
   GWB_TRY(need(sw, "sw"));
-  if (M >= 128) return gwb::launch_tc2_i8i4(qx, sx, M, wq, sw, N, K, y, acc, as_stream(stream));
-  return gwb::launch_tc_i8i4(qx, sx, M, wq, sw, N, K, y, acc, as_stream(stream));
+  return gwb::launch_tc2_i8i4(qx, sx, M, wq, sw, N, K, y, acc, as_stream(stream));
 }
 
 gwb_status gwb_qpack_sym_i8(const float *w, int64_t N, int64_t K, int8_t *wq, float *sw, void *stream) {

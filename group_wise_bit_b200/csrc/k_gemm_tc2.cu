@@ -275,7 +275,10 @@ struct Plan2 {
   static constexpr int RB = (Tr<F, BITS>::RAW + Tr<F, BITS>::SC + 127) / 128 * 128;
   // ATM: a bf16 staging tile [BT tokens][128 rows] for the epilogue, so that it
   // frees the single accumulator before writing the output
-  static constexpr int EPI = ATM ? BT * kTileN * 2 : 0;
+  // The epilogue's staging: ATM, a whole bf16 tile (so that it frees the single
+  // accumulator before writing); otherwise the chunked staging of 32-token chunks
+  // (two 32-bit partial chunks and one 16-bit output chunk, 40 KB)
+  static constexpr int EPI = ATM ? BT * kTileN * 2 : 2 * 32 * kTileN * 4 + 32 * kTileN * 2;
   static constexpr int BUDGET = kMaxSmem - 1024 - 1024 - 1024;   // alignment, barriers, static
   static constexpr int SW8 = (BUDGET - EPI) / (XB + AB) > 8 ? 8 : (BUDGET - EPI) / (XB + AB);
   static constexpr int SA = ATM ? 8 : W8 ? SW8 : (PAIR == 2 ? 6 : 3);
@@ -754,7 +757,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           named_bar_sync(1, 128);   // the staging tile is free for the next segment
           continue;
         }
-        if ((contrib || head) && (!kInt || a.acc == nullptr)) {
+      }
+      // split tiles (and, without tensor-memory A, whole tiles too) through the
+      // chunked staging
+      if ((contrib || head || !ATM) && (!kInt || a.acc == nullptr)) {
+        {
           // Split tile, in chunks of 32 tokens through the staging buffer: two fp32
           // (s32) partial chunks [32 tokens][128 rows] (double-buffered), then the
           // bf16 / fp16 output chunk.  A contributing segment copies each chunk to its
@@ -807,8 +814,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               named_bar_sync(1, 128);
             }
             uint32_t v0[16], v1[16];
-            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * CT), v0);
-            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * CT + 16), v1);
+            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BT + c * CT), v0);
+            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BT + c * CT + 16), v1);
             tmem_ld_wait();
             if (c == NCH - 1) {   // the accumulator is free for the next segment
               tc_fence_before();
@@ -1071,24 +1078,38 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
   int units = kSMs / PAIR;
   if (max_units > 0 && max_units < units) units = max_units;
   const int nk = (a.K + Tr<F, BITS>::BK - 1) / Tr<F, BITS>::BK;
-  // Stream-K when whole tiles would leave part of the last wave idle and every
-  // unit gets a few K steps; else whole tiles per unit.
+  // Fewer tiles than units: each tile is split into s equal K parts on s units
+  // (all parts finish together, so no head waits on a longer tail); s = 1 means
+  // whole tiles.  More tiles than units: stream-K over all units when whole tiles
+  // would leave part of the last wave idle and every unit gets a few K steps.
   int grid_units = a.T < units ? a.T : units;
+  int split_units = units;
+  bool want_ws;
+  if (a.T < units) {
+    int s = units / a.T;
+    if (s > 8) s = 8;                              // at most 7 partials per finished tile
+    while (s > 1 && nk / s < 4) s--;               // and at least 4 K steps per part
+    split_units = a.T * s;
+    want_ws = s > 1;
+  } else {
+    want_ws = a.T % units != 0 && (int64_t)a.T * nk >= 4LL * units;
+  }
   a.ws = nullptr;
   a.flags = nullptr;
   a.ctr = nullptr;
   a.stall = 0;
-  if (a.T % units != 0 && (int64_t)a.T * nk >= 4LL * units) {
+  if (want_ws) {
     uint32_t *ws = nullptr, *fl = nullptr, *ctr = nullptr;
     bool have_ws = false;
     if (fixed_ws) {
       // flags of the units, then the two counters, cleared for this call
       ws = fixed_ws;
-      fl = fixed_ws + (size_t)units * PAIR * BT * kTileN;
-      ctr = fl + units * PAIR;
-      have_ws = cudaMemsetAsync(fl, 0, ((size_t)units * PAIR + 2) * 4, st) == cudaSuccess;
+      fl = fixed_ws + (size_t)split_units * PAIR * BT * kTileN;
+      ctr = fl + split_units * PAIR;
+      have_ws = cudaMemsetAsync(fl, 0, ((size_t)split_units * PAIR + 2) * 4, st) == cudaSuccess;
     } else {
-      have_ws = stream_workspace(st, (size_t)kSMs * BT * kTileN * 4, kSMs + 2, &ws, &fl);
+      // sized for the widest token tile, so that later calls never grow it
+      have_ws = stream_workspace(st, (size_t)kSMs * 256 * kTileN * 4, kSMs + 2, &ws, &fl);
       ctr = fl + kSMs;
     }
     if (have_ws) {
@@ -1096,7 +1117,7 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
       a.flags = fl;
       a.ctr = ctr;
       a.stall = g_stall_next.exchange(0);
-      grid_units = units;
+      grid_units = split_units;
     }
   }
   cudaLaunchConfig_t cfg = {};
@@ -1122,6 +1143,8 @@ template <Fmt F, int BITS>
 gwb_status dispatch2(int64_t M, const void *x, CUtensorMapDataType xdt, int xelem, const CUtensorMap &tw,
                      const CUtensorMap &tsb, const Args &a, cudaStream_t st, uint32_t *fixed_ws = nullptr,
                      int max_units = 0) {
+  if (M <= 32) return run_tc2<F, BITS, 32, 1, false>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
+  if (M <= 64) return run_tc2<F, BITS, 64, 1, false>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
   if (M <= 128) return run_tc2<F, BITS, 128, 1, false>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
   return run_tc2<F, BITS, 256, 2, kAInTmem>(x, xdt, xelem, tw, tsb, a, st, fixed_ws, max_units);
 }
