@@ -88,24 +88,30 @@ def _call(name, *args):
         raise GwbError(name, st, lib().gwb_last_error().decode())
 
 
-def _stream():
-    return _P(torch.cuda.current_stream().cuda_stream)
+try:   # the raw handle of the current stream, without building a Stream object per call
+    _raw_stream = torch._C._cuda_getCurrentRawStream
+
+    def _stream():
+        return _raw_stream(torch.cuda.current_device())
+except AttributeError:   # pragma: no cover - older torch
+    def _stream():
+        return torch.cuda.current_stream().cuda_stream
 
 
 def _ptr(t):
-    return None if t is None else _P(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _dev(t, name, dtypes, shape=None):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
+    if t.device.type != "cuda":
         raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
     if t.dtype not in dtypes:
         raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != shape:
         raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
     return t
 

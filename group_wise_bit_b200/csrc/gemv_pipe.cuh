@@ -80,9 +80,12 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <functional>
 #include <map>
 #include <mutex>
 #include <type_traits>
+#include <unordered_map>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -1061,8 +1064,50 @@ CUresult weight_maps(const uint32_t *wq, const uint16_t *scales, const uint16_t 
   return r;
 }
 
+// The launch set-up of one weight (or weight pair) at one shape: the plan, the
+// weight-dependent kernel arguments and the weights' tensor maps.  It depends
+// only on the device, the weight pointers and N, K (a tensor map is a function
+// of its address, sizes and strides), so it is computed once and cached.
+struct PipeSetup {
+  PipeArgs a;
+  int P, S;
+  size_t smem;
+  MapSet<6> maps;
+};
+struct PipeKey {
+  int dev;
+  const void *w[6];
+  int64_t N, K;
+  bool operator==(const PipeKey &o) const {
+    return dev == o.dev && N == o.N && K == o.K && std::equal(w, w + 6, o.w);
+  }
+};
+struct PipeKeyHash {
+  size_t operator()(const PipeKey &k) const {
+    size_t h = std::hash<int64_t>()(k.N * 1315423911ll + k.K) ^ (size_t)k.dev;
+    for (const void *p : k.w) h = h * 1099511628211ull ^ std::hash<const void *>()(p);
+    return h;
+  }
+};
+struct PipeCache {
+  std::mutex mu;
+  std::unordered_map<PipeKey, PipeSetup, PipeKeyHash> map;
+  bool get(const PipeKey &k, PipeSetup &out) {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = map.find(k);
+    if (it == map.end()) return false;
+    out = it->second;
+    return true;
+  }
+  void put(const PipeKey &k, const PipeSetup &v) {
+    std::lock_guard<std::mutex> lk(mu);
+    if (map.size() >= 4096) map.clear();   // bounded: a model holds far fewer weights
+    map[k] = v;
+  }
+};
+
 template <int BITS, int GS, int MP, int OP>
-gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
+gwb_status setup_pipe(const PipeIn &in, PipeSetup &su) {
   using C = PCfg<BITS, GS>;
   const int64_t N = in.N, K = in.K;
   const int64_t G = K / GS;
@@ -1160,35 +1205,61 @@ gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
   a.sb_swap = swap;
   a.sb_swap2 = swap2;
 
+  su.a = a;
+  su.P = best.P;
+  su.S = best.S;
+  su.smem = best.smem;
+  su.maps.m[0] = tw;
+  su.maps.m[1] = tsb;
+  su.maps.m[2] = tb;
+  su.maps.m[3] = tw2;
+  su.maps.m[4] = tsb2;
+  su.maps.m[5] = tb2;
+  return GWB_OK;
+}
+
+template <int BITS, int GS, int MP, int OP>
+gwb_status run_pipe(const PipeIn &in, cudaStream_t st) {
+  static PipeCache cache;   // one per kernel instance
+  if ((in.K / GS) % 8 != 0 || (in.K * BITS / 8) % 16 != 0) return GWB_ERR_UNSUPPORTED;   // (see setup_pipe)
+  int dev = 0;
+  const cudaError_t de = cudaGetDevice(&dev);
+  if (de != cudaSuccess) return fail(GWB_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(de));
+  const PipeKey key{dev, {in.wq, in.scales, in.biases, in.wq2, in.scales2, in.biases2}, in.N, in.K};
+  PipeSetup su;
+  if (!cache.get(key, su)) {
+    const gwb_status s = setup_pipe<BITS, GS, MP, OP>(in, su);
+    if (s != GWB_OK) return s;
+    cache.put(key, su);
+  }
+  // the arguments of this call
+  PipeArgs a = su.a;
+  a.x = in.x; a.x2 = in.x2; a.resid = in.resid; a.sw = in.sw; a.sx = in.sx; a.acc = in.acc;
+  a.y = in.y; a.y2 = in.y2;
+  a.M = in.M;
+
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)best.P, (unsigned)best.S);
+  cfg.gridDim = dim3((unsigned)su.P, (unsigned)su.S);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = best.smem;
+  cfg.dynamicSmemBytes = su.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   int na = 0;
   attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[na].val.programmaticStreamSerializationAllowed = 1;
   na++;
-  if (best.S > 1) {
+  if (su.S > 1) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
     attr[na].val.clusterDim.x = 1;
-    attr[na].val.clusterDim.y = (unsigned)best.S;
+    attr[na].val.clusterDim.y = (unsigned)su.S;
     attr[na].val.clusterDim.z = 1;
     na++;
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
   MapsOf<OP> maps;
-  maps.m[0] = tw;
-  maps.m[1] = tsb;
-  maps.m[2] = tb;
-  if constexpr (OP == kOpDual) {
-    maps.m[3] = tw2;
-    maps.m[4] = tsb2;
-    maps.m[5] = tb2;
-  }
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, maps, a);
+  for (int i = 0; i < (OP == kOpDual ? 6 : 3); i++) maps.m[i] = su.maps.m[i];
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gemv_pipe<BITS, GS, MP, OP>, maps, a);
   if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "decode GEMV launch: %s", cudaGetErrorString(e));
   return GWB_OK;
 }
