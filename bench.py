@@ -107,17 +107,23 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def traffic_for(kernel_key):
-    """Per-launch DRAM bytes (read + write) of a kernel from the committed ncu summary, or None."""
+def traffic_entry(kernel_key):
+    """(per-launch DRAM bytes read + written, source summary) of a kernel from the committed ncu
+    summaries, or (None, None)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
             for line in f:
                 parts = line.split()
                 if parts and not parts[0].startswith("#") and parts[0] == kernel_key:
-                    return int(parts[1])
+                    return int(parts[1]), parts[2]
     except Exception:
         pass
-    return None
+    return None, None
+
+
+def traffic_for(kernel_key):
+    """Per-launch DRAM bytes (read + write) of a kernel from the committed ncu summary, or None."""
+    return traffic_entry(kernel_key)[0]
 
 
 class ClockSampler:
@@ -373,7 +379,7 @@ def run_works(works, stream):
     return [(w, graph_us(w.launch, w.n, stream)) for w in works]
 
 
-def aggregate(key, timed, peak, peak_source, unit, bound, traffic=None, extra=None):
+def aggregate(key, timed, peak, peak_source, unit, bound, traffic_key=None, extra=None):
     """Sum of work over sum of time across a workload's shapes, with its roofline."""
     work = (lambda w: w.nbytes) if bound == "hbm" else (lambda w: w.flops)
     scale = 1e3 if bound == "hbm" else 1e6          # bytes/us -> GB/s; ops/us -> T(FL)OP/s
@@ -382,7 +388,12 @@ def aggregate(key, timed, peak, peak_source, unit, bound, traffic=None, extra=No
     kernels = sorted({w.kernel for w, _ in timed})
     out = {"value": round(val, 1), "unit": unit,
            "shapes": [{"case": w.key, "us": round(us, 2), unit: round(work(w) / us / scale, 1)} for w, us in timed],
-           "roofline": roofline(" + ".join(kernels), bound, val, peak, unit, peak_source, traffic)}
+           "roofline": roofline(" + ".join(kernels), bound, val, peak, unit, peak_source)}
+    if traffic_key:
+        # DRAM bytes of one launch of the captured shape (profiles/<case>), not of the aggregate
+        tb, case = traffic_entry(traffic_key)
+        out["roofline"]["traffic"] = tb
+        out["roofline"]["traffic_case"] = case
     if extra:
         out.update(extra)
     return out
@@ -685,33 +696,37 @@ def run_gpu(args, world, rank, local):
             key = f"prefill_m{M}"
             if M <= 128:
                 out[key] = aggregate(key, t[key], hbm_peak, hbm_src, "GB/s", "hbm",
-                                     traffic=traffic_for(f"k_tc_affine4_m{M}"))
+                                     traffic_key=f"k_tc2_affine4_m{M}")
             if M >= 128:
                 k2 = key if M > 128 else key + "_tflops"
                 out[k2] = aggregate(key, t[key], bf16_peak, bf16_src, "TFLOP/s", "tensor",
-                                    traffic=traffic_for(f"k_tc2_affine4_m{M}"))
+                                    traffic_key=f"k_tc2_affine4_m{M}")
         for key in ("prefill_m2048_b8", "prefill_m2048_gs32", "prefill_m2048_gs128"):
             out[key] = aggregate(key, t[key], bf16_peak, bf16_src, "TFLOP/s", "tensor")
-        out["gptq_dequant"] = aggregate("gptq_dequant", t["gptq_dequant"], hbm_peak, hbm_src, "GB/s", "hbm")
+        out["gptq_dequant"] = aggregate("gptq_dequant", t["gptq_dequant"][:1], hbm_peak, hbm_src, "GB/s", "hbm",
+                                        traffic_key="k_gptq_dequant",
+                                        extra={"permuted_g_idx": aggregate("gptq_dequant", t["gptq_dequant"][1:],
+                                                                           hbm_peak, hbm_src, "GB/s", "hbm")})
         for M in (1, 32, 1024):
             key = f"gptq_m{M}"
             tm = t[key]
             if M >= 512:
                 out[key] = aggregate(key, tm[:1], bf16_peak, bf16_src + " (fp16 peak taken equal to bf16)",
-                                     "TFLOP/s", "tensor", extra={"permuted_g_idx": aggregate(
+                                     "TFLOP/s", "tensor", traffic_key="k_tc2_gptq_m1024", extra={"permuted_g_idx": aggregate(
                                          key, tm[1:], bf16_peak, bf16_src, "TFLOP/s", "tensor")})
             else:
                 out[key] = aggregate(key, tm[:1], hbm_peak, hbm_src, "GB/s", "hbm",
+                                     traffic_key="k_gemv_gptq_m1" if M == 1 else None,
                                      extra={"permuted_g_idx": aggregate(key, tm[1:], hbm_peak, hbm_src, "GB/s", "hbm")})
         for fmt in ("w4a8", "w8a8"):
             for M in INT8_M:
                 key = f"{fmt}_m{M}"
                 if M >= 512:
                     out[key] = aggregate(key, t[key], i8peak, i8src, "TOP/s", "tensor",
-                                         traffic=traffic_for(f"k_tc2_{fmt}_m{M}"))
+                                         traffic_key=f"k_tc2_{fmt}_m{M}")
                 else:
                     out[key] = aggregate(key, t[key], hbm_peak, hbm_src, "GB/s", "hbm")
-        out["w8a8_m1"] = aggregate("w8a8_m1", t["w8a8_m1"], hbm_peak, hbm_src, "GB/s", "hbm")
+        out["w8a8_m1"] = aggregate("w8a8_m1", t["w8a8_m1"], hbm_peak, hbm_src, "GB/s", "hbm", traffic_key="k_gemv_pipe_i8w8")
         out["int8_peak_tops"] = round(i8peak, 1)
     out["decode_mlp_fused"] = run_mlp_fused(gwb, dev, stream, hbm_peak, hbm_src)
     out["w4a8_decode_fused"] = run_w4a8_decode(gwb, dev, stream, hbm_peak, hbm_src)
@@ -781,7 +796,7 @@ def run_w4a8_decode(gwb, dev, stream, hbm_peak, hbm_src, N=14336, K=4096, M=1):
     return {"value": round(gbs, 1), "unit": "GB/s", "N": N, "K": K, "M": M,
             "us_fused": round(us_f, 2), "us_two_launch": round(us_t, 2),
             "roofline": roofline("k_gemv_pipe<4,64,1,w4a8> (per-token int8 quantization inside)", "hbm", gbs,
-                                 hbm_peak, "GB/s", hbm_src, bytes_per_launch=nbytes)}
+                                 hbm_peak, "GB/s", hbm_src, traffic_for("k_gemv_pipe_w4a8"), bytes_per_launch=nbytes)}
 
 
 def run_mlp_fused(gwb, dev, stream, hbm_peak, hbm_src, bits=4, M=1):
@@ -904,18 +919,31 @@ def run_layer(args):
                 gwb.gemv_gate_up(x, ws[0], ws[1], bits, GS, y_gate=y, y_up=y2)
             else:
                 gwb.gemv_silu_gate(x, x2, *ws[0], bits, GS, x_resid=res, y=y)
-    elif args.fmt == "gptq":
+    elif args.fmt in ("gptq", "gptq_perm", "gptq_dequant"):
+        perm = args.fmt == "gptq_perm"
         sets = []
         for s in range(2):
-            qw, sc, qz, _ = synth.gptq_quartet(K, N, GPTQ_GS, seed=s)
-            sets.append((qw.to(dev), sc.to(dev), qz.to(dev)))
+            qw, sc, qz, gi = synth.gptq_quartet(K, N, GPTQ_GS, seed=s, permuted=perm)
+            sets.append((qw.to(dev), sc.to(dev), qz.to(dev), gi.to(dev) if perm else None))
         x = synth.activations(M, K, seed=1, dtype=torch.float16).to(dev)
         y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        wo = torch.empty((N, K), dtype=torch.float16, device=dev) if args.fmt == "gptq_dequant" else None
         bits = 4
 
         def launch(i):
-            q, s, z = sets[i % 2]
-            gwb.gptq_qmm(x, q, s, z, None, GPTQ_GS, y=y)
+            q, s, z, gi = sets[i % 2]
+            if wo is not None:
+                gwb.gptq_dequant(q, s, z, None, GPTQ_GS, out=wo)
+            else:
+                gwb.gptq_qmm(x, q, s, z, gi, GPTQ_GS, y=y)
+    elif args.fmt == "w4a8_fused":
+        sets = [int8_operands(gwb, dev, "w4a8", N, K, M, seed=s)[:2] for s in range(2)]
+        x = synth.activations(M, K, seed=1).to(dev)
+        bits = 4
+
+        def launch(i):
+            wq, sw = sets[i % 2]
+            gwb.gemv_w4a8(x, wq, sw, y=y)
     else:
         sets = [int8_operands(gwb, dev, args.fmt, N, K, M, seed=s) for s in range(2)]
         gemm = int8_gemm(gwb, args.fmt)
@@ -949,8 +977,12 @@ def run_layer(args):
         nbytes = 2 * gemv_bytes(N, K, bits, M=M) - 2 * M * K      # x is read once
     elif args.fmt == "silu_resid":
         nbytes = gemv_bytes(N, K, bits, M=M) + 2 * M * K + 2 * M * N   # up and the residual
-    elif args.fmt == "gptq":
-        nbytes = gptq_bytes(K, N, GPTQ_GS, M, False) if M <= 32 else None
+    elif args.fmt == "gptq_dequant":
+        nbytes = gptq_dequant_bytes(K, N, GPTQ_GS, False)
+    elif args.fmt in ("gptq", "gptq_perm"):
+        nbytes = gptq_bytes(K, N, GPTQ_GS, M, args.fmt == "gptq_perm") if M <= 32 else None
+    elif args.fmt == "w4a8_fused":
+        nbytes = N * K // 2 + 4 * N + 2 * M * K + 2 * M * N
     else:
         nbytes = int8_bytes(N, K, M, bits) if M <= 64 else None
     out = {"layer": {"fmt": args.fmt, "N": N, "K": K, "bits": bits, "group_size": GS, "M": M},
@@ -958,7 +990,7 @@ def run_layer(args):
     if nbytes:
         out["GB/s"] = round(nbytes / us / 1e3, 1)
     else:
-        out["TFLOP/s" if args.fmt in ("affine", "gptq") else "TOP/s"] = round(2.0 * M * N * K / us / 1e6, 1)
+        out["TFLOP/s" if args.fmt in ("affine", "gptq", "gptq_perm") else "TOP/s"] = round(2.0 * M * N * K / us / 1e6, 1)
     print(json.dumps(out), flush=True)
 
 
@@ -970,8 +1002,10 @@ def main():
     ap.add_argument("--impl", choices=["gwb", "reference"], default="gwb")
     ap.add_argument("--no-prefill", action="store_true",
                     help="time the decode sweep (and the fused decode products) only")
-    ap.add_argument("--fmt", choices=["affine", "w4a8", "w8a8", "gate_up", "silu_resid", "gptq"], default="affine",
-                    help="--layer: weight format (affine: MLX group-wise, bits from --layer)")
+    ap.add_argument("--fmt", choices=["affine", "w4a8", "w8a8", "gate_up", "silu_resid", "gptq", "gptq_perm",
+                                      "gptq_dequant", "w4a8_fused"], default="affine",
+                    help="--layer: weight format (affine: MLX group-wise, bits from --layer; gptq*: N,K = out, in "
+                         "features at group size 128)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the CPU baseline leg (and with it the parity check before timing)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
