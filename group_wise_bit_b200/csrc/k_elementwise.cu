@@ -8,6 +8,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "dequant.cuh"
 #include "internal.h"
 
 namespace gwb {
@@ -168,18 +169,14 @@ __global__ void __launch_bounds__(256) k_gptq_dequant(const int32_t *__restrict_
     }
 #pragma unroll
     for (int i = 0; i < 8; i++) {
+      // pairs of fp16 (1024 + q) - (1024 + zero) = q - zero (exact), times the fp16
+      // scale: one IEEE rounding of the exact product, as the scalar recipe
       const int kql = kb * 8 + i;
-      const float s = __half2float(__ushort_as_half(sh[i]));
-      const int zero = (int)((zw[i] >> ((o % 8) * 4)) & 0xFu) + zadd;
-      uint32_t packed[4];
-#pragma unroll
-      for (int j = 0; j < 8; j++) {
-        const int q = (int)((word[i] >> (j * 4)) & 0xFu);
-        const uint16_t h = __half_as_ushort(__float2half_rn(__fmul_rn(s, (float)(q - zero))));
-        if (j & 1) packed[j / 2] |= (uint32_t)h << 16;
-        else packed[j / 2] = h;
-      }
-      *reinterpret_cast<uint4 *>(tile + nl * kGdRow + kql * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      const uint32_t zv = 0x6400u | (((zw[i] >> ((o % 8) * 4)) & 0xFu) + (uint32_t)zadd);
+      const uint32_t sv = sh[i];
+      const uint32_t z2[4] = {zv | (zv << 16), zv | (zv << 16), zv | (zv << 16), zv | (zv << 16)};
+      const uint32_t s2[4] = {sv | (sv << 16), sv | (sv << 16), sv | (sv << 16), sv | (sv << 16)};
+      *reinterpret_cast<uint4 *>(tile + nl * kGdRow + kql * 16) = dq::dq_gptq(word[i], z2, s2);
     }
   } else if (o < N) {
     // g_idx: every in-feature has its own group

@@ -183,7 +183,8 @@ struct Args {
   int sc_tma;               // affine: scales + biases arrive by TMA as [2 arrays][128 rows][8 groups]
   int sc_swap;              //   ... with the biases first (they sit below the scales in memory)
   int zadd;                 // gptq: added to the stored zero (1: GPTQ's convention, 0: AWQ's)
-  int Nt, T;                // feature tiles, tiles
+  int Nt, Mt, T;            // feature tiles, token tiles, tiles (token tiles fastest)
+  int dpw;                  // stream-K: whole waves walked round robin before the split tail
   const uint16_t *scales;   // affine: bf16 [N, K/gs];   gptq: fp16 [K/gs, N]
   const uint16_t *biases;   // affine: bf16 [N, K/gs]
   const int32_t *qzeros;    // gptq: [K/gs, N/8]
@@ -197,24 +198,35 @@ struct Args {
   int stall;                // a test made this launch's heads wait for an epoch nobody publishes
 };
 
-// A unit's contiguous share of the flattened (tile, K step) iteration space,
-// walked as segments of one tile each.  With a workspace the shares are equal
-// (stream-K: a tile may be split between units); without one they are whole
-// tiles.
+// A unit's work, walked as segments of one tile each: first whole tiles taken
+// round robin (unit, unit + units, ...: the units running at one time work on
+// consecutive tiles, which share their feature tile's weights and the token
+// tiles' activations through L2), then, with a workspace, an equal contiguous
+// share of the flattened (tile, K step) space of the remaining tiles (stream-K:
+// a tile may be split between units).  Without a workspace all tiles are whole.
 struct SegWalk {
   int64_t L, Le;
-  int nk;
-  __device__ SegWalk(const Args &a, int nk_, int unit, int units) : nk(nk_) {
-    const int64_t W = (int64_t)a.T * nk_;
+  int nk, dp_t, dp_left, step;
+  __device__ SegWalk(const Args &a, int nk_, int unit, int units) : nk(nk_), dp_t(unit), step(units) {
     if (a.ws) {
-      L = (int64_t)unit * W / units;
-      Le = (int64_t)(unit + 1) * W / units;
+      dp_left = a.dpw;
+      const int64_t T0 = (int64_t)a.dpw * units * nk_, W = (int64_t)a.T * nk_ - T0;
+      L = T0 + (int64_t)unit * W / units;
+      Le = T0 + (int64_t)(unit + 1) * W / units;
     } else {
-      L = (int64_t)unit * a.T / units * nk_;
-      Le = (int64_t)(unit + 1) * a.T / units * nk_;
+      dp_left = unit < a.T ? (a.T - 1 - unit) / units + 1 : 0;
+      L = Le = 0;
     }
   }
   __device__ bool next(int &t, int &k0, int &k1) {
+    if (dp_left > 0) {
+      t = dp_t;
+      dp_t += step;
+      dp_left--;
+      k0 = 0;
+      k1 = nk;
+      return true;
+    }
     if (L >= Le) return false;
     t = (int)(L / nk);
     k0 = (int)(L - (int64_t)t * nk);
@@ -473,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       SegWalk sw(a, nk, unit, units);
       while (ok && sw.next(t, k0, k1)) {
-        const int mx = (t / a.Nt) * BT + rank * XT;    // first token of this CTA's half
+        const int mx = (t % a.Mt) * BT + rank * XT;    // first token of this CTA's half
         for (int k = k0; k < k1; k++, it++) {
           const int s = it % SX;
           if (*abort_flag || !mbar_wait(&xempty[s], ((it / SX) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
@@ -500,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       SegWalk sw(a, nk, unit, units);
       while (ok && sw.next(t, k0, k1)) {
-        const int n0 = (t % a.Nt) * kTileN * PAIR + rank * kTileN;
+        const int n0 = (t / a.Mt) * kTileN * PAIR + rank * kTileN;
         for (int k = k0; k < k1; k++, it++) {
           const int s = it % SA;
           if (*abort_flag || !mbar_wait(&aempty[s], ((it / SA) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
@@ -522,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     SegWalk sw(a, nk, unit, units);
     while (ok && sw.next(t, k0, k1)) {
-      const int n0 = (t % a.Nt) * kTileN * PAIR + rank * kTileN;
+      const int n0 = (t / a.Mt) * kTileN * PAIR + rank * kTileN;
       for (int k = k0; k < k1; k++, it++) {
         const int s = it % SR;
         if (*abort_flag || !mbar_wait(&rempty[s], ((it / SR) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
@@ -681,17 +693,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     SegWalk sw(a, nk, unit, units);
     for (; sw.next(t, k0, k1); tc++) {
       const int buf = tc % NACC, use = tc / NACC;
-      const int n0 = (t % a.Nt) * kTileN * PAIR + rank * kTileN, m0 = (t / a.Nt) * BT;
+      const int n0 = (t / a.Mt) * kTileN * PAIR + rank * kTileN, m0 = (t % a.Mt) * BT;
       if (*abort_flag || !mbar_wait(&accfull[buf], use & 1)) { *abort_flag = 1; break; }
       tc_fence_after();
       const bool contrib = k0 > 0;                  // store a partial
       const bool head = k0 == 0 && k1 < nk;         // finish a split tile
       int vfirst = 0, vlast = -1;                   // contributing units of a split tile
       if (head) {
-        const int64_t W = (int64_t)a.T * nk, tile_end = (int64_t)(t + 1) * nk;
+        // the later units whose stream-K shares hold the rest of this tile
+        const int64_t T0 = (int64_t)a.dpw * units * nk, W = (int64_t)a.T * nk - T0;
+        const int64_t tile_end = (int64_t)(t + 1) * nk;
         vfirst = unit + 1;
         vlast = unit;
-        while (vlast + 1 < units && (int64_t)(vlast + 1) * W / units < tile_end) vlast++;
+        while (vlast + 1 < units && T0 + (int64_t)(vlast + 1) * W / units < tile_end) vlast++;
         if (lead_thread) {
           for (int v = vfirst; v <= vlast; v++) {
             const uint32_t *f = a.flags + v * PAIR + rank;
@@ -1067,7 +1081,9 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
                        (uint32_t)(BT / PAIR), CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != GWB_OK) return s;
   a.Nt = (a.N + kTileN * PAIR - 1) / (kTileN * PAIR);
-  a.T = a.Nt * ((a.M + BT - 1) / BT);
+  a.Mt = (a.M + BT - 1) / BT;
+  a.T = a.Nt * a.Mt;
+  a.dpw = 0;
   auto kern = k_tc2<F, BITS, BT, PAIR, ATM>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -1118,6 +1134,9 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
       a.ctr = ctr;
       a.stall = g_stall_next.exchange(0);
       grid_units = split_units;
+      // all but the last one or two waves of whole tiles go round robin; stream-K
+      // balances the rest
+      a.dpw = a.T >= 2 * split_units ? a.T / split_units - 1 : 0;
     }
   }
   cudaLaunchConfig_t cfg = {};
