@@ -68,8 +68,13 @@ gwb_status launch_gemv_gate_up(const uint16_t *x, int M, const uint32_t *wq_gate
 gwb_status launch_gemv_silu_gate(const uint16_t *gate, const uint16_t *up, int M, const uint32_t *wq,
                                  const uint16_t *scales, const uint16_t *biases, int64_t N, int64_t K, int bits,
                                  int gs, const uint16_t *resid, uint16_t *y, cudaStream_t st);
-// TMEM-operand tensor-core GEMV (the main decode kernel); GWB_ERR_UNSUPPORTED
-// (without a message) when the layout is outside what it covers.
+// GPTQ / AWQ GEMV: the shared-memory streamed kernel where the layout allows
+// (launch_gemv_gptq_pipe: N % 32 == 0, K % 256 == 0, 16-byte aligned weight
+// tensors, M <= 8; GWB_ERR_UNSUPPORTED without a message otherwise), else the
+// register-fed one.
+gwb_status launch_gemv_gptq_pipe(const uint16_t *x, int M, const int32_t *qweight, const uint16_t *scales,
+                                 const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
+                                 uint16_t *y, cudaStream_t st, int zadd);
 gwb_status launch_gemv_gptq(const uint16_t *x, int M, const int32_t *qweight, const uint16_t *scales,
                             const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
                             uint16_t *y, cudaStream_t st, int zadd = 1);
@@ -83,7 +88,7 @@ gwb_status launch_tc_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, 
                           uint16_t *y, cudaStream_t st, int zadd = 1);
 gwb_status launch_tc_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
                           int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
-// Persistent tensor-core GEMM (M >= 128); GWB_ERR_UNSUPPORTED (without a
+// Persistent tensor-core GEMM (M > 8); GWB_ERR_UNSUPPORTED (without a
 // message) when the layout needs the per-tile kernel (unstaged scales, g_idx).
 gwb_status launch_tc2_affine(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,
                              const uint16_t *biases, int64_t N, int64_t K, int bits, int gs, uint16_t *y,

@@ -166,6 +166,7 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 constexpr int kWarps = 15;
 constexpr int kThreads = kWarps * 32;
 constexpr int kDqWarps = 8;
+constexpr int kDqGroupWarps = kDqWarps / 2;   // dequantizer warps per K step (two groups alternate)
 constexpr int kFirstDq = 3, kFirstEpi = 11;
 constexpr int kTileN = 128;      // output features per tile (tensor-core M)
 constexpr int kMaxSmem = 232448;
@@ -308,23 +309,31 @@ __device__ __forceinline__ void put4(uint32_t (&o)[16], int j, uint4 v) {
   o[4 * j] = v.x; o[4 * j + 1] = v.y; o[4 * j + 2] = v.z; o[4 * j + 3] = v.w;
 }
 
+// Affine with scales by TMA: the 8-group block of scales and biases travels
+// only with the first two steps of a segment and of each new block (every 8
+// groups: 4 to 16 steps), one for each dequantizer group (they take alternate
+// steps); the dequantizers keep their row's block in registers.
+__device__ __forceinline__ bool affine_box_step(int k, int k0, int gs_log2) {
+  constexpr int BK = Tr<Fmt::Affine, 4>::BK;
+  return k - k0 < 2 || ((k * BK) & ((8 << gs_log2) - 1)) < 2 * BK;
+}
+
 // Dequantizes K step `k` (row r, half h of the step) from the R stage into the
 // 16 words of A the thread owns: o[4j .. 4j+3] = 16-byte chunk 4h + j of row r
 // (k = 8 (4h + j) .. +7 for 16-bit operands, 16 (4h + j) .. +15 for int8).
+// sbv: affine with scales by TMA, the row's block of 8 scales and 8 biases.
 template <Fmt F, int BITS>
 __device__ __forceinline__ void dequant_words(const Args &a, int k, int r, int h, const unsigned char *R,
-                                              uint32_t (&o)[16]) {
+                                              const uint4 (&sbv)[2], uint32_t (&o)[16]) {
   using T = Tr<F, BITS>;
   constexpr int BK = T::BK;
   const int kh = k * BK + h * (BK / 2);    // first k of this thread's half step
   if constexpr (F == Fmt::Affine) {
     float sf, bfv;
     if (a.sc_tma) {
-      // the row's 8 scales (16 bytes, one conflict-free load) of the aligned
-      // block of 8 groups that holds this half step's group
+      // the half step's group within the row's block of 8 groups
       const int g8 = (kh >> a.gs_log2) & 7;
-      const uint4 *box = reinterpret_cast<const uint4 *>(R + T::RAW);
-      const uint4 vs = box[a.sc_swap ? kTileN + r : r], vb = box[a.sc_swap ? r : kTileN + r];
+      const uint4 vs = sbv[0], vb = sbv[1];
       const int wsel = g8 >> 1;
       const uint32_t ws = wsel == 0 ? vs.x : wsel == 1 ? vs.y : wsel == 2 ? vs.z : vs.w;
       const uint32_t wb = wsel == 0 ? vb.x : wsel == 1 ? vb.y : wsel == 2 ? vb.z : vb.w;
@@ -443,10 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; s++) { mbar_init(&xfull[s], 1); mbar_init(&xempty[s], 1); }
-    for (int s = 0; s < SA; s++) { mbar_init(&afull[s], F == Fmt::W8 ? 1 : kDqWarps * PAIR); mbar_init(&aempty[s], 1); }
+    for (int s = 0; s < SA; s++) { mbar_init(&afull[s], F == Fmt::W8 ? 1 : kDqGroupWarps * PAIR); mbar_init(&aempty[s], 1); }
     for (int s = 0; s < SR; s++) {
       mbar_init(&rfull[s], 1 + (F == Fmt::Affine && a.sc_tma ? 0 : T::CP));
-      mbar_init(&rempty[s], kDqWarps);
+      mbar_init(&rempty[s], kDqGroupWarps);
     }
     for (int b = 0; b < 2; b++) { mbar_init(&accfull[b], 1); mbar_init(&accempty[b], 4 * PAIR); }
     *abort_flag = 0;
@@ -540,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*abort_flag || !mbar_wait(&rempty[s], ((it / SR) & 1) ^ 1)) { *abort_flag = 1; ok = false; break; }
         unsigned char *st = ringR + s * P::RB;
         if (lane == 0) {
-          const bool sct = F == Fmt::Affine && a.sc_tma;
+          const bool sct = F == Fmt::Affine && a.sc_tma && affine_box_step(k, k0, a.gs_log2);
           mbar_arrive_expect_tx(&rfull[s], T::RAW + (sct ? 4096 : 0));
           if constexpr (F == Fmt::Gptq) tma_load_2d(st, &tm_w, n0, k * (BK / 8), &rfull[s]);
           else if constexpr (F == Fmt::I8) tma_load_2d(st, &tm_w, k * (BK / 8), n0, &rfull[s]);
@@ -642,35 +651,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kFirstEpi) {
     // ------------------------------------------------------------ dequantizers
+    // Two groups of four warps take alternate K steps, so that two steps are
+    // dequantized at once; a thread writes a whole row of its group's steps
+    // (both halves).  With A in TMEM a warp owns the row quarter its warp index
+    // may address (32 * (warp % 4) ..); each group covers all four quarters.
     if constexpr (F != Fmt::W8) {
     const int d = threadIdx.x - kFirstDq * 32;
-    // tile row and half of the K step; with A in TMEM a warp owns the row
-    // quarter its warp index may address (32 * (warp % 4) ..)
+    const int grp = (warp - kFirstDq) >> 2;
     const int r = ATM ? 32 * (warp & 3) + lane : (d & (kTileN - 1));
-    const int h = ATM ? (warp - kFirstDq) >> 2 : (d >> 7);
+    uint4 sbv[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
     int it = 0, t, k0, k1;
     bool ok = true;
     SegWalk sw(a, nk, unit, units);
     while (ok && sw.next(t, k0, k1)) {
       for (int k = k0; k < k1; k++, it++) {
+        if ((it & 1) != grp) continue;
         const int sr = it % SR, sa = it % SA;
         if (*abort_flag || !mbar_wait(&rfull[sr], (it / SR) & 1) || !mbar_wait(&aempty[sa], ((it / SA) & 1) ^ 1)) {
           *abort_flag = 1;
           ok = false;
           break;
         }
-        {
-          uint32_t o[16];
-          dequant_words<F, BITS>(a, k, r, h, ringR + sr * P::RB, o);
-          if constexpr (ATM) {
-            tmem_st<16>(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + ACOL + (uint32_t)(32 * sa + 16 * h), o);
-            tmem_st_wait();
-            tc_fence_before();
-          } else {
-            store_a_smem(ringA + sa * P::AB, r, h, o);
+        const unsigned char *R = ringR + sr * P::RB;
+        if constexpr (F == Fmt::Affine) {
+          if (a.sc_tma && affine_box_step(k, k0, a.gs_log2)) {
+            // a new block: the row's 8 scales and 8 biases (16 bytes each, conflict-free)
+            const uint4 *box = reinterpret_cast<const uint4 *>(R + T::RAW);
+            sbv[0] = box[a.sc_swap ? kTileN + r : r];
+            sbv[1] = box[a.sc_swap ? r : kTileN + r];
           }
         }
-        if constexpr (!ATM) fence_proxy_async_smem();
+        if constexpr (ATM) {
+          uint32_t o0[16], o1[16];
+          dequant_words<F, BITS>(a, k, r, 0, R, sbv, o0);
+          dequant_words<F, BITS>(a, k, r, 1, R, sbv, o1);
+          const uint32_t col = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + ACOL + (uint32_t)(32 * sa);
+          tmem_st<16>(col, o0);
+          tmem_st<16>(col + 16, o1);
+          tmem_st_wait();
+          tc_fence_before();
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2; h++) {
+            uint32_t o[16];
+            dequant_words<F, BITS>(a, k, r, h, R, sbv, o);
+            store_a_smem(ringA + sa * P::AB, r, h, o);
+          }
+          fence_proxy_async_smem();
+        }
         __syncwarp();
         if (lane == 0) {
           if constexpr (PAIR == 2) mbar_arrive_remote(lead_afull + sa * 8);
@@ -1094,10 +1122,12 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
   int units = kSMs / PAIR;
   if (max_units > 0 && max_units < units) units = max_units;
   const int nk = (a.K + Tr<F, BITS>::BK - 1) / Tr<F, BITS>::BK;
-  // Fewer tiles than units: each tile is split into s equal K parts on s units
-  // (all parts finish together, so no head waits on a longer tail); s = 1 means
-  // whole tiles.  More tiles than units: stream-K over all units when whole tiles
-  // would leave part of the last wave idle and every unit gets a few K steps.
+  // At most half as many tiles as units: each tile is split into s equal K parts
+  // on s units (all parts finish together, so no head waits on a longer tail).
+  // More than half: stream-K over all units (a tile then spans two or three
+  // units), rather than whole tiles on part of the GPU.  More tiles than units:
+  // stream-K over all units when whole tiles would leave part of the last wave
+  // idle.  Stream-K only where every unit gets a few K steps.
   int grid_units = a.T < units ? a.T : units;
   int split_units = units;
   bool want_ws;
@@ -1105,8 +1135,12 @@ gwb_status run_tc2(const void *xptr, CUtensorMapDataType xdt, int xelem, const C
     int s = units / a.T;
     if (s > 8) s = 8;                              // at most 7 partials per finished tile
     while (s > 1 && nk / s < 4) s--;               // and at least 4 K steps per part
-    split_units = a.T * s;
-    want_ws = s > 1;
+    if (s > 1) {
+      split_units = a.T * s;
+      want_ws = true;
+    } else {
+      want_ws = (int64_t)a.T * nk >= 4LL * units;
+    }
   } else {
     want_ws = a.T % units != 0 && (int64_t)a.T * nk >= 4LL * units;
   }

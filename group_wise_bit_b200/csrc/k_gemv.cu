@@ -536,6 +536,10 @@ gwb_status launch_gemv_affine(const uint16_t *x, int M, const uint32_t *wq, cons
 gwb_status launch_gemv_gptq(const uint16_t *x, int M, const int32_t *qweight, const uint16_t *scales,
                             const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
                             uint16_t *y, cudaStream_t st, int zadd) {
+  {   // the shared-memory streamed GEMV where the layout allows
+    const gwb_status s = launch_gemv_gptq_pipe(x, M, qweight, scales, qzeros, g_idx, K, N, gs, y, st, zadd);
+    if (s != GWB_ERR_UNSUPPORTED) return s;
+  }
   const int MP = pad_tokens(M);
 #define GWB_GG(P)                                                                                   \
   if (MP == P) {                                                                                     \

@@ -149,6 +149,16 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
       : "memory");
 }
 
+// Contiguous (untiled) bulk copy of `bytes` from global to this CTA's shared
+// memory, completing that many bytes of transaction count on `bar`.  Both
+// addresses 16-byte aligned, `bytes` a multiple of 16; nothing is zero-filled.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 // TMEM allocation: executed by one full warp; the allocated base address is
 // written to *dst (shared memory).  ncols is a power of two >= 32.

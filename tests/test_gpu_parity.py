@@ -259,6 +259,19 @@ def test_gptq_qmm_small(permuted, M):
     Gptq(384, 264, 128 if M % 2 else 64, permuted, seed=M).check_qmm(M)
 
 
+@pytest.mark.parametrize("permuted", [False, True])
+@pytest.mark.parametrize("K,N,gs", [(256, 32, 32), (768, 96, 64), (1280, 4800, 64), (2048, 9536, 32),
+                                    (1024, 4800, 128)])
+def test_gptq_gemv_streamed_layouts(permuted, K, N, gs):
+    """The shared-memory streamed GEMV (N % 32 == 0, K % 256 == 0): one strip; fewer strips
+    than SMs; more strips than SMs with a remainder (150 and 298 strips on 148 SMs); strips cut
+    between warps at every stage boundary (5 stages a strip); 8, 4 and 2 groups a stage; M from 1
+    to 8 (token padding 1, 2, 4, 8 with ragged M)."""
+    g = Gptq(K, N, gs, permuted, seed=K + N)
+    for M in (1, 2, 3, 5, 8):
+        g.check_qmm(M, seed=M)
+
+
 # --------------------------------------------------------------------------- fused decode products
 def _gate_up_case(N, K, bits, gs, M, seed):
     g = Affine(N, K, bits, gs, seed=seed)
@@ -366,6 +379,13 @@ def test_awq_dequant_bit_exact(gs):
 @pytest.mark.parametrize("M", [1, 4, 8, 32, 150, 300])
 def test_awq_qmm_small(M):
     Awq(384, 264, 128 if M % 2 else 64, seed=M).check_qmm(M)
+
+
+@pytest.mark.parametrize("K,N,gs", [(1280, 4800, 64), (512, 64, 128)])
+def test_awq_gemv_streamed_layouts(K, N, gs):
+    a = Awq(K, N, gs, seed=K + N)
+    for M in (1, 3, 8):
+        a.check_qmm(M, seed=M)
 
 
 def test_awq_equals_gptq_with_stored_zero_minus_one():
