@@ -990,7 +990,8 @@ def run_layer(args):
         nbytes = N * K // 2 + 4 * N + 2 * M * K + 2 * M * N
     else:
         nbytes = int8_bytes(N, K, M, bits) if M <= 64 else None
-    out = {"layer": {"fmt": args.fmt, "N": N, "K": K, "bits": bits, "group_size": GS, "M": M},
+    out = {"layer": {"fmt": args.fmt, "N": N, "K": K, "bits": bits,
+                     "group_size": GPTQ_GS if args.fmt.startswith("gptq") else GS, "M": M},
            "us_per_launch": round(us, 2)}
     if nbytes:
         out["GB/s"] = round(nbytes / us / 1e3, 1)

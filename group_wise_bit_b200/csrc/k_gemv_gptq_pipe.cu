@@ -14,30 +14,46 @@
 // groups.  One CTA of 8 warps per SM takes a contiguous range of strips and
 // cuts its (strip, stage) list into 8 equal contiguous pieces, one per warp.
 // A warp streams its stages through a private ring of D shared-memory slots:
-// each lane issues one bulk copy (one 128-byte run), and two more lanes per
-// group copy the scale and zero runs, all completing on the slot's mbarrier;
-// a slot is refilled as soon as the warp has read it.  A warp holds only a few
+// lane 0 issues three tiled TMA loads per stage (the codes as one box of 32
+// rows x 128 bytes, the scales and the zero words as boxes of the stage's
+// groups), all completing on the slot's mbarrier; a slot is refilled as soon
+// as the warp has read it.  (Copies of single 128-byte runs were bound by the
+// rate of TMA operations, about one per 25 cycles per SM.)  A warp holds only a few
 // stages, so most of a CTA's weights are requested at once, at kernel start.
 //
-// Per 32 in-features of a stage (4 qweight rows), lane (g = lane / 4,
-// c = lane % 4) reads the 16 bytes of row c that hold features 4g .. 4g + 3
-// of the strip.  Each code becomes the fp16 value 1024 + code (one LOP3 per
-// two codes); subtracting 1024 + zero and multiplying by the scale (one half2
-// operation each, one rounding) gives exactly the fp16 weight that
-// gptq_dequant writes.  The weights of features (4g, 4g + 1) and of
-// (4g + 2, 4g + 3) are the A fragments (rows g, g + 8) of two m16n8k16 MMA
-// chains (fp16 in, fp32 accumulate), against activations staged once per CTA
-// as ready-made B fragments (tokens are the MMA's N dimension, padded to 8).
-// The order of in-features inside the 32 is free, so the staged activations
-// follow the order the unpacked registers imply.
+// Per 32 in-features of a stage (4 qweight rows, stored with the 128-byte
+// swizzle), lane (g = lane / 4, c = lane % 4) reads the 16 bytes of row c that
+// hold the strip's features 4G .. 4G + 3 (G = g / 2 + 4 (g % 2): the two quads
+// of a quarter-warp read chunks q and q + 4, conflict-free).  Each code
+// becomes the fp16 value 1024 + code (one LOP3 per two codes).  The codes of
+// features (4G, 4G + 1) and of (4G + 2, 4G + 3) are the A fragments (rows g,
+// g + 8) of two m16n8k16 MMAs (fp16 in, fp32 accumulate) against activations
+// staged once per CTA as ready-made B fragments (tokens are the MMA's N
+// dimension, padded to 8); the order of in-features inside the 32 is free, so
+// the staged activations follow the order the unpacked registers imply.
+//   * Without g_idx the MMAs sum (1024 + q) x over each group, and the group
+//     adds s * (that - (1024 + zero) * sum_k x) to the output (the x sums are
+//     staged with the fragments): the scale and zero cost two FMAs per value
+//     and group, not one operation per weight.
+//   * With g_idx every in-feature has its own group, so the weights are
+//     dequantized before the MMA: (1024 + q) - (1024 + zero), times the scale
+//     (one half2 operation each, one rounding: the fp16 weight gptq_dequant
+//     writes), with the scales and zeros read through the L1 cache.
+// Consecutive units feed four rotating accumulator chains, so that the MMAs of
+// a stage do not wait on one another.
 //
 // A strip whose stages are split between warps is finished through shared
 // memory in warp order, i.e. in K order: results are deterministic.
 #include <cuda_fp16.h>
 
+#include <cudaTypedefs.h>
+
 #include <atomic>
 #include <climits>
 #include <cstdint>
+#include <functional>
+#include <mutex>
+#include <unordered_map>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -45,6 +61,7 @@
 namespace gwb {
 namespace {
 
+constexpr unsigned kFull = 0xffffffffu;
 constexpr int kGW = 8;                               // warps per CTA
 constexpr int kGThreads = kGW * 32;
 constexpr int kStripN = 32;                          // output features per strip
@@ -52,6 +69,8 @@ constexpr int kStageK = 256;                         // in-features per stage
 constexpr int kCodesB = kStripN * 4 * (kStageK / 8); // 4096 bytes of codes per stage
 constexpr int kScaleBoxB = 8 * kStripN * 2;          // up to 8 groups x 32 fp16 scales
 constexpr int kZeroBoxB = 8 * 16;                    // up to 8 groups x 4 zero words
+constexpr int kSlotB = 5120;                         // codes (1024-aligned for the swizzle), scales, zeros
+static_assert(kCodesB + kScaleBoxB + kZeroBoxB <= kSlotB && kSlotB % 1024 == 0, "ring slot layout");
 constexpr int kMaxDynSmem = 232448;
 constexpr int kNumSMs = 148;
 constexpr int kMaxSlots = 8;
@@ -88,18 +107,26 @@ __device__ __forceinline__ uint32_t dq2(uint32_t q2, uint32_t z2, uint32_t s2) {
   return *reinterpret_cast<uint32_t *>(&q);
 }
 
+// Feature chunk of quad g: quads 2q and 2q + 1 take the 4-feature chunks q and
+// q + 4, so that a quarter-warp's eight 16-byte reads (four qweight rows x two
+// chunks) fall in eight different bank groups of the 128-byte-swizzled stage.
+__device__ __forceinline__ int quad_chunk(int g) { return (g >> 1) | ((g & 1) << 2); }
+
 template <int MP, bool GIDX>
-__global__ void __launch_bounds__(kGThreads, 1) k_gemv_gptq_pipe(const GArgs a) {
-  constexpr int SLOT = GIDX ? kCodesB : kCodesB + kScaleBoxB + kZeroBoxB;
-  extern __shared__ __align__(128) unsigned char smem[];
+__global__ void __launch_bounds__(kGThreads, 1)
+    k_gemv_gptq_pipe(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+                     const __grid_constant__ CUtensorMap tm_z, const GArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ int rec[kGW][2];   // strip of each warp's partial slot (first, last segment), or -1
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, c = lane & 3;
+  const int g = lane >> 2, c = lane & 3, G4 = quad_chunk(g);
   const int D = a.D, nks = a.nks, N = a.N;
-  unsigned char *ring = smem + (size_t)warp * D * SLOT;
-  uint2 *XB = reinterpret_cast<uint2 *>(smem + (size_t)kGW * D * SLOT);   // [K/32][2][4][MP]
-  float *PART = reinterpret_cast<float *>(XB + (size_t)(a.K / 32) * 8 * MP);   // [kGW][2][32][MP]
+  unsigned char *ring = smem + (size_t)warp * D * kSlotB;
+  uint2 *XB = reinterpret_cast<uint2 *>(smem + (size_t)kGW * D * kSlotB);      // [K/32][2][4][MP]
+  float *XS = reinterpret_cast<float *>(XB + (size_t)(a.K / 32) * 8 * MP);      // [G][MP] group sums of x
+  float *PART = XS + (GIDX ? 0 : (size_t)a.G * MP);                              // [kGW][2][32][MP]
   uint64_t *full = reinterpret_cast<uint64_t *>(PART + kGW * 2 * 32 * MP) + warp * D;
 
   // this CTA's strips [sb, se) and this warp's stages [u0, u1) of their list
@@ -112,28 +139,32 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemv_gptq_pipe(const GArgs a) 
 
   if (lane < D) mbar_init(&full[lane], 1);
   if (lane < 2) rec[warp][lane] = -1;
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tm_w);
+    if (!GIDX) {
+      tma_prefetch_desc(&tm_s);
+      tma_prefetch_desc(&tm_z);
+    }
+  }
   fence_mbar_init();
   __syncwarp();
 
-  // stage i of this warp into ring slot `slot` (the whole warp takes part)
+  // stage i of this warp into ring slot `slot` (issued by lane 0)
   auto issue = [&](int i, int slot) {
+    if (lane != 0) return;
     const int su = u0 + i;
     const int sq = su / nks;
     const int strip = sb + sq, ks = su - sq * nks;
     const int n0 = strip * kStripN;
-    unsigned char *dst = ring + slot * SLOT;
+    unsigned char *dst = ring + slot * kSlotB;
     uint64_t *bar = &full[slot];
     const int gps = kStageK >> a.gs_log2;             // groups per stage (gs <= 256)
-    if (lane == 0) mbar_arrive_expect_tx(bar, kCodesB + (GIDX ? 0 : gps * (kStripN * 2 + 16)));
-    __syncwarp();
-    bulk_load(dst + lane * 128, a.qw + (size_t)(ks * (kStageK / 8) + lane) * N + n0, 128, bar);
+    mbar_arrive_expect_tx(bar, kCodesB + (GIDX ? 0 : gps * (kStripN * 2 + 16)));
+    tma_load_2d(dst, &tm_w, n0, ks * (kStageK / 8), bar);
     if constexpr (!GIDX) {
       const int g0 = (ks * kStageK) >> a.gs_log2;
-      if (lane < gps)
-        bulk_load(dst + kCodesB + lane * (kStripN * 2), a.scales + (size_t)(g0 + lane) * N + n0, kStripN * 2, bar);
-      else if (lane >= 16 && lane < 16 + gps)
-        bulk_load(dst + kCodesB + kScaleBoxB + (lane - 16) * 16, a.qzeros + (size_t)(g0 + lane - 16) * (N / 8) + n0 / 8,
-                  16, bar);
+      tma_load_2d(dst + kCodesB, &tm_s, n0, g0, bar);
+      tma_load_2d(dst + kCodesB + kScaleBoxB, &tm_z, n0 / 8, g0, bar);
     }
   };
 
@@ -141,24 +172,42 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemv_gptq_pipe(const GArgs a) 
   for (int i = 0; i < pre; i++) issue(i, i);
   int issued = pre;
 
-  // activations as B fragments: XB[u][j][c][t] = pairs (x[k + 2j], x[k + 2j + 4]) and
-  // (x[k + 2j + 1], x[k + 2j + 5]) with k = 32u + 8c, matching the unpacked registers
+  // Activations.  Item e = (token t, chunk q of 8 in-features) loads x[t, 8q .. 8q + 7]
+  // with one 16-byte load and writes the two B fragments of quad lane c = q % 4 of
+  // unit u = q / 4: XB[u][j][c][t] = pairs (x[k + 2j], x[k + 2j + 4]) and
+  // (x[k + 2j + 1], x[k + 2j + 5]), k = 8q, matching the unpacked registers.
+  // Without g_idx the chunk sums (fp32, in order) are added over each group's
+  // chunks, which sit in consecutive lanes, by a fixed shuffle tree: XS[group][t].
   {
-    const int total = (a.K / 32) * 8 * MP;
+    const int kq = a.K / 8;                 // chunks per token, a multiple of 32
+    const int total = kq * MP;
+    const int cpg = 1 << (a.gs_log2 - 3);   // chunks per group: 4, 8 or 16
     for (int e = threadIdx.x; e < total; e += kGThreads) {
-      const int t = e % MP, cc = (e / MP) & 3, j = (e / (4 * MP)) & 1, u = e / (8 * MP);
-      uint32_t b0 = 0u, b1 = 0u;
-      if (t < a.M) {
-        const uint16_t *xr = a.x + (size_t)t * a.K + u * 32 + cc * 8 + 2 * j;
-        b0 = (uint32_t)__ldg(xr) | ((uint32_t)__ldg(xr + 4) << 16);
-        b1 = (uint32_t)__ldg(xr + 1) | ((uint32_t)__ldg(xr + 5) << 16);
+      const int t = e / kq, q = e - t * kq;
+      const int u = q >> 2, cc = q & 3;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (t < a.M) v = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.K + (size_t)q * 8));
+      XB[((u * 2 + 0) * 4 + cc) * MP + t] = make_uint2(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632));
+      XB[((u * 2 + 1) * 4 + cc) * MP + t] = make_uint2(__byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+      if constexpr (!GIDX) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float s = 0.0f;
+#pragma unroll
+        for (int p = 0; p < 4; p++) {
+          s += __half2float(__ushort_as_half((uint16_t)(w[p] & 0xffffu)));
+          s += __half2float(__ushort_as_half((uint16_t)(w[p] >> 16)));
+        }
+        for (int off = 1; off < cpg; off <<= 1) s += __shfl_xor_sync(kFull, s, off);
+        if ((q & (cpg - 1)) == 0) XS[(q >> (a.gs_log2 - 3)) * MP + t] = s;
       }
-      XB[e] = make_uint2(b0, b1);
     }
   }
   __syncthreads();
 
-  float acc[8];   // features 4g, 4g+1 (tokens 2c, 2c+1 each), then 4g+2, 4g+3
+  // Output accumulators (features 4G4, 4G4 + 1 at tokens 2c, 2c + 1, then 4G4 + 2,
+  // 4G4 + 3) and four rotating MMA chains (unit u feeds chain u % 4), so that no
+  // MMA waits for the one before it in the same stage.
+  float yacc[8], pc[4][8];
   int cur = -1, seg_first = 0, seg_last = 0;
   bool first_seg = true;
   // writes the open segment: whole strips straight to y, a partial strip to
@@ -171,7 +220,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemv_gptq_pipe(const GArgs a) 
 #pragma unroll
         for (int h = 0; h < 2; h++) {
           const int t = 2 * c + h;
-          if (t < a.M) a.y[(size_t)t * N + n0 + 4 * g + jn] = __half_as_ushort(__float2half_rn(acc[2 * jn + h]));
+          if (t < a.M) a.y[(size_t)t * N + n0 + 4 * G4 + jn] = __half_as_ushort(__float2half_rn(yacc[2 * jn + h]));
         }
     } else {
       const int sl = first_seg ? 0 : 1;
@@ -181,7 +230,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemv_gptq_pipe(const GArgs a) 
 #pragma unroll
         for (int h = 0; h < 2; h++) {
           const int t = 2 * c + h;
-          if (t < MP) P[(4 * g + jn) * MP + t] = acc[2 * jn + h];
+          if (t < MP) P[(4 * G4 + jn) * MP + t] = yacc[2 * jn + h];
         }
       if (lane == 0) rec[warp][sl] = cur;
     }
@@ -189,6 +238,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemv_gptq_pipe(const GArgs a) 
   };
 
   const bool hasB = g < MP;
+  const int nch = 1 << (a.gs_log2 - 5);   // chains a group uses: gs / 32 units
   int i = 0;
   bool ok = true;
   for (; i < nst; i++) {
@@ -203,37 +253,53 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemv_gptq_pipe(const GArgs a) 
     if (strip != cur) {
       if (cur >= 0) flush();
 #pragma unroll
-      for (int q = 0; q < 8; q++) acc[q] = 0.0f;
+      for (int q = 0; q < 8; q++) yacc[q] = 0.0f;
       cur = strip;
       seg_first = ks;
     }
     seg_last = ks;
-    const unsigned char *S = ring + slot * SLOT;
+#pragma unroll
+    for (int ch = 0; ch < 4; ch++)
+#pragma unroll
+      for (int q = 0; q < 8; q++) pc[ch][q] = 0.0f;
+    const unsigned char *S = ring + slot * kSlotB;
     const uint2 *xb = XB + (size_t)ks * 8 * 8 * MP + c * MP + (hasB ? g : 0);
+    float sf[4], zf[4], X0 = 0.0f, X1 = 0.0f;   // the current group's scales, 1024 + zero, and x sums
 #pragma unroll
     for (int u = 0; u < 8; u++) {
-      const uint4 wv = *reinterpret_cast<const uint4 *>(S + (4 * u + c) * 128 + 16 * g);
+      const int r = 4 * u + c;                  // qweight row of the stage (128-byte swizzle)
+      const uint4 wv = *reinterpret_cast<const uint4 *>(S + r * 128 + ((G4 ^ (r & 7)) << 4));
       const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
-      uint32_t A[4][4];   // [feature 4g + jn][register i: codes (i, i + 4)]
+      uint32_t A[4][4];   // [feature 4G4 + jn][register r: codes (r, r + 4)]
       if constexpr (!GIDX) {
-        const int gl = (32 * u) >> a.gs_log2;       // the stage-local group of these 32 in-features
-        const uint2 s4 = *reinterpret_cast<const uint2 *>(S + kCodesB + gl * (kStripN * 2) + 8 * g);
-        const uint32_t zw = *reinterpret_cast<const uint32_t *>(S + kCodesB + kScaleBoxB + gl * 16 + 4 * (g >> 1));
-        const uint32_t sv[4] = {s4.x & 0xffffu, s4.x >> 16, s4.y & 0xffffu, s4.y >> 16};
+        // y = sum_groups s * (sum_k (1024 + q) x - (1024 + zero) * sum_k x): the MMAs take the
+        // codes as unpacked, the group's scale and zero are applied once per group
+        if (((32 * u) & ((1 << a.gs_log2) - 1)) == 0) {
+          const int gl = (32 * u) >> a.gs_log2;
+          const uint2 s4 = *reinterpret_cast<const uint2 *>(S + kCodesB + gl * (kStripN * 2) + 8 * G4);
+          const uint32_t zw =
+              *reinterpret_cast<const uint32_t *>(S + kCodesB + kScaleBoxB + gl * 16 + 4 * (G4 >> 1)) >> ((G4 & 1) * 16);
+          sf[0] = __half2float(__ushort_as_half((uint16_t)(s4.x & 0xffffu)));
+          sf[1] = __half2float(__ushort_as_half((uint16_t)(s4.x >> 16)));
+          sf[2] = __half2float(__ushort_as_half((uint16_t)(s4.y & 0xffffu)));
+          sf[3] = __half2float(__ushort_as_half((uint16_t)(s4.y >> 16)));
 #pragma unroll
-        for (int jn = 0; jn < 4; jn++) {
-          const uint32_t z = 0x6400u | (((zw >> ((g & 1) * 16 + 4 * jn)) & 0xFu) + (uint32_t)a.zadd);
-          const uint32_t z2 = z | (z << 16), s2 = sv[jn] | (sv[jn] << 16);
-#pragma unroll
-          for (int r = 0; r < 4; r++) A[jn][r] = dq2(((w4[jn] >> (4 * r)) & 0x000F000Fu) | 0x64006400u, z2, s2);
+          for (int jn = 0; jn < 4; jn++) zf[jn] = (float)(1024 + (int)((zw >> (4 * jn)) & 0xFu) + a.zadd);
+          const int gq = ((ks * kStageK) >> a.gs_log2) + gl;
+          X0 = 2 * c < MP ? XS[gq * MP + 2 * c] : 0.0f;
+          X1 = 2 * c + 1 < MP ? XS[gq * MP + 2 * c + 1] : 0.0f;
         }
+#pragma unroll
+        for (int jn = 0; jn < 4; jn++)
+#pragma unroll
+          for (int q = 0; q < 4; q++) A[jn][q] = ((w4[jn] >> (4 * q)) & 0x000F000Fu) | 0x64006400u;
       } else {
         // every in-feature has its own group: the lane's eight in-features k0 .. k0 + 7
         const int k0 = ks * kStageK + 32 * u + 8 * c;
         const int4 ga = __ldg(reinterpret_cast<const int4 *>(a.g_idx + k0));
         const int4 gb = __ldg(reinterpret_cast<const int4 *>(a.g_idx + k0 + 4));
         const int gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-        const int ncol = cur * kStripN + 4 * g;
+        const int ncol = cur * kStripN + 4 * G4;
         uint32_t sv[8][2], zv[8];
 #pragma unroll
         for (int p = 0; p < 8; p++) {
@@ -241,27 +307,54 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemv_gptq_pipe(const GArgs a) 
           const uint2 s = __ldg(reinterpret_cast<const uint2 *>(a.scales + (size_t)gq * N + ncol));
           sv[p][0] = s.x;
           sv[p][1] = s.y;
-          zv[p] = __ldg(a.qzeros + (size_t)gq * (N / 8) + ncol / 8) >> ((g & 1) * 16);
+          zv[p] = __ldg(a.qzeros + (size_t)gq * (N / 8) + ncol / 8) >> ((G4 & 1) * 16);
         }
 #pragma unroll
         for (int jn = 0; jn < 4; jn++)
 #pragma unroll
-          for (int r = 0; r < 4; r++) {
-            // codes r (low half) and r + 4 (high half) of feature 4g + jn
-            const uint32_t slo = (sv[r][jn >> 1] >> ((jn & 1) * 16)) & 0xffffu;
-            const uint32_t shi = (sv[r + 4][jn >> 1] >> ((jn & 1) * 16)) & 0xffffu;
-            const uint32_t zlo = 0x6400u | (((zv[r] >> (4 * jn)) & 0xFu) + (uint32_t)a.zadd);
-            const uint32_t zhi = 0x6400u | (((zv[r + 4] >> (4 * jn)) & 0xFu) + (uint32_t)a.zadd);
-            A[jn][r] = dq2(((w4[jn] >> (4 * r)) & 0x000F000Fu) | 0x64006400u, zlo | (zhi << 16), slo | (shi << 16));
+          for (int q = 0; q < 4; q++) {
+            // codes q (low half) and q + 4 (high half) of feature 4G4 + jn
+            const uint32_t slo = (sv[q][jn >> 1] >> ((jn & 1) * 16)) & 0xffffu;
+            const uint32_t shi = (sv[q + 4][jn >> 1] >> ((jn & 1) * 16)) & 0xffffu;
+            const uint32_t zlo = 0x6400u | (((zv[q] >> (4 * jn)) & 0xFu) + (uint32_t)a.zadd);
+            const uint32_t zhi = 0x6400u | (((zv[q + 4] >> (4 * jn)) & 0xFu) + (uint32_t)a.zadd);
+            A[jn][q] = dq2(((w4[jn] >> (4 * q)) & 0x000F000Fu) | 0x64006400u, zlo | (zhi << 16), slo | (shi << 16));
           }
       }
+      float *chn = pc[u & 3];
 #pragma unroll
       for (int j = 0; j < 2; j++) {
         uint2 b = make_uint2(0u, 0u);
         if (hasB) b = xb[(u * 2 + j) * 4 * MP];
-        mma_f16_16816(acc, A[0][2 * j], A[1][2 * j], A[0][2 * j + 1], A[1][2 * j + 1], b.x, b.y);
-        mma_f16_16816(acc + 4, A[2][2 * j], A[3][2 * j], A[2][2 * j + 1], A[3][2 * j + 1], b.x, b.y);
+        mma_f16_16816(chn, A[0][2 * j], A[1][2 * j], A[0][2 * j + 1], A[1][2 * j + 1], b.x, b.y);
+        mma_f16_16816(chn + 4, A[2][2 * j], A[3][2 * j], A[2][2 * j + 1], A[3][2 * j + 1], b.x, b.y);
       }
+      if constexpr (!GIDX) {
+        if (((32 * (u + 1)) & ((1 << a.gs_log2) - 1)) == 0) {
+          // the group's last unit: its chains (units u - nch + 1 .. u), then scale and zero
+          float P[8];
+#pragma unroll
+          for (int q = 0; q < 8; q++) P[q] = 0.0f;
+#pragma unroll
+          for (int ch = 0; ch < 4; ch++)
+            if (((u - ch) & 3) < nch) {
+#pragma unroll
+              for (int q = 0; q < 8; q++) {
+                P[q] += pc[ch][q];
+                pc[ch][q] = 0.0f;
+              }
+            }
+#pragma unroll
+          for (int jn = 0; jn < 4; jn++) {
+            yacc[2 * jn] = fmaf(sf[jn], fmaf(-zf[jn], X0, P[2 * jn]), yacc[2 * jn]);
+            yacc[2 * jn + 1] = fmaf(sf[jn], fmaf(-zf[jn], X1, P[2 * jn + 1]), yacc[2 * jn + 1]);
+          }
+        }
+      }
+    }
+    if constexpr (GIDX) {
+#pragma unroll
+      for (int q = 0; q < 8; q++) yacc[q] += (pc[0][q] + pc[1][q]) + (pc[2][q] + pc[3][q]);
     }
     __syncwarp();   // every lane has read the slot
     if (issued < nst) {
@@ -297,24 +390,102 @@ __global__ void __launch_bounds__(kGThreads, 1) k_gemv_gptq_pipe(const GArgs a) 
 
 int pad_tokens(int M) { return M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8)); }
 
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// A 2-D row-major view [rows][cols] (cols contiguous) read in boxes of
+// [box_rows][box_cols]; false when the driver refuses it.
+bool map_2d(CUtensorMap *m, CUtensorMapDataType dt, int es, const void *base, uint64_t cols, uint64_t rows,
+            uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_NONE) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * (uint64_t)es};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The three maps of one weight (codes, scales, zero words), cached per
+// (device, tensors, shape, group size): encoding costs host time on every call.
+struct GMaps {
+  CUtensorMap w, s, z;
+};
+struct GKey {
+  int dev, gs;
+  const void *p[3];
+  int64_t N, K;
+  bool operator==(const GKey &o) const {
+    return dev == o.dev && gs == o.gs && N == o.N && K == o.K && p[0] == o.p[0] && p[1] == o.p[1] && p[2] == o.p[2];
+  }
+};
+struct GKeyHash {
+  size_t operator()(const GKey &k) const {
+    size_t h = std::hash<int64_t>()(k.N * 1315423911ll + k.K * 31 + k.gs) ^ (size_t)k.dev;
+    for (const void *q : k.p) h = h * 1099511628211ull ^ std::hash<const void *>()(q);
+    return h;
+  }
+};
+
+gwb_status gptq_maps(const GArgs &a, int gs, GMaps &out) {
+  static std::mutex mu;
+  static std::unordered_map<GKey, GMaps, GKeyHash> cache;
+  if (!encode_fn()) return fail(GWB_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  const GKey key{dev, gs, {a.qw, a.scales, a.qzeros}, a.N, a.K};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      out = it->second;
+      return GWB_OK;
+    }
+  }
+  const uint32_t gps = (uint32_t)(kStageK / gs);
+  GMaps m;
+  if (!map_2d(&m.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.qw, (uint64_t)a.N, (uint64_t)a.K / 8, kStripN, kStageK / 8,
+              CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !map_2d(&m.s, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.scales, (uint64_t)a.N, (uint64_t)a.G, kStripN, gps) ||
+      !map_2d(&m.z, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.qzeros, (uint64_t)a.N / 8, (uint64_t)a.G, kStripN / 8, gps))
+    return GWB_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache.size() >= 4096) cache.clear();   // bounded: a model holds far fewer weights
+  cache.emplace(key, m);
+  out = m;
+  return GWB_OK;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <int MP, bool GIDX>
-gwb_status run_gptq_pipe(const GArgs &a0, int strips, cudaStream_t st) {
-  constexpr int SLOT = GIDX ? kCodesB : kCodesB + kScaleBoxB + kZeroBoxB;
+gwb_status run_gptq_pipe(const GArgs &a0, const GMaps &m, int strips, cudaStream_t st) {
+  constexpr int SLOT = kSlotB;
   GArgs a = a0;
   const int grid = strips < kNumSMs ? strips : kNumSMs;
   a.ns_per = strips / grid;
   a.ns_rem = strips % grid;
-  const size_t xb = (size_t)a.K * 2 * MP, part = (size_t)kGW * 2 * 32 * MP * 4;
+  const size_t xb = (size_t)a.K * 2 * MP + (GIDX ? 0 : (size_t)a.G * MP * 4), part = (size_t)kGW * 2 * 32 * MP * 4;
   const int64_t max_stages = ((int64_t)(a.ns_per + (a.ns_rem ? 1 : 0)) * a.nks + kGW - 1) / kGW;
-  const int64_t room = (int64_t)kMaxDynSmem - 1024 - (int64_t)xb - (int64_t)part;
+  const int64_t room = (int64_t)kMaxDynSmem - 1024 - 1024 - (int64_t)xb - (int64_t)part;
   int64_t D = room / (kGW * (SLOT + 8));
   if (D > max_stages) D = max_stages;
   if (D > kMaxSlots) D = kMaxSlots;
   if (D < 2 && !(D == 1 && max_stages == 1)) return GWB_ERR_UNSUPPORTED;
   a.D = (int)D;
-  const size_t smem = (size_t)kGW * D * SLOT + xb + part + (size_t)kGW * D * 8;
+  const size_t smem = 1024 + (size_t)kGW * D * SLOT + xb + part + (size_t)kGW * D * 8;   // + the alignment
   auto kern = k_gemv_gptq_pipe<MP, GIDX>;
   // the shared-memory allowance is per device: raised once on each to what any
   // plan may take (the block's static shared memory stays within the other 1 KB)
@@ -328,7 +499,7 @@ gwb_status run_gptq_pipe(const GArgs &a0, int strips, cudaStream_t st) {
     if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     allowed.fetch_or(bit);
   }
-  kern<<<grid, kGThreads, smem, st>>>(a);
+  kern<<<grid, kGThreads, smem, st>>>(m.w, m.s, m.z, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail(GWB_ERR_CUDA, "GPTQ GEMV launch: %s", cudaGetErrorString(e));
   return GWB_OK;
@@ -341,7 +512,7 @@ gwb_status launch_gemv_gptq_pipe(const uint16_t *x, int M, const int32_t *qweigh
                                  uint16_t *y, cudaStream_t st, int zadd) {
   // the layout this kernel covers; anything else takes the register-fed GEMV
   if (N % kStripN != 0 || K % kStageK != 0 || (gs != 32 && gs != 64 && gs != 128)) return GWB_ERR_UNSUPPORTED;
-  if (!aligned16(qweight) || !aligned16(scales) || !aligned16(qzeros)) return GWB_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(qzeros)) return GWB_ERR_UNSUPPORTED;
   if (M < 1 || M > 8 || N > INT_MAX || K > INT_MAX) return GWB_ERR_UNSUPPORTED;
   GArgs a{};
   a.x = x;
@@ -359,8 +530,11 @@ gwb_status launch_gemv_gptq_pipe(const uint16_t *x, int M, const int32_t *qweigh
   a.nks = (int)(K / kStageK);
   const int strips = (int)(N / kStripN);
   const int MP = pad_tokens(M);
-#define GWB_GP(P)                                                     \
-  if (MP == P) return g_idx ? run_gptq_pipe<P, true>(a, strips, st) : run_gptq_pipe<P, false>(a, strips, st);
+  GMaps m;
+  const gwb_status ms = gptq_maps(a, gs, m);
+  if (ms != GWB_OK) return ms;
+#define GWB_GP(P)                                                           \
+  if (MP == P) return g_idx ? run_gptq_pipe<P, true>(a, m, strips, st) : run_gptq_pipe<P, false>(a, m, strips, st);
   GWB_GP(1) GWB_GP(2) GWB_GP(4) GWB_GP(8)
 #undef GWB_GP
   return GWB_ERR_UNSUPPORTED;
