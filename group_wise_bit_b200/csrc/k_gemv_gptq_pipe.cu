@@ -71,7 +71,8 @@ constexpr int kScaleBoxB = 8 * kStripN * 2;          // up to 8 groups x 32 fp16
 constexpr int kZeroBoxB = 8 * 16;                    // up to 8 groups x 4 zero words
 constexpr int kSlotB = 5120;                         // codes (1024-aligned for the swizzle), scales, zeros
 static_assert(kCodesB + kScaleBoxB + kZeroBoxB <= kSlotB && kSlotB % 1024 == 0, "ring slot layout");
-constexpr int kMaxDynSmem = 232448;
+constexpr int kMaxDynSmem = 232448;                  // per CTA
+constexpr int kSmemPerSM = 233472;
 constexpr int kNumSMs = 148;
 constexpr int kMaxSlots = 8;
 
@@ -113,7 +114,7 @@ __device__ __forceinline__ uint32_t dq2(uint32_t q2, uint32_t z2, uint32_t s2) {
 __device__ __forceinline__ int quad_chunk(int g) { return (g >> 1) | ((g & 1) << 2); }
 
 template <int MP, bool GIDX>
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __launch_bounds__(kGThreads, 2)
     k_gemv_gptq_pipe(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                      const __grid_constant__ CUtensorMap tm_z, const GArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -474,16 +475,31 @@ template <int MP, bool GIDX>
 gwb_status run_gptq_pipe(const GArgs &a0, const GMaps &m, int strips, cudaStream_t st) {
   constexpr int SLOT = kSlotB;
   GArgs a = a0;
-  const int grid = strips < kNumSMs ? strips : kNumSMs;
-  a.ns_per = strips / grid;
-  a.ns_rem = strips % grid;
   const size_t xb = (size_t)a.K * 2 * MP + (GIDX ? 0 : (size_t)a.G * MP * 4), part = (size_t)kGW * 2 * 32 * MP * 4;
-  const int64_t max_stages = ((int64_t)(a.ns_per + (a.ns_rem ? 1 : 0)) * a.nks + kGW - 1) / kGW;
-  const int64_t room = (int64_t)kMaxDynSmem - 1024 - 1024 - (int64_t)xb - (int64_t)part;
-  int64_t D = room / (kGW * (SLOT + 8));
-  if (D > max_stages) D = max_stages;
-  if (D > kMaxSlots) D = kMaxSlots;
-  if (D < 2 && !(D == 1 && max_stages == 1)) return GWB_ERR_UNSUPPORTED;
+  // Two CTAs per SM where each still gets a ring of two slots per warp (a warp
+  // takes a few thousand cycles per stage, bound by latency: 16 warps per SM
+  // hide twice as much of it as 8), else one CTA per SM with a deeper ring.
+  int grid = 0;
+  int64_t D = 0;
+  for (int per_sm = 2; per_sm >= 1 && grid == 0; per_sm--) {
+    const int cap = kNumSMs * per_sm;
+    const int gr = strips < cap ? strips : cap;
+    const int ns_per = strips / gr, ns_rem = strips % gr;
+    const int64_t max_stages = ((int64_t)(ns_per + (ns_rem ? 1 : 0)) * a.nks + kGW - 1) / kGW;
+    // dynamic shared memory a CTA may take: half an SM less the static part and the
+    // per-CTA reservation, or a whole CTA's maximum
+    const int64_t budget = per_sm == 2 ? kSmemPerSM / 2 - 3 * 1024 : kMaxDynSmem - 1024;
+    int64_t d = (budget - 1024 - (int64_t)xb - (int64_t)part) / (kGW * (SLOT + 8));
+    if (d > max_stages) d = max_stages;
+    if (d > kMaxSlots) d = kMaxSlots;
+    if (d >= 2 || (d == 1 && max_stages == 1)) {
+      grid = gr;
+      D = d;
+      a.ns_per = ns_per;
+      a.ns_rem = ns_rem;
+    }
+  }
+  if (grid == 0) return GWB_ERR_UNSUPPORTED;
   a.D = (int)D;
   const size_t smem = 1024 + (size_t)kGW * D * SLOT + xb + part + (size_t)kGW * D * 8;   // + the alignment
   auto kern = k_gemv_gptq_pipe<MP, GIDX>;
