@@ -113,7 +113,7 @@ __device__ __forceinline__ uint32_t dq2(uint32_t q2, uint32_t z2, uint32_t s2) {
 // chunks) fall in eight different bank groups of the 128-byte-swizzled stage.
 __device__ __forceinline__ int quad_chunk(int g) { return (g >> 1) | ((g & 1) << 2); }
 
-template <int MP, bool GIDX>
+template <int MP, bool GIDX, int GS>
 __global__ void __launch_bounds__(kGThreads, 2)
     k_gemv_gptq_pipe(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                      const __grid_constant__ CUtensorMap tm_z, const GArgs a) {
@@ -159,11 +159,11 @@ __global__ void __launch_bounds__(kGThreads, 2)
     const int n0 = strip * kStripN;
     unsigned char *dst = ring + slot * kSlotB;
     uint64_t *bar = &full[slot];
-    const int gps = kStageK >> a.gs_log2;             // groups per stage (gs <= 256)
+    constexpr int gps = kStageK / GS;                 // groups per stage
     mbar_arrive_expect_tx(bar, kCodesB + (GIDX ? 0 : gps * (kStripN * 2 + 16)));
     tma_load_2d(dst, &tm_w, n0, ks * (kStageK / 8), bar);
     if constexpr (!GIDX) {
-      const int g0 = (ks * kStageK) >> a.gs_log2;
+      const int g0 = ks * gps;
       tma_load_2d(dst + kCodesB, &tm_s, n0, g0, bar);
       tma_load_2d(dst + kCodesB + kScaleBoxB, &tm_z, n0 / 8, g0, bar);
     }
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kGThreads, 2)
   {
     const int kq = a.K / 8;                 // chunks per token, a multiple of 32
     const int total = kq * MP;
-    const int cpg = 1 << (a.gs_log2 - 3);   // chunks per group: 4, 8 or 16
+    constexpr int cpg = GS / 8;             // chunks per group: 4, 8 or 16
     for (int e = threadIdx.x; e < total; e += kGThreads) {
       const int t = e / kq, q = e - t * kq;
       const int u = q >> 2, cc = q & 3;
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kGThreads, 2)
           s += __half2float(__ushort_as_half((uint16_t)(w[p] >> 16)));
         }
         for (int off = 1; off < cpg; off <<= 1) s += __shfl_xor_sync(kFull, s, off);
-        if ((q & (cpg - 1)) == 0) XS[(q >> (a.gs_log2 - 3)) * MP + t] = s;
+        if ((q & (cpg - 1)) == 0) XS[(q / cpg) * MP + t] = s;
       }
     }
   }
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kGThreads, 2)
   // Output accumulators (features 4G4, 4G4 + 1 at tokens 2c, 2c + 1, then 4G4 + 2,
   // 4G4 + 3) and four rotating MMA chains (unit u feeds chain u % 4), so that no
   // MMA waits for the one before it in the same stage.
-  float yacc[8], pc[4][8];
+  float yacc[8], pc[GIDX ? 4 : GS / 32][8];
   int cur = -1, seg_first = 0, seg_last = 0;
   bool first_seg = true;
   // writes the open segment: whole strips straight to y, a partial strip to
@@ -239,7 +239,8 @@ __global__ void __launch_bounds__(kGThreads, 2)
   };
 
   const bool hasB = g < MP;
-  const int nch = 1 << (a.gs_log2 - 5);   // chains a group uses: gs / 32 units
+  constexpr int UPG = GS / 32;                  // units per group (without g_idx): 1, 2 or 4
+  constexpr int NCH = GIDX ? 4 : UPG;           // MMA chains: one per unit of a group
   int i = 0;
   bool ok = true;
   for (; i < nst; i++) {
@@ -260,95 +261,104 @@ __global__ void __launch_bounds__(kGThreads, 2)
     }
     seg_last = ks;
 #pragma unroll
-    for (int ch = 0; ch < 4; ch++)
+    for (int ch = 0; ch < NCH; ch++)
 #pragma unroll
       for (int q = 0; q < 8; q++) pc[ch][q] = 0.0f;
     const unsigned char *S = ring + slot * kSlotB;
     const uint2 *xb = XB + (size_t)ks * 8 * 8 * MP + c * MP + (hasB ? g : 0);
     float sf[4], zf[4], X0 = 0.0f, X1 = 0.0f;   // the current group's scales, 1024 + zero, and x sums
 #pragma unroll
-    for (int u = 0; u < 8; u++) {
-      const int r = 4 * u + c;                  // qweight row of the stage (128-byte swizzle)
-      const uint4 wv = *reinterpret_cast<const uint4 *>(S + r * 128 + ((G4 ^ (r & 7)) << 4));
-      const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
-      uint32_t A[4][4];   // [feature 4G4 + jn][register r: codes (r, r + 4)]
-      if constexpr (!GIDX) {
-        // y = sum_groups s * (sum_k (1024 + q) x - (1024 + zero) * sum_k x): the MMAs take the
-        // codes as unpacked, the group's scale and zero are applied once per group
-        if (((32 * u) & ((1 << a.gs_log2) - 1)) == 0) {
-          const int gl = (32 * u) >> a.gs_log2;
-          const uint2 s4 = *reinterpret_cast<const uint2 *>(S + kCodesB + gl * (kStripN * 2) + 8 * G4);
-          const uint32_t zw =
-              *reinterpret_cast<const uint32_t *>(S + kCodesB + kScaleBoxB + gl * 16 + 4 * (G4 >> 1)) >> ((G4 & 1) * 16);
-          sf[0] = __half2float(__ushort_as_half((uint16_t)(s4.x & 0xffffu)));
-          sf[1] = __half2float(__ushort_as_half((uint16_t)(s4.x >> 16)));
-          sf[2] = __half2float(__ushort_as_half((uint16_t)(s4.y & 0xffffu)));
-          sf[3] = __half2float(__ushort_as_half((uint16_t)(s4.y >> 16)));
+    for (int hh = 0; hh < 2; hh++) {
+      // the half-stage's codes first (four 16-byte reads in flight together)
+      uint4 wv[4];
 #pragma unroll
-          for (int jn = 0; jn < 4; jn++) zf[jn] = (float)(1024 + (int)((zw >> (4 * jn)) & 0xFu) + a.zadd);
-          const int gq = ((ks * kStageK) >> a.gs_log2) + gl;
-          X0 = 2 * c < MP ? XS[gq * MP + 2 * c] : 0.0f;
-          X1 = 2 * c + 1 < MP ? XS[gq * MP + 2 * c + 1] : 0.0f;
-        }
+      for (int q = 0; q < 4; q++) {
+        const int r = 4 * (4 * hh + q) + c;     // qweight row of the stage (128-byte swizzle)
+        wv[q] = *reinterpret_cast<const uint4 *>(S + r * 128 + ((G4 ^ (r & 7)) << 4));
+      }
 #pragma unroll
-        for (int jn = 0; jn < 4; jn++)
+      for (int q = 0; q < 4; q++) {
+        const int u = 4 * hh + q;
+        const uint32_t w4[4] = {wv[q].x, wv[q].y, wv[q].z, wv[q].w};
+        uint32_t A[4][4];   // [feature 4G4 + jn][register p: codes (p, p + 4)]
+        if constexpr (!GIDX) {
+          // y = sum_groups s * (sum_k (1024 + q) x - (1024 + zero) * sum_k x): the MMAs take the
+          // codes as unpacked, the group's scale and zero are applied once per group
+          if (u % UPG == 0) {
+            const int gl = u / UPG;
+            const uint2 s4 = *reinterpret_cast<const uint2 *>(S + kCodesB + gl * (kStripN * 2) + 8 * G4);
+            const uint32_t zw =
+                *reinterpret_cast<const uint32_t *>(S + kCodesB + kScaleBoxB + gl * 16 + 4 * (G4 >> 1)) >>
+                ((G4 & 1) * 16);
+            sf[0] = __half2float(__ushort_as_half((uint16_t)(s4.x & 0xffffu)));
+            sf[1] = __half2float(__ushort_as_half((uint16_t)(s4.x >> 16)));
+            sf[2] = __half2float(__ushort_as_half((uint16_t)(s4.y & 0xffffu)));
+            sf[3] = __half2float(__ushort_as_half((uint16_t)(s4.y >> 16)));
 #pragma unroll
-          for (int q = 0; q < 4; q++) A[jn][q] = ((w4[jn] >> (4 * q)) & 0x000F000Fu) | 0x64006400u;
-      } else {
-        // every in-feature has its own group: the lane's eight in-features k0 .. k0 + 7
-        const int k0 = ks * kStageK + 32 * u + 8 * c;
-        const int4 ga = __ldg(reinterpret_cast<const int4 *>(a.g_idx + k0));
-        const int4 gb = __ldg(reinterpret_cast<const int4 *>(a.g_idx + k0 + 4));
-        const int gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-        const int ncol = cur * kStripN + 4 * G4;
-        uint32_t sv[8][2], zv[8];
-#pragma unroll
-        for (int p = 0; p < 8; p++) {
-          const unsigned gq = (unsigned)gv[p] < (unsigned)a.G ? (unsigned)gv[p] : 0u;
-          const uint2 s = __ldg(reinterpret_cast<const uint2 *>(a.scales + (size_t)gq * N + ncol));
-          sv[p][0] = s.x;
-          sv[p][1] = s.y;
-          zv[p] = __ldg(a.qzeros + (size_t)gq * (N / 8) + ncol / 8) >> ((G4 & 1) * 16);
-        }
-#pragma unroll
-        for (int jn = 0; jn < 4; jn++)
-#pragma unroll
-          for (int q = 0; q < 4; q++) {
-            // codes q (low half) and q + 4 (high half) of feature 4G4 + jn
-            const uint32_t slo = (sv[q][jn >> 1] >> ((jn & 1) * 16)) & 0xffffu;
-            const uint32_t shi = (sv[q + 4][jn >> 1] >> ((jn & 1) * 16)) & 0xffffu;
-            const uint32_t zlo = 0x6400u | (((zv[q] >> (4 * jn)) & 0xFu) + (uint32_t)a.zadd);
-            const uint32_t zhi = 0x6400u | (((zv[q + 4] >> (4 * jn)) & 0xFu) + (uint32_t)a.zadd);
-            A[jn][q] = dq2(((w4[jn] >> (4 * q)) & 0x000F000Fu) | 0x64006400u, zlo | (zhi << 16), slo | (shi << 16));
+            for (int jn = 0; jn < 4; jn++) zf[jn] = (float)(1024 + (int)((zw >> (4 * jn)) & 0xFu) + a.zadd);
+            const int gq = ks * (kStageK / GS) + gl;
+            X0 = 2 * c < MP ? XS[gq * MP + 2 * c] : 0.0f;
+            X1 = 2 * c + 1 < MP ? XS[gq * MP + 2 * c + 1] : 0.0f;
           }
-      }
-      float *chn = pc[u & 3];
 #pragma unroll
-      for (int j = 0; j < 2; j++) {
-        uint2 b = make_uint2(0u, 0u);
-        if (hasB) b = xb[(u * 2 + j) * 4 * MP];
-        mma_f16_16816(chn, A[0][2 * j], A[1][2 * j], A[0][2 * j + 1], A[1][2 * j + 1], b.x, b.y);
-        mma_f16_16816(chn + 4, A[2][2 * j], A[3][2 * j], A[2][2 * j + 1], A[3][2 * j + 1], b.x, b.y);
-      }
-      if constexpr (!GIDX) {
-        if (((32 * (u + 1)) & ((1 << a.gs_log2) - 1)) == 0) {
-          // the group's last unit: its chains (units u - nch + 1 .. u), then scale and zero
-          float P[8];
+          for (int jn = 0; jn < 4; jn++)
 #pragma unroll
-          for (int q = 0; q < 8; q++) P[q] = 0.0f;
+            for (int p = 0; p < 4; p++) A[jn][p] = ((w4[jn] >> (4 * p)) & 0x000F000Fu) | 0x64006400u;
+        } else {
+          // every in-feature has its own group: the lane's eight in-features k0 .. k0 + 7
+          const int k0 = ks * kStageK + 32 * u + 8 * c;
+          const int4 ga = __ldg(reinterpret_cast<const int4 *>(a.g_idx + k0));
+          const int4 gb = __ldg(reinterpret_cast<const int4 *>(a.g_idx + k0 + 4));
+          const int gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+          const int ncol = cur * kStripN + 4 * G4;
+          uint32_t sv[8][2], zv[8];
 #pragma unroll
-          for (int ch = 0; ch < 4; ch++)
-            if (((u - ch) & 3) < nch) {
+          for (int p = 0; p < 8; p++) {
+            const unsigned gq = (unsigned)gv[p] < (unsigned)a.G ? (unsigned)gv[p] : 0u;
+            const uint2 s = __ldg(reinterpret_cast<const uint2 *>(a.scales + (size_t)gq * N + ncol));
+            sv[p][0] = s.x;
+            sv[p][1] = s.y;
+            zv[p] = __ldg(a.qzeros + (size_t)gq * (N / 8) + ncol / 8) >> ((G4 & 1) * 16);
+          }
 #pragma unroll
-              for (int q = 0; q < 8; q++) {
-                P[q] += pc[ch][q];
-                pc[ch][q] = 0.0f;
+          for (int jn = 0; jn < 4; jn++)
+#pragma unroll
+            for (int p = 0; p < 4; p++) {
+              // codes p (low half) and p + 4 (high half) of feature 4G4 + jn
+              const uint32_t slo = (sv[p][jn >> 1] >> ((jn & 1) * 16)) & 0xffffu;
+              const uint32_t shi = (sv[p + 4][jn >> 1] >> ((jn & 1) * 16)) & 0xffffu;
+              const uint32_t zlo = 0x6400u | (((zv[p] >> (4 * jn)) & 0xFu) + (uint32_t)a.zadd);
+              const uint32_t zhi = 0x6400u | (((zv[p + 4] >> (4 * jn)) & 0xFu) + (uint32_t)a.zadd);
+              A[jn][p] = dq2(((w4[jn] >> (4 * p)) & 0x000F000Fu) | 0x64006400u, zlo | (zhi << 16), slo | (shi << 16));
+            }
+        }
+        float *chn = pc[u % NCH];
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+          uint2 b = make_uint2(0u, 0u);
+          if (hasB) b = xb[(u * 2 + j) * 4 * MP];
+          mma_f16_16816(chn, A[0][2 * j], A[1][2 * j], A[0][2 * j + 1], A[1][2 * j + 1], b.x, b.y);
+          mma_f16_16816(chn + 4, A[2][2 * j], A[3][2 * j], A[2][2 * j + 1], A[3][2 * j + 1], b.x, b.y);
+        }
+        if constexpr (!GIDX) {
+          if (u % UPG == UPG - 1) {
+            // the group's last unit: its chains, then the scale and zero
+            float P[8];
+#pragma unroll
+            for (int q2 = 0; q2 < 8; q2++) {
+              float v = 0.0f;
+#pragma unroll
+              for (int ch = 0; ch < NCH; ch++) {
+                v += pc[ch][q2];
+                pc[ch][q2] = 0.0f;
               }
+              P[q2] = v;
             }
 #pragma unroll
-          for (int jn = 0; jn < 4; jn++) {
-            yacc[2 * jn] = fmaf(sf[jn], fmaf(-zf[jn], X0, P[2 * jn]), yacc[2 * jn]);
-            yacc[2 * jn + 1] = fmaf(sf[jn], fmaf(-zf[jn], X1, P[2 * jn + 1]), yacc[2 * jn + 1]);
+            for (int jn = 0; jn < 4; jn++) {
+              yacc[2 * jn] = fmaf(sf[jn], fmaf(-zf[jn], X0, P[2 * jn]), yacc[2 * jn]);
+              yacc[2 * jn + 1] = fmaf(sf[jn], fmaf(-zf[jn], X1, P[2 * jn + 1]), yacc[2 * jn + 1]);
+            }
           }
         }
       }
@@ -471,7 +481,7 @@ gwb_status gptq_maps(const GArgs &a, int gs, GMaps &out) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int MP, bool GIDX>
+template <int MP, bool GIDX, int GS>
 gwb_status run_gptq_pipe(const GArgs &a0, const GMaps &m, int strips, cudaStream_t st) {
   constexpr int SLOT = kSlotB;
   GArgs a = a0;
@@ -502,7 +512,7 @@ gwb_status run_gptq_pipe(const GArgs &a0, const GMaps &m, int strips, cudaStream
   if (grid == 0) return GWB_ERR_UNSUPPORTED;
   a.D = (int)D;
   const size_t smem = 1024 + (size_t)kGW * D * SLOT + xb + part + (size_t)kGW * D * 8;   // + the alignment
-  auto kern = k_gemv_gptq_pipe<MP, GIDX>;
+  auto kern = k_gemv_gptq_pipe<MP, GIDX, GS>;
   // the shared-memory allowance is per device: raised once on each to what any
   // plan may take (the block's static shared memory stays within the other 1 KB)
   static std::atomic<uint64_t> allowed{0};
@@ -549,8 +559,14 @@ gwb_status launch_gemv_gptq_pipe(const uint16_t *x, int M, const int32_t *qweigh
   GMaps m;
   const gwb_status ms = gptq_maps(a, gs, m);
   if (ms != GWB_OK) return ms;
-#define GWB_GP(P)                                                           \
-  if (MP == P) return g_idx ? run_gptq_pipe<P, true>(a, m, strips, st) : run_gptq_pipe<P, false>(a, m, strips, st);
+  // act order: one kernel for every group size (its groups are per in-feature)
+#define GWB_GP(P)                                                                           \
+  if (MP == P) {                                                                             \
+    if (g_idx) return run_gptq_pipe<P, true, 128>(a, m, strips, st);                         \
+    if (gs == 32) return run_gptq_pipe<P, false, 32>(a, m, strips, st);                      \
+    if (gs == 64) return run_gptq_pipe<P, false, 64>(a, m, strips, st);                      \
+    return run_gptq_pipe<P, false, 128>(a, m, strips, st);                                   \
+  }
   GWB_GP(1) GWB_GP(2) GWB_GP(4) GWB_GP(8)
 #undef GWB_GP
   return GWB_ERR_UNSUPPORTED;
