@@ -341,7 +341,10 @@ def gptq_work(gwb, dev, M, permuted, dequant=False):
     def check():
         return ("gptq", dict(x=x, h=(qw, sc, qz, gi if permuted else None), y=y.cpu(), K=K, N=N, gs=gs, M=M))
 
-    kern = "k_gemv_gptq" if M <= 8 else ("k_tc2<Gptq>" if M > 128 and not permuted else "k_tc<Gptq>")
+    if M <= 8:
+        kern = "k_gemv_gptq_pipe" if N % 32 == 0 and K % 256 == 0 else "k_gemv_gptq"
+    else:
+        kern = "k_tc<Gptq>" if permuted else "k_tc2<Gptq>"
     return Work(f"gptq M={M} perm={int(permuted)}", launch, len(cps), gptq_bytes(K, N, gs, M, permuted),
                 2.0 * M * N * K, kern, [check])
 
@@ -719,7 +722,7 @@ def run_gpu(args, world, rank, local):
                                          key, tm[1:], bf16_peak, bf16_src, "TFLOP/s", "tensor")})
             else:
                 out[key] = aggregate(key, tm[:1], hbm_peak, hbm_src, "GB/s", "hbm",
-                                     traffic_key="k_gemv_gptq_m1" if M == 1 else None,
+                                     traffic_key="k_gemv_gptq_pipe_m1" if M == 1 else None,
                                      extra={"permuted_g_idx": aggregate(key, tm[1:], hbm_peak, hbm_src, "GB/s", "hbm")})
         for fmt in ("w4a8", "w8a8"):
             for M in INT8_M:
