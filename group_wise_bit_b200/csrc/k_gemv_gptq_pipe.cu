@@ -169,8 +169,10 @@ __global__ void __launch_bounds__(kGThreads, 2)
     }
   };
 
+  // the first stage is requested before the activations are staged, the rest of
+  // the ring after (the staging's loads are not held up by the copies' issue)
   const int pre = nst < D ? nst : D;
-  for (int i = 0; i < pre; i++) issue(i, i);
+  if (pre > 0) issue(0, 0);
   int issued = pre;
 
   // Activations.  Item e = (token t, chunk q of 8 in-features) loads x[t, 8q .. 8q + 7]
@@ -179,30 +181,46 @@ __global__ void __launch_bounds__(kGThreads, 2)
   // (x[k + 2j + 1], x[k + 2j + 5]), k = 8q, matching the unpacked registers.
   // Without g_idx the chunk sums (fp32, in order) are added over each group's
   // chunks, which sit in consecutive lanes, by a fixed shuffle tree: XS[group][t].
+  // Two items per round, both loaded before either is used.
   {
     const int kq = a.K / 8;                 // chunks per token, a multiple of 32
     const int total = kq * MP;
     constexpr int cpg = GS / 8;             // chunks per group: 4, 8 or 16
-    for (int e = threadIdx.x; e < total; e += kGThreads) {
-      const int t = e / kq, q = e - t * kq;
-      const int u = q >> 2, cc = q & 3;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (t < a.M) v = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.K + (size_t)q * 8));
-      XB[((u * 2 + 0) * 4 + cc) * MP + t] = make_uint2(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632));
-      XB[((u * 2 + 1) * 4 + cc) * MP + t] = make_uint2(__byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
-      if constexpr (!GIDX) {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float s = 0.0f;
+    for (int e0 = threadIdx.x; e0 < total; e0 += 2 * kGThreads) {
+      uint4 v[2];
 #pragma unroll
-        for (int p = 0; p < 4; p++) {
-          s += __half2float(__ushort_as_half((uint16_t)(w[p] & 0xffffu)));
-          s += __half2float(__ushort_as_half((uint16_t)(w[p] >> 16)));
+      for (int h = 0; h < 2; h++) {
+        const int e = e0 + h * kGThreads;
+        const int t = e / kq, q = e - t * kq;
+        v[h] = make_uint4(0u, 0u, 0u, 0u);
+        if (e < total && t < a.M) v[h] = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.K + (size_t)q * 8));
+      }
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int e = e0 + h * kGThreads;
+        if (e >= total) break;                // the same for the whole warp (total is a multiple of 32)
+        const int t = e / kq, q = e - t * kq;
+        const int u = q >> 2, cc = q & 3;
+        XB[((u * 2 + 0) * 4 + cc) * MP + t] =
+            make_uint2(__byte_perm(v[h].x, v[h].z, 0x5410), __byte_perm(v[h].x, v[h].z, 0x7632));
+        XB[((u * 2 + 1) * 4 + cc) * MP + t] =
+            make_uint2(__byte_perm(v[h].y, v[h].w, 0x5410), __byte_perm(v[h].y, v[h].w, 0x7632));
+        if constexpr (!GIDX) {
+          const uint32_t w[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+          float s = 0.0f;
+#pragma unroll
+          for (int p = 0; p < 4; p++) {
+            s += __half2float(__ushort_as_half((uint16_t)(w[p] & 0xffffu)));
+            s += __half2float(__ushort_as_half((uint16_t)(w[p] >> 16)));
+          }
+#pragma unroll
+          for (int off = 1; off < cpg; off <<= 1) s += __shfl_xor_sync(kFull, s, off);
+          if ((q & (cpg - 1)) == 0) XS[(q / cpg) * MP + t] = s;
         }
-        for (int off = 1; off < cpg; off <<= 1) s += __shfl_xor_sync(kFull, s, off);
-        if ((q & (cpg - 1)) == 0) XS[(q / cpg) * MP + t] = s;
       }
     }
   }
+  for (int i = 1; i < pre; i++) issue(i, i);
   __syncthreads();
 
   // Output accumulators (features 4G4, 4G4 + 1 at tokens 2c, 2c + 1, then 4G4 + 2,
@@ -271,10 +289,16 @@ __global__ void __launch_bounds__(kGThreads, 2)
     for (int hh = 0; hh < 2; hh++) {
       // the half-stage's codes first (four 16-byte reads in flight together)
       uint4 wv[4];
+      uint2 bv[4][2];   // and the half-stage's activation fragments
 #pragma unroll
       for (int q = 0; q < 4; q++) {
         const int r = 4 * (4 * hh + q) + c;     // qweight row of the stage (128-byte swizzle)
         wv[q] = *reinterpret_cast<const uint4 *>(S + r * 128 + ((G4 ^ (r & 7)) << 4));
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+          bv[q][j] = make_uint2(0u, 0u);
+          if (hasB) bv[q][j] = xb[((4 * hh + q) * 2 + j) * 4 * MP];
+        }
       }
 #pragma unroll
       for (int q = 0; q < 4; q++) {
@@ -335,8 +359,7 @@ __global__ void __launch_bounds__(kGThreads, 2)
         float *chn = pc[u % NCH];
 #pragma unroll
         for (int j = 0; j < 2; j++) {
-          uint2 b = make_uint2(0u, 0u);
-          if (hasB) b = xb[(u * 2 + j) * 4 * MP];
+          const uint2 b = bv[q][j];
           mma_f16_16816(chn, A[0][2 * j], A[1][2 * j], A[0][2 * j + 1], A[1][2 * j + 1], b.x, b.y);
           mma_f16_16816(chn + 4, A[2][2 * j], A[3][2 * j], A[2][2 * j + 1], A[3][2 * j + 1], b.x, b.y);
         }
