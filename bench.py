@@ -344,7 +344,7 @@ def gptq_work(gwb, dev, M, permuted, dequant=False):
     if M <= 8:
         kern = "k_gemv_gptq_pipe" if N % 32 == 0 and K % 256 == 0 else "k_gemv_gptq"
     else:
-        kern = "k_tc<Gptq>" if permuted else "k_tc2<Gptq>"
+        kern = "k_gptq_dequant + k_tc2<F16>" if permuted else "k_tc2<Gptq>"
     return Work(f"gptq M={M} perm={int(permuted)}", launch, len(cps), gptq_bytes(K, N, gs, M, permuted),
                 2.0 * M * N * K, kern, [check])
 

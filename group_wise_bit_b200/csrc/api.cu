@@ -289,10 +289,22 @@ gwb_status gptq_qmm_impl(const uint16_t *x, int64_t M, const int32_t *qweight, c
   if (M <= 8)
     return gwb::launch_gemv_gptq(x, (int)M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream),
                                  zadd);
-  {   // the persistent stream-K GEMM without g_idx; the per-tile kernel with it
+  {   // the persistent stream-K GEMM without g_idx
     const gwb_status s =
         gwb::launch_tc2_gptq(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream), zadd);
     if (s != GWB_ERR_UNSUPPORTED) return s;
+  }
+  if (g_idx) {
+    // act order: every in-feature has its own group, so the weights are dequantized
+    // once (exactly as gwb_gptq_dequant writes them) into the library's scratch and
+    // multiplied as dense fp16 on the persistent GEMM
+    uint16_t *wd = nullptr;
+    if (aligned16(x) && gwb::dequant_scratch(as_stream(stream), (size_t)N * (size_t)K * 2, &wd)) {
+      gwb::launch_gptq_dequant(qweight, scales, qzeros, g_idx, K, N, group_size, wd, as_stream(stream), zadd);
+      GWB_TRY(gwb::check_launch("gptq_dequant"));
+      const gwb_status s = gwb::launch_tc2_f16(x, M, wd, N, K, y, as_stream(stream));
+      if (s != GWB_ERR_UNSUPPORTED) return s;
+    }
   }
   return gwb::launch_tc_gptq(x, M, qweight, scales, qzeros, g_idx, K, N, group_size, y, as_stream(stream), zadd);
 }

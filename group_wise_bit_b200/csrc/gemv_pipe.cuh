@@ -583,6 +583,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // split-bf16 B operand of the bias MMAs (XF).
     {
       if (OP == kOpW4A8 && threadIdx.x < MP) tok_sx[threadIdx.x] = __fdiv_rn(token_amax(threadIdx.x), 127.0f);
+      if constexpr (OP == kOpW4A8) __syncthreads();   // every item reads its token's scale
       const int total = items;
       for (int b0 = 0; b0 < total; b0 += PB * kThreads) {
       Item itb[PB];
@@ -605,8 +606,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int t = tq[u], c = cq[u], g = gq[u];
         const bool live = sq[u] >= 0;
         const float sc = pow2f(live ? token_exp(t) : 0);
-        // w4a8: the token's int8 scale, max|x| / 127 over the whole row (K is not split)
-        [[maybe_unused]] const float sq = OP == kOpW4A8 ? __fdiv_rn(token_amax(t), 127.0f) : 0.0f;
+        // w4a8: the token's int8 scale, max|x| / 127 over the whole row (over every CTA's
+        // K-slice when a cluster splits K)
+        [[maybe_unused]] const float sq = OP == kOpW4A8 ? tok_sx[t] : 0.0f;
         const Item &rawb = itb[u];
         float sx = 0.0f, sn = 0.0f;
         uint32_t pr[C::NREG];

@@ -100,6 +100,14 @@ gwb_status launch_tc2_i8i8(const int8_t *qx, const float *sx, int64_t M, const i
                            int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 gwb_status launch_tc2_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
                            int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
+// Dense fp16 weights [N, K] on the persistent GEMM (fp16 in and out);
+// GWB_ERR_UNSUPPORTED (without a message) for K % 8 != 0 or unaligned operands.
+gwb_status launch_tc2_f16(const uint16_t *x, int64_t M, const uint16_t *w, int64_t N, int64_t K, uint16_t *y,
+                          cudaStream_t st);
+// The library's scratch for dequantized weights on this stream, at least
+// `bytes` long; false when it cannot be had (allocation under stream capture,
+// or out of memory).
+bool dequant_scratch(cudaStream_t st, size_t bytes, uint16_t **out);
 // The persistent GEMM with its stream-K scratch in a fixed device array (no
 // allocation); M must exceed 128.
 gwb_status launch_tc2_affine_noalloc(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,

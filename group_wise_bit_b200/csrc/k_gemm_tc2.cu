@@ -176,7 +176,7 @@ constexpr bool kAInTmem = true;   // pairs keep the dequantized A operand in ten
 // Affine / Gptq: 16-bit activations x dequantized weights; I8: int8
 // activations x int4 codes; W8: int8 activations x int8 weights, which need no
 // dequantization and go by TMA straight into the A stages.
-enum class Fmt { Affine, Gptq, I8, W8 };
+enum class Fmt { Affine, Gptq, I8, W8, F16 };
 
 struct Args {
   int M, N, K, gs;
@@ -264,6 +264,14 @@ struct Tr<Fmt::W8, 8> {
   static constexpr int CP = 0;
 };
 template <>
+struct Tr<Fmt::F16, 16> {                             // dense fp16 weights (act-order GPTQ, dequantized first)
+  static constexpr int BK = 64;
+  static constexpr int RAW = 0;
+  static constexpr int SC = 0;
+  static constexpr int NMMA = BK / 16;
+  static constexpr int CP = 0;
+};
+template <>
 struct Tr<Fmt::I8, 4> {
   static constexpr int BK = 128;                      // 128 int8 = 128 bytes per row
   static constexpr int RAW = kTileN * BK / 2;
@@ -278,11 +286,11 @@ struct Tr<Fmt::I8, 4> {
 // activation slots as it can.  The packed-weight ring takes what is left, up to 8.
 // With ATM the dequantized A stages live in tensor memory (8 slots of 32
 // columns next to one 256-column accumulator) and take no shared memory.
-// W8 has no packed-weight ring: activation and weight stages go in lockstep,
-// as many of each as fit (up to 8).
+// W8 and F16 (weights that need no dequantization) have no packed-weight ring:
+// activation and weight stages go in lockstep, as many of each as fit (up to 8).
 template <Fmt F, int BITS, int BT, int PAIR, bool ATM>
 struct Plan2 {
-  static constexpr bool W8 = F == Fmt::W8;
+  static constexpr bool W8 = F == Fmt::W8 || F == Fmt::F16;   // the weight tile goes straight to the A stage
   static constexpr int XB = BT / PAIR * 128;
   static constexpr int AB = kTileN * 128;
   static constexpr int RB = (Tr<F, BITS>::RAW + Tr<F, BITS>::SC + 127) / 128 * 128;
@@ -302,7 +310,7 @@ struct Plan2 {
   static constexpr int SR = W8 ? 0 : SR0 > 8 ? 8 : SR0;
   static constexpr int SMEM = SX * XB + A_SMEM + EPI + SR * RB + 1024 + 1024;
   static_assert(SX >= 2 && (W8 || SR >= 4), "shared memory too small");
-  static_assert(!(W8 && ATM), "int8 weights are read from shared memory");
+  static_assert(!(W8 && ATM), "dense weights are read from shared memory");
 };
 
 __device__ __forceinline__ void put4(uint32_t (&o)[16], int j, uint4 v) {
@@ -421,8 +429,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t ACOL = BT;                        // first A slot column (ATM)
   static_assert(!ATM || (PAIR == 2 && BT == 256), "A in tensor memory is laid out for 256-token pairs");
   constexpr bool kInt = F == Fmt::I8 || F == Fmt::W8;   // kind::i8, s32 accumulators
+  constexpr bool kDense = F == Fmt::W8 || F == Fmt::F16;   // weights by TMA straight into the A stage
+  constexpr bool kOutF16 = F == Fmt::Gptq || F == Fmt::F16;
   constexpr uint32_t IDESC = kInt ? make_idesc(2, 1, kTileN * PAIR, BT)
-                             : (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN * PAIR, BT)
+                             : kOutF16 ? make_idesc(1, 0, kTileN * PAIR, BT)
                                                 : make_idesc(1, 1, kTileN * PAIR, BT);
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -452,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; s++) { mbar_init(&xfull[s], 1); mbar_init(&xempty[s], 1); }
-    for (int s = 0; s < SA; s++) { mbar_init(&afull[s], F == Fmt::W8 ? 1 : kDqGroupWarps * PAIR); mbar_init(&aempty[s], 1); }
+    for (int s = 0; s < SA; s++) { mbar_init(&afull[s], kDense ? 1 : kDqGroupWarps * PAIR); mbar_init(&aempty[s], 1); }
     for (int s = 0; s < SR; s++) {
       mbar_init(&rfull[s], 1 + (F == Fmt::Affine && a.sc_tma ? 0 : T::CP));
       mbar_init(&rempty[s], kDqGroupWarps);
@@ -512,10 +522,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = it - SX < 0 ? 0 : it - SX; i < it; i++) mbar_wait(&xfull[i % SX], (i / SX) & 1);
     }
   } else if (warp == 2) {
-    if constexpr (F == Fmt::W8) {
-    // ------------------------------------------------------------ A producer (int8 weights)
-    // The weight tile [128 rows][128 k] lands in the A stage by one swizzled
-    // TMA copy; with a pair, both CTAs' copies complete on the leader's barrier.
+    if constexpr (kDense) {
+    // ------------------------------------------------------------ A producer (dense weights)
+    // The weight tile [128 rows][128 bytes of k] lands in the A stage by one
+    // swizzled TMA copy; with a pair, both CTAs' copies complete on the leader's barrier.
     if (lane == 0) {
       int it = 0, t, k0, k1;
       bool ok = true;
@@ -655,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dequantized at once; a thread writes a whole row of its group's steps
     // (both halves).  With A in TMEM a warp owns the row quarter its warp index
     // may address (32 * (warp % 4) ..); each group covers all four quarters.
-    if constexpr (F != Fmt::W8) {
+    if constexpr (!kDense) {
     const int d = threadIdx.x - kFirstDq * 32;
     const int grp = (warp - kFirstDq) >> 2;
     const int r = ATM ? 32 * (warp & 3) + lane : (d & (kTileN - 1));
@@ -772,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               } else {
                 f = __uint_as_float(u);
               }
-              stage[(ch * 16 + j) * kTileN + lrow] = F == Fmt::Gptq ? __half_as_ushort(__float2half_rn(f))
+              stage[(ch * 16 + j) * kTileN + lrow] = kOutF16 ? __half_as_ushort(__float2half_rn(f))
                                                                     : __bfloat16_as_ushort(__float2bfloat16_rn(f));
             }
           }
@@ -889,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                   f = __uint_as_float(u) + __uint_as_float(p);
                 }
-                po[j * kTileN + lrow] = F == Fmt::Gptq ? __half_as_ushort(__float2half_rn(f))
+                po[j * kTileN + lrow] = kOutF16 ? __half_as_ushort(__float2half_rn(f))
                                                        : __bfloat16_as_ushort(__float2bfloat16_rn(f));
               }
               named_bar_sync(1, 128);
@@ -979,7 +989,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int acc = F == Fmt::I8 ? static_cast<int>(v[j]) >> 4 : static_cast<int>(v[j]);
                 if (a.acc) a.acc[o] = acc;
                 if (a.y) a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn((float)acc * (sxv[j] * swn)));
-              } else if constexpr (F == Fmt::Gptq) {
+              } else if constexpr (kOutF16) {
                 a.y[o] = __half_as_ushort(__float2half_rn(__uint_as_float(v[j])));
               } else {
                 a.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
@@ -1361,6 +1371,58 @@ gwb_status launch_tc2_i8i8(const int8_t *qx, const float *sx, int64_t M, const i
   if (M <= 32) return run_tc2<Fmt::W8, 8, 32, 1, false>(qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
   if (M <= 128) return run_tc2<Fmt::W8, 8, 128, 1, false>(qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
   return run_tc2<Fmt::W8, 8, 256, 2, false>(qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, tw, a, st);
+}
+
+// Dense fp16 weights [N, K] (act-order GPTQ after its dequantization): the weight
+// tile goes by one swizzled TMA copy into the A stage, fp16 operands, fp16 output.
+gwb_status launch_tc2_f16(const uint16_t *x, int64_t M, const uint16_t *w, int64_t N, int64_t K, uint16_t *y,
+                          cudaStream_t st) {
+  if (K % 8 != 0 || (reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(w) & 15))
+    return GWB_ERR_UNSUPPORTED;
+  Args a{};
+  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = 0;
+  a.y = y;
+  CUtensorMap tw;
+  gwb_status s = map2d(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, 64u,
+                       (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != GWB_OK) return s;
+  if (M <= 32) return run_tc2<Fmt::F16, 16, 32, 1, false>(x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, tw, tw, a, st);
+  if (M <= 64) return run_tc2<Fmt::F16, 16, 64, 1, false>(x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, tw, tw, a, st);
+  if (M <= 128) return run_tc2<Fmt::F16, 16, 128, 1, false>(x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, tw, tw, a, st);
+  return run_tc2<Fmt::F16, 16, 256, 2, false>(x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, tw, tw, a, st);
+}
+
+// Scratch for dequantized weights, owned by the library like the stream-K
+// workspace: one per (device, stream), grown on demand outside stream capture
+// and kept until exit.  False when it would have to be allocated under capture
+// (or the allocation fails); the caller then takes a path without it.
+namespace {
+std::mutex g_dq_mu;
+std::map<std::pair<int, cudaStream_t>, std::pair<void *, size_t>> g_dq;
+}  // namespace
+
+bool dequant_scratch(cudaStream_t st, size_t bytes, uint16_t **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lk(g_dq_mu);
+  auto &e = g_dq[std::make_pair(dev, st)];
+  if (e.first == nullptr || e.second < bytes) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return false;
+    if (e.first) {
+      if (cudaStreamSynchronize(st) != cudaSuccess) return false;
+      cudaFree(e.first);
+      e = {nullptr, 0};
+    }
+    void *p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return false;
+    }
+    e = {p, bytes};
+  }
+  *out = static_cast<uint16_t *>(e.first);
+  return true;
 }
 
 }  // namespace gwb

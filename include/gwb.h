@@ -198,7 +198,11 @@ gwb_status gwb_gptq_dequant(const int32_t *qweight, const uint16_t *scales, cons
 /* gptq_qmm -- y[m,o] = sum_i x[m,i] * W[o,i] with W as gwb_gptq_dequant defines
  * it (each weight rounded to fp16, as the dequantized checkpoint would hold it),
  * fp32 accumulation, fp16 result.
- *   x  fp16 [M, K],  y  fp16 [M, N].   Limits as gwb_gptq_dequant; M >= 1. */
+ *   x  fp16 [M, K],  y  fp16 [M, N].   Limits as gwb_gptq_dequant; M >= 1.
+ * With g_idx and M > 8 the weights are first dequantized into a scratch buffer
+ * owned by the library (2*N*K bytes, one per device and stream, grown to the
+ * largest layer seen and kept until exit; a call under stream capture never
+ * allocates it and then runs a slower kernel without it). */
 gwb_status gwb_gptq_qmm(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
                         const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N,
                         int group_size, uint16_t *y, void *stream);
