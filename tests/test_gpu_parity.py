@@ -580,6 +580,36 @@ def test_stream_k_gemm_replayed_in_a_cuda_graph_with_new_inputs():
     gwb.check_device_error()
 
 
+def test_gptq_act_order_captured_with_and_without_the_scratch():
+    """Act-order GPTQ at M > 8 in a CUDA graph.  A stream that has no dequant scratch yet
+    cannot allocate one under capture, so the captured call takes the per-tile kernel; once an
+    eager call on the stream has made the scratch, a captured call dequantizes into it and
+    runs the dense fp16 GEMM.  Both replays match the oracle."""
+    K, N, gs, M = 512, 264, 128, 40
+    g = Gptq(K, N, gs, True, seed=21)
+    x = synth.activations(M, K, seed=22, dtype=torch.float16)
+    ref = oracle.gptq_qmm(synth.bits16(x), *g.h, K, N, gs)
+    max_w = float(np.abs(oracle.gptq_dequant_f16(*g.h, K, N, gs).view(np.float16).astype(np.float32)).max())
+    xd = x.to(DEV)
+    st = torch.cuda.Stream()
+    y = torch.empty((M, N), dtype=torch.float16, device=DEV)
+    with torch.cuda.stream(st):
+        for eager_first in (False, True):
+            if eager_first:
+                gwb.gptq_qmm(xd, *g.d, gs, y=y)           # the stream's scratch exists from here on
+                st.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=st):
+                gwb.gptq_qmm(xd, *g.d, gs, y=y)
+            y.fill_(float("nan"))
+            graph.replay()
+            st.synchronize()
+            check_float(y.float().cpu().numpy(), ref, K, max_w, float(x.float().abs().max()),
+                        f"act order captured, scratch={'yes' if eager_first else 'no'}")
+            del graph
+    gwb.check_device_error()
+
+
 # --------------------------------------------------------------------------- full sizes
 def test_full_single_affine_linear_512():
     a = Affine(512, 512, 4, 64)
