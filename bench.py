@@ -349,6 +349,11 @@ def gptq_work(gwb, dev, M, permuted, dequant=False):
                 2.0 * M * N * K, kern, [check])
 
 
+def tc2_tile(M):
+    """The persistent GEMM's token tile for M tokens (single CTAs up to 128, CTA pairs above)."""
+    return "32" if M <= 32 else "64" if M <= 64 else "128" if M <= 128 else "256,pair"
+
+
 def int8_work(gwb, dev, fmt, shapes, M):
     works = []
     for j, (N, K) in enumerate(shapes):
@@ -372,9 +377,10 @@ def int8_work(gwb, dev, fmt, shapes, M):
                               acc=acc.cpu(), N=N, K=K))
 
         if fmt == "w4a8":
-            kern = "k_tc2<I8,4,256,pair>" if M >= 128 else "k_tc<I8>"
+            kern = f"k_tc2<I8,4,{tc2_tile(M)}>"
         else:
-            kern = "k_gemv_pipe<8,64,M,i8w8>" if M <= 8 and K % 512 == 0 else "k_tc2<W8>"
+            kern = "k_gemv_pipe<8,64,M,i8w8>" if M <= 8 and K % 512 == 0 else \
+                f"k_tc2<W8,8,{'32' if M <= 32 else '128' if M <= 128 else '256,pair'}>"
         works.append(Work(f"{fmt} {N}x{K} M={M}", launch, len(cps), int8_bytes(N, K, M, wbits), 2.0 * M * N * K,
                           kern, [check]))
     return works
@@ -552,7 +558,7 @@ def run_gpu(args, world, rank, local):
     groups = {}
     if full:
         pk = "k_tc2<Affine,4,256,pair,A in TMEM>"
-        groups["prefill_m16"] = affine_work(gwb, dev, "prefill M=16", PREFILL, 16, 4, GS, "k_tc<Affine>")
+        groups["prefill_m16"] = affine_work(gwb, dev, "prefill M=16", PREFILL, 16, 4, GS, "k_tc2<Affine,4,32>")
         groups["prefill_m128"] = affine_work(gwb, dev, "prefill M=128", PREFILL, 128, 4, GS, "k_tc2<Affine,4,128>")
         groups["prefill_m512"] = affine_work(gwb, dev, "prefill M=512", PREFILL, 512, 4, GS, pk)
         groups["prefill_m2048"] = affine_work(gwb, dev, "prefill M=2048", PREFILL, M_PREFILL, 4, GS, pk)
@@ -707,23 +713,28 @@ def run_gpu(args, world, rank, local):
                 k2 = key if M > 128 else key + "_tflops"
                 out[k2] = aggregate(key, t[key], bf16_peak, bf16_src, "TFLOP/s", "tensor",
                                     traffic_key=f"k_tc2_affine4_m{M}")
-        for key in ("prefill_m2048_b8", "prefill_m2048_gs32", "prefill_m2048_gs128"):
-            out[key] = aggregate(key, t[key], bf16_peak, bf16_src, "TFLOP/s", "tensor")
+        for key, tk in (("prefill_m2048_b8", "k_tc2_affine8_m2048"), ("prefill_m2048_gs32", "k_tc2_affine4_gs32_m2048"),
+                        ("prefill_m2048_gs128", "k_tc2_affine4_gs128_m2048")):
+            out[key] = aggregate(key, t[key], bf16_peak, bf16_src, "TFLOP/s", "tensor", traffic_key=tk)
         out["gptq_dequant"] = aggregate("gptq_dequant", t["gptq_dequant"][:1], hbm_peak, hbm_src, "GB/s", "hbm",
                                         traffic_key="k_gptq_dequant",
                                         extra={"permuted_g_idx": aggregate("gptq_dequant", t["gptq_dequant"][1:],
-                                                                           hbm_peak, hbm_src, "GB/s", "hbm")})
+                                                                           hbm_peak, hbm_src, "GB/s", "hbm",
+                                                                           traffic_key="k_gptq_dequant_perm")})
         for M in (1, 32, 1024):
             key = f"gptq_m{M}"
             tm = t[key]
             if M >= 512:
                 out[key] = aggregate(key, tm[:1], bf16_peak, bf16_src + " (fp16 peak taken equal to bf16)",
                                      "TFLOP/s", "tensor", traffic_key="k_tc2_gptq_m1024", extra={"permuted_g_idx": aggregate(
-                                         key, tm[1:], bf16_peak, bf16_src, "TFLOP/s", "tensor")})
+                                         key, tm[1:], bf16_peak, bf16_src, "TFLOP/s", "tensor",
+                                         traffic_key="k_gptq_dequant_tc2_f16_m1024")})
             else:
                 out[key] = aggregate(key, tm[:1], hbm_peak, hbm_src, "GB/s", "hbm",
-                                     traffic_key="k_gemv_gptq_pipe_m1" if M == 1 else None,
-                                     extra={"permuted_g_idx": aggregate(key, tm[1:], hbm_peak, hbm_src, "GB/s", "hbm")})
+                                     traffic_key="k_gemv_gptq_pipe_m1" if M == 1 else "k_tc2_gptq_m32",
+                                     extra={"permuted_g_idx": aggregate(
+                                         key, tm[1:], hbm_peak, hbm_src, "GB/s", "hbm",
+                                         traffic_key="k_gemv_gptq_pipe_perm_m1" if M == 1 else "k_gptq_dequant_tc2_f16_m32")})
         for fmt in ("w4a8", "w8a8"):
             for M in INT8_M:
                 key = f"{fmt}_m{M}"
@@ -731,7 +742,9 @@ def run_gpu(args, world, rank, local):
                     out[key] = aggregate(key, t[key], i8peak, i8src, "TOP/s", "tensor",
                                          traffic_key=f"k_tc2_{fmt}_m{M}")
                 else:
-                    out[key] = aggregate(key, t[key], hbm_peak, hbm_src, "GB/s", "hbm")
+                    out[key] = aggregate(key, t[key], hbm_peak, hbm_src, "GB/s", "hbm",
+                                         traffic_key=f"k_gemv_pipe_i8w8_m{M}" if fmt == "w8a8" and M <= 8
+                                         else f"k_tc2_{fmt}_m{M}")
         out["w8a8_m1"] = aggregate("w8a8_m1", t["w8a8_m1"], hbm_peak, hbm_src, "GB/s", "hbm", traffic_key="k_gemv_pipe_i8w8")
         out["int8_peak_tops"] = round(i8peak, 1)
     out["decode_mlp_fused"] = run_mlp_fused(gwb, dev, stream, hbm_peak, hbm_src)
@@ -835,7 +848,13 @@ def run_mlp_fused(gwb, dev, stream, hbm_peak, hbm_src, bits=4, M=1):
     return {"value": round(gbs, 1), "unit": "GB/s", "M": M, "bits": bits, "group_size": GS,
             "us_per_mlp": round(us, 2), "bytes_per_mlp": nbytes, "launches_per_mlp": 2,
             "roofline": roofline("k_gemv_pipe<dual> + k_gemv_pipe<silu> (Llama-3-8B MLP, hidden 4096)", "hbm", gbs,
-                                 hbm_peak, "GB/s", hbm_src)}
+                                 hbm_peak, "GB/s", hbm_src, traffic=mlp_traffic())}
+
+
+def mlp_traffic():
+    """DRAM bytes of one fused MLP at decode: the gate/up launch plus the silu launch."""
+    a, b = traffic_for("k_gemv_pipe_dual"), traffic_for("k_gemv_pipe_silu")
+    return None if a is None or b is None else a + b
 
 
 # ------------------------------------------------------------------ CPU oracle (reference arm)
@@ -900,13 +919,13 @@ def run_layer(args):
         sets = []
         for s in range(2):
             w = dev_weight(dev, N, K, s)
-            sets.append(gwb.qpack_affine(w, bits, GS))
+            sets.append(gwb.qpack_affine(w, bits, args.gs))
             del w
         x = synth.activations(M, K, seed=1).to(dev)
 
         def launch(i):
             wq, sc, bi = sets[i % 2]
-            gwb.qmm_affine(x, wq, sc, bi, bits, GS, y=y)
+            gwb.qmm_affine(x, wq, sc, bi, bits, args.gs, y=y)
     elif args.fmt in ("gate_up", "silu_resid"):
         sets = []
         for s in range(2):
@@ -927,21 +946,21 @@ def run_layer(args):
                 gwb.gemv_gate_up(x, ws[0], ws[1], bits, GS, y_gate=y, y_up=y2)
             else:
                 gwb.gemv_silu_gate(x, x2, *ws[0], bits, GS, x_resid=res, y=y)
-    elif args.fmt in ("gptq", "gptq_perm", "gptq_dequant"):
-        perm = args.fmt == "gptq_perm"
+    elif args.fmt in ("gptq", "gptq_perm", "gptq_dequant", "gptq_dequant_perm"):
+        perm = args.fmt in ("gptq_perm", "gptq_dequant_perm")
         sets = []
         for s in range(2):
             qw, sc, qz, gi = synth.gptq_quartet(K, N, GPTQ_GS, seed=s, permuted=perm)
             sets.append((qw.to(dev), sc.to(dev), qz.to(dev), gi.to(dev) if perm else None))
         x = synth.activations(M, K, seed=1, dtype=torch.float16).to(dev)
         y = torch.empty((M, N), dtype=torch.float16, device=dev)
-        wo = torch.empty((N, K), dtype=torch.float16, device=dev) if args.fmt == "gptq_dequant" else None
+        wo = torch.empty((N, K), dtype=torch.float16, device=dev) if args.fmt.startswith("gptq_dequant") else None
         bits = 4
 
         def launch(i):
             q, s, z, gi = sets[i % 2]
             if wo is not None:
-                gwb.gptq_dequant(q, s, z, None, GPTQ_GS, out=wo)
+                gwb.gptq_dequant(q, s, z, gi, GPTQ_GS, out=wo)
             else:
                 gwb.gptq_qmm(x, q, s, z, gi, GPTQ_GS, y=y)
     elif args.fmt == "w4a8_fused":
@@ -985,8 +1004,8 @@ def run_layer(args):
         nbytes = 2 * gemv_bytes(N, K, bits, M=M) - 2 * M * K      # x is read once
     elif args.fmt == "silu_resid":
         nbytes = gemv_bytes(N, K, bits, M=M) + 2 * M * K + 2 * M * N   # up and the residual
-    elif args.fmt == "gptq_dequant":
-        nbytes = gptq_dequant_bytes(K, N, GPTQ_GS, False)
+    elif args.fmt.startswith("gptq_dequant"):
+        nbytes = gptq_dequant_bytes(K, N, GPTQ_GS, args.fmt == "gptq_dequant_perm")
     elif args.fmt in ("gptq", "gptq_perm"):
         nbytes = gptq_bytes(K, N, GPTQ_GS, M, args.fmt == "gptq_perm") if M <= 32 else None
     elif args.fmt == "w4a8_fused":
@@ -994,7 +1013,7 @@ def run_layer(args):
     else:
         nbytes = int8_bytes(N, K, M, bits) if M <= 64 else None
     out = {"layer": {"fmt": args.fmt, "N": N, "K": K, "bits": bits,
-                     "group_size": GPTQ_GS if args.fmt.startswith("gptq") else GS, "M": M},
+                     "group_size": GPTQ_GS if args.fmt.startswith("gptq") else args.gs, "M": M},
            "us_per_launch": round(us, 2)}
     if nbytes:
         out["GB/s"] = round(nbytes / us / 1e3, 1)
@@ -1012,7 +1031,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true",
                     help="time the decode sweep (and the fused decode products) only")
     ap.add_argument("--fmt", choices=["affine", "w4a8", "w8a8", "gate_up", "silu_resid", "gptq", "gptq_perm",
-                                      "gptq_dequant", "w4a8_fused"], default="affine",
+                                      "gptq_dequant", "gptq_dequant_perm", "w4a8_fused"], default="affine",
                     help="--layer: weight format (affine: MLX group-wise, bits from --layer; gptq*: N,K = out, in "
                          "features at group size 128)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
@@ -1021,6 +1040,7 @@ def main():
     ap.add_argument("--ref-frac", type=float, default=1 / 16)
     ap.add_argument("--layer", default=None,
                     help="N,K,bits[,M]: time one layer (qmm_affine at group size 64, or --fmt) instead of the sweep")
+    ap.add_argument("--gs", type=int, default=GS, help="--layer with --fmt affine: the group size")
     args = ap.parse_args()
     if args.layer:
         run_layer(args)
