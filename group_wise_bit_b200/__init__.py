@@ -82,8 +82,14 @@ def version() -> str:
     return lib().gwb_version().decode()
 
 
+_fns = {}
+
+
 def _call(name, *args):
-    st = getattr(lib(), name)(*args)
+    fn = _fns.get(name)
+    if fn is None:
+        fn = _fns[name] = getattr(lib(), name)
+    st = fn(*args)
     if st != 0:
         raise GwbError(name, st, lib().gwb_last_error().decode())
 
@@ -105,7 +111,7 @@ def _ptr(t):
 def _dev(t, name, dtypes, shape=None):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda":
+    if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
     if t.dtype not in dtypes:
         raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
