@@ -86,8 +86,6 @@ gwb_status launch_tc_affine(const uint16_t *x, int64_t M, const uint32_t *wq, co
 gwb_status launch_tc_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, const uint16_t *scales,
                           const int32_t *qzeros, const int32_t *g_idx, int64_t K, int64_t N, int gs,
                           uint16_t *y, cudaStream_t st, int zadd = 1);
-gwb_status launch_tc_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
-                          int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st);
 // Persistent tensor-core GEMM (M > 8); GWB_ERR_UNSUPPORTED (without a
 // message) when the layout needs the per-tile kernel (unstaged scales, g_idx).
 gwb_status launch_tc2_affine(const uint16_t *x, int64_t M, const uint32_t *wq, const uint16_t *scales,

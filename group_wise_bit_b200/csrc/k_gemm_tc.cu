@@ -1,7 +1,10 @@
-// Tensor-core (tcgen05) GEMM regime of the fused dequant + matmul, for
-//   * the MLX affine layout (bf16 activations, kind::f16 with bf16 operands),
-//   * the GPTQ layout (fp16 activations, kind::f16 with fp16 operands),
-//   * W4A8 (int8 activations x symmetric int4 weights, kind::i8, s32).
+// Per-tile tensor-core (tcgen05) GEMM of the fused dequant + matmul, for the
+// layouts the persistent kernel (k_gemm_tc2.cu) does not take:
+//   * the MLX affine layout (bf16 activations, kind::f16 with bf16 operands)
+//     with an odd number of groups per row or scale tensors without a common
+//     stride,
+//   * the GPTQ layout (fp16 activations, kind::f16 with fp16 operands) with an
+//     act-order g_idx when no dequant scratch can be had.
 //
 // The problem is computed transposed ("swap AB"): the tensor core's M side is
 // 128 output features (rows of W), its N side is BT tokens.  One CTA owns a
@@ -12,7 +15,7 @@
 //               (raw words) into a ring of STAGES shared-memory stages.
 //   warp 1      TMEM allocation and the single MMA-issuing thread: waits for the
 //               dequantized A tile and the activation tile of a stage, issues
-//               BK/16 (BK/32 for int8) tcgen05.mma into the TMEM accumulator and
+//               BK/16 tcgen05.mma into the TMEM accumulator and
 //               commits the stage back to the producer.
 //   warps 2-9   dequantizers: unpack the stage's raw words in registers, apply
 //               the group scale / bias (or zero), and store the 128 x BK A tile
@@ -41,7 +44,7 @@ constexpr int kDqThreads = 256;
 constexpr int kTileN = 128;  // output features per CTA (tensor-core M)
 constexpr int kMaxSmem = 232448;
 
-enum class Fmt { Affine, Gptq, I8 };
+enum class Fmt { Affine, Gptq };
 
 struct TcArgs {
   int M, N, K, gs;
@@ -49,9 +52,7 @@ struct TcArgs {
   const uint16_t *biases;   // affine: bf16 [N, K/gs]
   const int32_t *qzeros;    // gptq: [K/gs, N/8]
   const int32_t *g_idx;     // gptq: [K] or null
-  const float *sx, *sw;     // i8: per-token / per-channel scales
-  uint16_t *y;              // bf16 (affine, i8) or fp16 (gptq) [M, N]
-  int32_t *acc;             // i8: optional int32 [M, N]
+  uint16_t *y;              // bf16 (affine) or fp16 (gptq) [M, N]
   int staged_scales;        // 1: the producer copies each stage's scales (and zeros) into shared memory
   int zadd;                 // gptq: added to the stored zero (1: GPTQ's convention, 0: AWQ's)
 };
@@ -72,13 +73,6 @@ struct Traits<Fmt::Gptq, 4> {
   static constexpr int NMMA = BK / 16;
   static constexpr int SC_BYTES = 1024;               // 2 groups x (128 fp16 scales + 16 qzeros words)
 };
-template <>
-struct Traits<Fmt::I8, 4> {
-  static constexpr int BK = 128;                      // int8: 128 elements = 128 bytes per row
-  static constexpr int RAW_BYTES = kTileN * BK / 2;
-  static constexpr int NMMA = BK / 32;
-  static constexpr int SC_BYTES = 0;
-};
 
 // ---------------------------------------------------------------- the kernel
 template <Fmt F, int BITS, int BT, int STAGES>
@@ -90,9 +84,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr int A_BYTES = kTileN * 128;
   constexpr int STAGE = B_BYTES + A_BYTES + T::RAW_BYTES + T::SC_BYTES;
   constexpr uint32_t NCOLS = BT < 32 ? 32 : BT;
-  constexpr uint32_t IDESC = (F == Fmt::I8) ? make_idesc(2, 1, kTileN, BT)
-                             : (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN, BT)
-                                                : make_idesc(1, 1, kTileN, BT);
+  constexpr uint32_t IDESC = (F == Fmt::Gptq) ? make_idesc(1, 0, kTileN, BT) : make_idesc(1, 1, kTileN, BT);
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *base = align_smem_1024(smem_raw);
@@ -194,8 +186,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < T::NMMA; kk++) {
           const uint64_t ad = smem_desc_sw128(a0 + kk * 32), bd = smem_desc_sw128(b0 + kk * 32);
-          if constexpr (F == Fmt::I8) umma_i8(tmem, ad, bd, IDESC, (i | kk) != 0);
-          else umma_f16(tmem, ad, bd, IDESC, (i | kk) != 0);
+          umma_f16(tmem, ad, bd, IDESC, (i | kk) != 0);
         }
         umma_commit(&empty[s]);
         done = i + 1;
@@ -312,15 +303,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           *reinterpret_cast<uint4 *>(A + sw128_off(r, kq)) = dq_gptq(w, z2, s2);
         }
-      } else {  // I8
-        const uint4 *rp = reinterpret_cast<const uint4 *>(R + (r * 16 + h * 8) * 4);
-        const uint4 ra = rp[0], rb = rp[1];
-        const uint32_t wv[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-          const uint2 lo = dq_i4(wv[2 * j]), hi = dq_i4(wv[2 * j + 1]);
-          *reinterpret_cast<uint4 *>(A + sw128_off(r, 4 * h + j)) = make_uint4(lo.x, lo.y, hi.x, hi.y);
-        }
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -337,19 +319,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(ch * 16), v);
         tmem_ld_wait();
         if (row < args.N) {
-          float swn = 0.f;
-          if constexpr (F == Fmt::I8) swn = args.sw[row];
 #pragma unroll
           for (int j = 0; j < 16; j++) {
             const int m = m0 + ch * 16 + j;
             if (m < args.M) {
               const int64_t o = (int64_t)m * args.N + row;
-              if constexpr (F == Fmt::I8) {
-                const int a = static_cast<int>(v[j]) >> 4;   // the tensor core summed 16 * code
-                if (args.acc) args.acc[o] = a;
-                if (args.y)
-                  args.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn((float)a * (args.sx[m] * swn)));
-              } else if constexpr (F == Fmt::Gptq) {
+              if constexpr (F == Fmt::Gptq) {
                 args.y[o] = __half_as_ushort(__float2half_rn(__uint_as_float(v[j])));
               } else {
                 args.y[o] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
@@ -474,18 +449,6 @@ gwb_status launch_tc_gptq(const uint16_t *x, int64_t M, const int32_t *qweight, 
                           (uint64_t)N * 4, (uint32_t)kTileN, 8u, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (s != GWB_OK) return s;
   return dispatch_bt<Fmt::Gptq, 4>(M, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, tw, a, st);
-}
-
-gwb_status launch_tc_i8i4(const int8_t *qx, const float *sx, int64_t M, const uint32_t *wq, const float *sw,
-                          int64_t N, int64_t K, uint16_t *y, int32_t *acc, cudaStream_t st) {
-  TcArgs a{};
-  a.M = (int)M; a.N = (int)N; a.K = (int)K; a.gs = 0;
-  a.sx = sx; a.sw = sw; a.y = y; a.acc = acc;
-  CUtensorMap tw;
-  gwb_status s = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, (uint64_t)(K / 8), (uint64_t)N,
-                          (uint64_t)(K / 8) * 4, 16u, (uint32_t)kTileN, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (s != GWB_OK) return s;
-  return dispatch_bt<Fmt::I8, 4>(M, qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, tw, a, st);
 }
 
 }  // namespace gwb

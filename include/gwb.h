@@ -7,13 +7,13 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
  *    never allocates, frees or retains them.  Tensors are dense and row-major
  *    with the shapes stated per call; no strides are taken.
- *  - The one device buffer the library owns is the persistent tensor-core
- *    GEMM's stream-K workspace (partial tiles, up to about 19 MB): one per
- *    (device, stream), allocated by the first call on that stream that runs
- *    that GEMM with split tiles (qmm_affine, gptq_qmm and awq_qmm above 128
- *    tokens, gemm_i8i4 from 128, gemm_i8i8 off its decode path), grown once
- *    if a later call needs more (after synchronizing the stream), and kept
- *    until the process exits.  A call made while its stream is being captured
+ *  - The library owns two kinds of device buffer.  The first is the persistent
+ *    tensor-core GEMM's stream-K workspace (partial tiles, up to about 19 MB):
+ *    one per (device, stream), allocated by the first call on that stream that
+ *    runs that GEMM with split tiles (qmm_affine, gptq_qmm and awq_qmm above 8
+ *    tokens, gemm_i8i4, gemm_i8i8 off its decode path), grown once if a later
+ *    call needs more (after synchronizing the stream), and kept until the
+ *    process exits.  The second is gptq_qmm's act-order scratch (see there).  A call made while its stream is being captured
  *    into a CUDA graph never allocates: it uses the stream's workspace if an
  *    earlier call made one, else it runs without (whole tiles per CTA or pair).
  *    Each launch takes its stream-K epoch from a counter in the workspace, on
