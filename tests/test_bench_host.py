@@ -36,6 +36,34 @@ def test_traffic_entries_resolve():
                 assert os.path.exists(os.path.join(ROOT, "profiles", parts[2])), parts[2]
 
 
+def test_every_traffic_key_the_bench_quotes_resolves():
+    """Every traffic key bench.py passes to a roofline object has a committed ncu figure, so
+    no `traffic` in the bench line is null."""
+    import re
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    keys = set(re.findall(r'traffic_for\("(k_[A-Za-z0-9_]+)"\)', src))
+    keys |= set(re.findall(r'"(k_tc2_affine[0-9a-z_]+)"', src))
+    # every plain key on a line that passes one (f-strings are expanded below)
+    for line in src.splitlines():
+        if "traffic_key=" in line:
+            keys |= set(re.findall(r'(?<![{f])"(k_[A-Za-z0-9_]+)"', line))
+    for M in bench.PREFILL_M:
+        keys.add(f"k_tc2_affine4_m{M}")
+    for fmt in ("w4a8", "w8a8"):
+        for M in bench.INT8_M:
+            keys.add(f"k_gemv_pipe_i8w8_m{M}" if fmt == "w8a8" and M <= 8 else f"k_tc2_{fmt}_m{M}")
+    assert len(keys) > 20, keys
+    missing = sorted(k for k in keys if bench.traffic_for(k) is None)
+    assert not missing, missing
+    # the fused MLP's traffic is the sum of its two launches
+    assert bench.mlp_traffic() == bench.traffic_for("k_gemv_pipe_dual") + bench.traffic_for("k_gemv_pipe_silu")
+
+
+def test_token_tile_labels():
+    assert [bench.tc2_tile(M) for M in (9, 32, 33, 64, 65, 128, 129, 4096)] == \
+        ["32", "32", "64", "64", "128", "128", "256,pair", "256,pair"]
+
+
 def test_job_throughput_scales_with_ranks():
     assert bench.job_gbs(1, 10 ** 9, 1, 1000.0) == 1.0
     assert bench.job_gbs(8, 10 ** 9, 1, 1000.0) == 8.0
